@@ -1,0 +1,176 @@
+/*
+ * attn_oracle.c -- plain fp64 CPU oracle for the scaled-dot-product attention
+ * forward with log-sum-exp output, over varlen batches, grouped-query heads,
+ * an optional paged KV cache and causal / patch masks.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path links, loads or calls
+ * this file; only the tests, the smoke check and the bench's CPU-baseline leg
+ * do.  It shares no code with the CUDA library.
+ *
+ * What it computes (the plain definition, written out without blocking,
+ * fusion or reordering):
+ *   For sequence b, query head h, query i:
+ *     g      = h / (Hq / Hkv)                       grouped-query head sharing
+ *     s_ij   = scale * sum_d q[i,h,d] * k[j,g,d]    explicit score row, all j < Lk_b
+ *     allowed(i,j) by index (none / causal / patch)
+ *     M      = max_{allowed j} s_ij
+ *     p_ij   = exp(s_ij - M) for allowed j, else 0
+ *     O[i,h] = sum_j p_ij v[j,g] / sum_j p_ij
+ *     LSE    = M + ln(sum_j p_ij)                   natural log, scale included
+ *   A row with no allowed key gives O = 0 and LSE = -inf.
+ *
+ * Sources (page title, section):
+ *   - "[FlexAttention] Enforce Q,K,V memory layouts for fp8 flex attention"
+ *     (pytorch commit 7e16cb99), flex_attention docstring: shapes
+ *     (B,Hq,L,E)/(B,Hkv,S,E), default scale 1/sqrt(E), enable_gqa; the causal
+ *     mask_mod q_idx >= kv_idx in the test's expected graph.
+ *   - "Cross Attention does not work on CPU and older GPUs" (BLT issue #6),
+ *     FlexAttention lowering arguments: OUTPUT_LOGSUMEXP, ROWS_GUARANTEED_SAFE
+ *     False (rows may be fully masked), scale 0.0625 for E = 256.
+ *   - "[CUDA] PagedAttention: add SM<80 fp16 fallback via memory-efficient
+ *     attention" (onnxruntime PR 28200), Implementation: block_table walk over
+ *     the paged cache, packed varlen [total_tokens, num_heads, head_size]
+ *     addressed by cumulative sequence lengths, GQA head expansion.
+ *   - "Rope dim" (vllm-project/flash-attention PR 172): seqused_k beside the
+ *     varlen arguments (number of KV tokens used per sequence).
+ *
+ * Readings where the pages are silent (each is listed in the design notes):
+ *   - causal alignment for Lq != Lk is bottom-right: j <= i + (Lk - Lq); it is
+ *     the page's q_idx >= kv_idx when Lq == Lk;
+ *   - the patch predicate is start_i <= j < end_i, sequence-local;
+ *   - paged layout [num_blocks][block_size][Hkv][D], block_table[b][j / bs].
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+enum { ORACLE_MASK_NONE = 0, ORACLE_MASK_CAUSAL = 1, ORACLE_MASK_PATCH = 2 };
+
+/* Row j of head g of sequence b in the K (or V) store. */
+static const double *kv_row(const double *base, int b, int j, int g, int Hkv, int D,
+                            const int32_t *block_table, int max_blocks_per_seq,
+                            int block_size, const int32_t *cu_seqlens_k) {
+    long long row;
+    if (block_table) {
+        int page = block_table[(long long)b * max_blocks_per_seq + j / block_size];
+        row = (long long)page * block_size + (j % block_size);
+    } else {
+        row = (long long)cu_seqlens_k[b] + j;
+    }
+    return base + (row * Hkv + g) * (long long)D;
+}
+
+static int allowed(int mask, int i, int j, int Lq, int Lk, const int32_t *range_i) {
+    switch (mask) {
+    case ORACLE_MASK_NONE: return 1;
+    case ORACLE_MASK_CAUSAL: return j <= i + (Lk - Lq);
+    case ORACLE_MASK_PATCH: return range_i[0] <= j && j < range_i[1];
+    default: return 0;
+    }
+}
+
+/*
+ * q    [total_q][Hq][D]
+ * k, v paged: [num_blocks][block_size][Hkv][D] (block_table != NULL)
+ *      else : [total_k][Hkv][D] addressed by cu_seqlens_k
+ * Lk_b = seqused_k[b] if seqused_k, else cu_seqlens_k[b+1] - cu_seqlens_k[b]
+ * o    [total_q][Hq][D];  lse [Hq][total_q]
+ * Returns 0, or -1 for arguments it cannot interpret.
+ */
+int attn_oracle_fwd(const double *q, const double *k, const double *v,
+                    const int32_t *block_table, int max_blocks_per_seq, int block_size,
+                    const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
+                    const int32_t *seqused_k, int B, int Hq, int Hkv, int D,
+                    double scale, int mask, const int32_t *patch_kv_range,
+                    double *o, double *lse, int total_q, int nthreads) {
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || Hq % Hkv != 0) return -1;
+    if (!seqused_k && !cu_seqlens_k) return -1;
+    if (!block_table && !cu_seqlens_k) return -1;
+    if (mask == ORACLE_MASK_PATCH && !patch_kv_range) return -1;
+    const int group = Hq / Hkv;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+    (void)nthreads;
+#endif
+    int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(|| : bad)
+    for (long long task = 0; task < (long long)B * Hq; ++task) {
+        const int b = (int)(task / Hq), h = (int)(task % Hq);
+        const int g = h / group;
+        const int q0 = cu_seqlens_q[b];
+        const int Lq = cu_seqlens_q[b + 1] - q0;
+        const int Lk = seqused_k ? seqused_k[b] : cu_seqlens_k[b + 1] - cu_seqlens_k[b];
+        double *s = (double *)malloc(sizeof(double) * (size_t)(Lk > 0 ? Lk : 1));
+        if (!s) { bad = 1; continue; }
+        for (int i = 0; i < Lq; ++i) {
+            const double *qi = q + ((long long)(q0 + i) * Hq + h) * D;
+            const int32_t *range_i = patch_kv_range ? patch_kv_range + 2LL * (q0 + i) : NULL;
+            double *oi = o + ((long long)(q0 + i) * Hq + h) * D;
+            double *lse_i = lse + (long long)h * total_q + (q0 + i);
+            /* explicit score row */
+            for (int j = 0; j < Lk; ++j) {
+                const double *kj = kv_row(k, b, j, g, Hkv, D, block_table,
+                                          max_blocks_per_seq, block_size, cu_seqlens_k);
+                double acc = 0.0;
+                for (int d = 0; d < D; ++d) acc += qi[d] * kj[d];
+                s[j] = scale * acc;
+            }
+            /* max over the allowed keys */
+            double M = -INFINITY;
+            int any = 0;
+            for (int j = 0; j < Lk; ++j) {
+                if (!allowed(mask, i, j, Lq, Lk, range_i)) continue;
+                if (!any || s[j] > M) M = s[j];
+                any = 1;
+            }
+            for (int d = 0; d < D; ++d) oi[d] = 0.0;
+            if (!any) { *lse_i = -INFINITY; continue; }
+            /* max-subtracted softmax and the weighted sum of V rows */
+            double Z = 0.0;
+            for (int j = 0; j < Lk; ++j) {
+                if (!allowed(mask, i, j, Lq, Lk, range_i)) continue;
+                const double p = exp(s[j] - M);
+                const double *vj = kv_row(v, b, j, g, Hkv, D, block_table,
+                                          max_blocks_per_seq, block_size, cu_seqlens_k);
+                Z += p;
+                for (int d = 0; d < D; ++d) oi[d] += p * vj[d];
+            }
+            for (int d = 0; d < D; ++d) oi[d] /= Z;
+            *lse_i = M + log(Z);
+        }
+        free(s);
+    }
+    return bad ? -2 : 0;
+}
+
+/*
+ * Merge of partial results over disjoint key ranges (split-KV):
+ *   LSE = ln sum_s exp(LSE_s),   O = sum_s exp(LSE_s - LSE) * O_s
+ * o_parts [S][N][D], lse_parts [S][N] -> o [N][D], lse [N].
+ * Parts with LSE_s = -inf (no keys) contribute nothing; if every part is
+ * empty the result is O = 0, LSE = -inf.
+ */
+void attn_oracle_combine(const double *o_parts, const double *lse_parts, int S, int N,
+                         int D, double *o, double *lse) {
+    for (int n = 0; n < N; ++n) {
+        double M = -INFINITY;
+        for (int s = 0; s < S; ++s)
+            if (lse_parts[(long long)s * N + n] > M) M = lse_parts[(long long)s * N + n];
+        double *on = o + (long long)n * D;
+        for (int d = 0; d < D; ++d) on[d] = 0.0;
+        if (M == -INFINITY) { lse[n] = -INFINITY; continue; }
+        double W = 0.0;
+        for (int s = 0; s < S; ++s) W += exp(lse_parts[(long long)s * N + n] - M);
+        lse[n] = M + log(W);
+        for (int s = 0; s < S; ++s) {
+            const double w = exp(lse_parts[(long long)s * N + n] - lse[n]);
+            const double *os = o_parts + ((long long)s * N + n) * D;
+            for (int d = 0; d < D; ++d) on[d] += w * os[d];
+        }
+    }
+}
