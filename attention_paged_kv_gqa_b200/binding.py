@@ -1,0 +1,191 @@
+"""Python binding of libattn_b200.so (argument marshalling only).
+
+Every function here has the name of the C entry point it calls (declared in
+include/attn_b200.h).  It takes torch tensors, allocates the outputs with torch
+when they are not given, passes raw device pointers, sizes and the current
+CUDA stream, and raises ``AttnError`` on a non-OK status.  All arithmetic
+happens in the CUDA kernels; there is no fallback: if the library is missing
+or the device is not a B200, the call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+from pathlib import Path
+
+import torch
+
+_LIB_PATH = Path(__file__).resolve().parent / "libattn_b200.so"
+_lib = None
+
+MASK_NONE, MASK_CAUSAL, MASK_PATCH = 0, 1, 2
+BF16, FP8_E4M3 = 0, 1
+
+
+class AttnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__("%s: %s (status %d)" % (where, status_string(status), status))
+
+
+def library_path() -> Path:
+    return _LIB_PATH
+
+
+def lib():
+    """Loads the CUDA library (raises if it was not built)."""
+    global _lib
+    if _lib is None:
+        if not _LIB_PATH.exists():
+            raise RuntimeError("libattn_b200.so is not built; run "
+                               "`python -m attention_paged_kv_gqa_b200.build`")
+        L = ctypes.CDLL(str(_LIB_PATH))
+        P, I, F, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+        L.attn_check_device.argtypes = [I]
+        L.attn_check_device.restype = I
+        L.attn_status_string.argtypes = [I]
+        L.attn_status_string.restype = ctypes.c_char_p
+        L.attn_device_error.argtypes = [ctypes.POINTER(I), P]
+        L.attn_device_error.restype = I
+        L.attn_fwd_dense.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P, P, P, F, I, I, P, P, P, P]
+        L.attn_fwd_dense.restype = I
+        L.attn_fwd_varlen_paged.argtypes = [P, P, P, P, I, I, I, P, P, P, I, I, I, I, I, I, I,
+                                            F, I, P, I, P, P, P, P, P, P, Z, P]
+        L.attn_fwd_varlen_paged.restype = I
+        L.attn_decode_workspace_size.argtypes = [I, I, I, I, I, I, I]
+        L.attn_decode_workspace_size.restype = Z
+        L.attn_decode_paged.argtypes = [P, P, P, P, I, I, I, P, I, I, I, I, F, I, I, P, P, P,
+                                        P, P, P, Z, P]
+        L.attn_decode_paged.restype = I
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().attn_status_string(int(status)).decode()
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise AttnError(status, where)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return BF16
+    if t.dtype == torch.float8_e4m3fn:
+        return FP8_E4M3
+    raise TypeError("q/k/v must be bfloat16 or float8_e4m3fn, got %s" % t.dtype)
+
+
+def _scale(scale):
+    return 0.0 if scale is None else float(scale)
+
+
+def _strides3(t: torch.Tensor):
+    if t.stride(-1) != 1:
+        raise ValueError("head_dim must be the contiguous dimension")
+    return (ctypes.c_int64 * 3)(t.stride(0), t.stride(1), t.stride(2))
+
+
+def attn_check_device(device: int = 0) -> int:
+    return lib().attn_check_device(int(device))
+
+
+def attn_device_error(stream=None) -> int:
+    code = ctypes.c_int(0)
+    st = lib().attn_device_error(ctypes.byref(code), _stream(stream))
+    if st not in (0, 7):
+        _check(st, "attn_device_error")
+    return code.value
+
+
+def attn_fwd_dense(q, k, v, *, causal=False, scale=None, descale_q=None, descale_k=None,
+                   descale_v=None, out=None, lse=None, return_lse=True, stream=None):
+    """q [B, Lq, Hq, D], k/v [B, Lk, Hkv, D] -> (o [B, Lq, Hq, D] bf16, lse [B, Hq, Lq] fp32)."""
+    B, Lq, Hq, D = q.shape
+    Lk, Hkv = k.shape[1], k.shape[2]
+    if out is None:
+        out = torch.empty((B, Lq, Hq, D), dtype=torch.bfloat16, device=q.device)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=q.device)
+    st = lib().attn_fwd_dense(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Lq, Lk, Hq, Hkv,
+                              D, _strides3(q), _strides3(k), _strides3(v), _scale(scale),
+                              MASK_CAUSAL if causal else MASK_NONE, _dtype_code(q),
+                              _ptr(descale_q), _ptr(descale_k), _ptr(descale_v), _stream(stream))
+    _check(st, "attn_fwd_dense")
+    return out, lse
+
+
+def attn_fwd_varlen_paged(q, k_cache, v_cache, *, cu_seqlens_q, max_seqlen_q, block_table=None,
+                          cu_seqlens_k=None, seqused_k=None, mask=MASK_NONE, scale=None,
+                          patch_kv_range=None, descale_q=None, descale_k=None, descale_v=None,
+                          out=None, lse=None, return_lse=True, stream=None):
+    """q [total_q, Hq, D]; paged k/v [num_blocks, 16, Hkv, D] (or packed [total_k, Hkv, D]).
+
+    Returns (o [total_q, Hq, D] bf16, lse [Hq, total_q] fp32).
+    """
+    total_q, Hq, D = q.shape
+    B = cu_seqlens_q.numel() - 1
+    if block_table is not None:
+        num_blocks, block_size, Hkv = k_cache.shape[0], k_cache.shape[1], k_cache.shape[2]
+        mbps, total_k = block_table.shape[1], 0
+    else:
+        num_blocks, block_size, mbps = 0, 0, 0
+        total_k, Hkv = k_cache.shape[0], k_cache.shape[1]
+    if out is None:
+        out = torch.empty((total_q, Hq, D), dtype=torch.bfloat16, device=q.device)
+    if lse is None and return_lse:
+        lse = torch.empty((Hq, total_q), dtype=torch.float32, device=q.device)
+    st = lib().attn_fwd_varlen_paged(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), mbps, num_blocks, block_size,
+        _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), _ptr(seqused_k), B, total_q, total_k,
+        int(max_seqlen_q), Hq, Hkv, D, _scale(scale), int(mask), _ptr(patch_kv_range),
+        _dtype_code(q), _ptr(descale_q), _ptr(descale_k), _ptr(descale_v), _ptr(out), _ptr(lse),
+        None, 0, _stream(stream))
+    _check(st, "attn_fwd_varlen_paged")
+    return out, lse
+
+
+def attn_decode_workspace_size(B, num_heads_q, num_heads_kv, head_dim, max_blocks_per_seq,
+                               block_size=16, num_splits=0) -> int:
+    return int(lib().attn_decode_workspace_size(B, num_heads_q, num_heads_kv, head_dim,
+                                                max_blocks_per_seq, block_size, num_splits))
+
+
+def attn_decode_paged(q, k_cache, v_cache, block_table, seqused_k, *, scale=None, num_splits=0,
+                      out=None, lse=None, workspace=None, return_lse=True, stream=None):
+    """q [B, Hq, D] against a paged cache -> (o [B, Hq, D] bf16, lse [B, Hq] fp32)."""
+    B, Hq, D = q.shape
+    num_blocks, block_size, Hkv = k_cache.shape[0], k_cache.shape[1], k_cache.shape[2]
+    mbps = block_table.shape[1]
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=torch.bfloat16, device=q.device)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    ws_bytes = attn_decode_workspace_size(B, Hq, Hkv, D, mbps, block_size, num_splits)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=q.device)
+    st = lib().attn_decode_paged(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), mbps,
+                                 num_blocks, block_size, _ptr(seqused_k), B, Hq, Hkv, D,
+                                 _scale(scale), int(num_splits), _dtype_code(q), None, None, None,
+                                 _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(),
+                                 _stream(stream))
+    _check(st, "attn_decode_paged")
+    return out, lse
+
+
+def default_scale(head_dim: int) -> float:
+    return 1.0 / math.sqrt(head_dim)

@@ -1,0 +1,534 @@
+// attn_api.cu -- the C ABI of libattn_b200.so (declared in include/attn_b200.h):
+// argument validation, the once-per-device architecture check, a cache of TMA
+// descriptors, and the kernel launches on the caller's stream.
+//
+// Nothing here allocates device memory, synchronises the stream or reads
+// device data on the host (the lesson of "[CUDA] PagedAttention: add SM<80
+// fp16 fallback via memory-efficient attention", Scratch allocation: its
+// fallback pays a per-call device-to-host sync to size buffers).  TMA
+// descriptors are encoded once per (pointer, shape, stride, box) and reused,
+// because host-side encoding is not free ("Rope dim", review comment: tens of
+// microseconds of descriptor work per call on H200).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "attn_b200.h"
+#include "decode.cuh"
+#include "prefill.cuh"
+
+using namespace attn;
+
+namespace {
+
+// ------------------------------------------------------------------ device check
+constexpr int kMaxDevices = 64;
+std::atomic<int> g_dev_status[kMaxDevices];   // 0 unknown, 1 ok, else attn_status_t + 100
+
+attn_status_t check_device_uncached(int device) {
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, device) != cudaSuccess) {
+        cudaGetLastError();
+        return ATTN_ERR_CUDA;
+    }
+    if (prop.major != 10 || prop.minor != 0) return ATTN_ERR_NO_KERNEL_IMAGE;
+    int prev = -1;
+    cudaGetDevice(&prev);
+    if (prev != device) cudaSetDevice(device);
+    cudaFuncAttributes fa;
+    const cudaError_t e = cudaFuncGetAttributes(&fa, prefill_kernel<128, false>);
+    if (prev != device && prev >= 0) cudaSetDevice(prev);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return ATTN_ERR_NO_KERNEL_IMAGE;
+    }
+    return ATTN_OK;
+}
+
+attn_status_t current_device_ok(int* dev_out) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return ATTN_ERR_CUDA;
+    }
+    if (dev_out) *dev_out = dev;
+    if (dev < 0 || dev >= kMaxDevices) return check_device_uncached(dev);
+    int s = g_dev_status[dev].load(std::memory_order_acquire);
+    if (s == 0) {
+        const attn_status_t r = check_device_uncached(dev);
+        s = (r == ATTN_OK) ? 1 : 100 + static_cast<int>(r);
+        g_dev_status[dev].store(s, std::memory_order_release);
+    }
+    return s == 1 ? ATTN_OK : static_cast<attn_status_t>(s - 100);
+}
+
+// ------------------------------------------------------------------ TMA descriptors
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encoder() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+        else
+            cudaGetLastError();
+    });
+    return fn;
+}
+
+// A 4-d tiled map: dims {d, head, row, batch} (innermost first), strides in bytes
+// for dims 1..3, box {box_d, 1, box_rows, 1}, 128-byte swizzle, zero fill.
+struct MapKey {
+    const void* ptr;
+    int dtype;
+    int device;
+    uint64_t dims[4];
+    uint64_t strides[3];
+    uint32_t box[4];
+    bool operator==(const MapKey& o) const { return std::memcmp(this, &o, sizeof(MapKey)) == 0; }
+};
+
+struct MapEntry {
+    MapKey key;
+    CUtensorMap map;
+    bool used;
+};
+
+constexpr int kMapCache = 128;
+MapEntry g_maps[kMapCache];
+int g_map_next = 0;
+std::mutex g_map_mu;
+
+attn_status_t get_map(CUtensorMap* out, const void* ptr, int dtype, const uint64_t dims[4],
+                      const uint64_t strides[3], const uint32_t box[4]) {
+    MapKey k;
+    std::memset(&k, 0, sizeof(k));
+    k.ptr = ptr;
+    k.dtype = dtype;
+    cudaGetDevice(&k.device);
+    std::memcpy(k.dims, dims, sizeof(k.dims));
+    std::memcpy(k.strides, strides, sizeof(k.strides));
+    std::memcpy(k.box, box, sizeof(k.box));
+    std::lock_guard<std::mutex> lock(g_map_mu);
+    for (int i = 0; i < kMapCache; ++i)
+        if (g_maps[i].used && g_maps[i].key == k) {
+            *out = g_maps[i].map;
+            return ATTN_OK;
+        }
+    EncodeTiledFn enc = get_encoder();
+    if (!enc) return ATTN_ERR_TMA_ENCODE;
+    CUtensorMap m;
+    const cuuint32_t estride[4] = {1, 1, 1, 1};
+    const CUresult r = enc(&m,
+                           dtype == ATTN_FP8_E4M3 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                                  : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                           4, const_cast<void*>(ptr), reinterpret_cast<const cuuint64_t*>(dims),
+                           reinterpret_cast<const cuuint64_t*>(strides),
+                           reinterpret_cast<const cuuint32_t*>(box), estride,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return ATTN_ERR_TMA_ENCODE;
+    MapEntry& e = g_maps[g_map_next];
+    g_map_next = (g_map_next + 1) % kMapCache;
+    e.key = k;
+    e.map = m;
+    e.used = true;
+    *out = m;
+    return ATTN_OK;
+}
+
+// ------------------------------------------------------------------ validation helpers
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline int elem_bytes(int dtype) { return dtype == ATTN_FP8_E4M3 ? 1 : 2; }
+
+inline bool dtype_ok(int dtype) { return dtype == ATTN_BF16 || dtype == ATTN_FP8_E4M3; }
+
+float resolve_scale(float s, int head_dim) {
+    return (s > 0.0f && std::isfinite(s)) ? s : 1.0f / std::sqrt(static_cast<float>(head_dim));
+}
+
+template <typename K>
+attn_status_t set_smem(K kernel, int bytes) {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+        cudaSuccess) {
+        cudaGetLastError();
+        return ATTN_ERR_CUDA;
+    }
+    return ATTN_OK;
+}
+
+attn_status_t launch_status() {
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------ prefill dispatch
+template <int D, bool FP8>
+attn_status_t launch_prefill_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                               const PrefillArgs& a, long long grid, cudaStream_t stream) {
+    using Cfg = PrefillCfg<D, FP8>;
+    static std::atomic<bool> attr_done{false};
+    if (!attr_done.load()) {
+        const attn_status_t s = set_smem(prefill_kernel<D, FP8>, Cfg::SMEM_BYTES);
+        if (s != ATTN_OK) return s;
+        attr_done.store(true);
+    }
+    prefill_kernel<D, FP8><<<static_cast<unsigned>(grid), kPrefillThreads, Cfg::SMEM_BYTES, stream>>>(
+        mq, mk, mv, a);
+    return launch_status();
+}
+
+attn_status_t launch_prefill(int D, int dtype, const CUtensorMap& mq, const CUtensorMap& mk,
+                             const CUtensorMap& mv, const PrefillArgs& a, long long grid,
+                             cudaStream_t stream) {
+    if (grid <= 0) return ATTN_OK;
+    if (grid >= (1LL << 31)) return ATTN_ERR_UNSUPPORTED;
+    if (dtype == ATTN_BF16 && D == 128) return launch_prefill_t<128, false>(mq, mk, mv, a, grid, stream);
+    if (dtype == ATTN_BF16 && D == 64) return launch_prefill_t<64, false>(mq, mk, mv, a, grid, stream);
+    if (dtype == ATTN_FP8_E4M3 && D == 128) return launch_prefill_t<128, true>(mq, mk, mv, a, grid, stream);
+    return ATTN_ERR_UNSUPPORTED;
+}
+
+void unit_grid(PrefillArgs& a, int max_seqlen_q, long long* grid) {
+    const int nqt = (max_seqlen_q + kBM - 1) / kBM;
+    a.pair_heads = (a.group % 2 == 0) ? 1 : 0;
+    a.NH = a.pair_heads ? a.Hq / 2 : a.Hq;
+    a.NQ = a.pair_heads ? nqt : (nqt + 1) / 2;
+    *grid = static_cast<long long>(a.NQ) * a.B * a.NH;
+}
+
+}  // namespace
+
+// ==================================================================== C ABI
+extern "C" {
+
+const char* attn_status_string(attn_status_t s) {
+    switch (s) {
+    case ATTN_OK: return "ok";
+    case ATTN_ERR_INVALID_ARG: return "invalid argument";
+    case ATTN_ERR_UNSUPPORTED: return "unsupported configuration";
+    case ATTN_ERR_NO_KERNEL_IMAGE: return "device is not sm_100 (B200) or the kernel image does not load";
+    case ATTN_ERR_TMA_ENCODE: return "TMA descriptor encoding failed";
+    case ATTN_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case ATTN_ERR_CUDA: return "CUDA runtime error";
+    case ATTN_ERR_DEVICE_TIMEOUT: return "a kernel gave up on a bounded wait";
+    default: return "unknown status";
+    }
+}
+
+attn_status_t attn_check_device(int device) {
+    int n = 0;
+    if (cudaGetDeviceCount(&n) != cudaSuccess) {
+        cudaGetLastError();
+        return ATTN_ERR_CUDA;
+    }
+    if (device < 0 || device >= n) return ATTN_ERR_INVALID_ARG;
+    return check_device_uncached(device);
+}
+
+attn_status_t attn_device_error(int* code_out, attn_stream_t stream) {
+    if (!code_out) return ATTN_ERR_INVALID_ARG;
+    const attn_status_t dv = current_device_ok(nullptr);
+    if (dv != ATTN_OK) return dv;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int host = 0;
+    const int zero = 0;
+    if (cudaMemcpyFromSymbolAsync(&host, g_device_error, sizeof(int), 0, cudaMemcpyDeviceToHost, st) !=
+            cudaSuccess ||
+        cudaMemcpyToSymbolAsync(g_device_error, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, st) !=
+            cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess) {
+        cudaGetLastError();
+        return ATTN_ERR_CUDA;
+    }
+    *code_out = host;
+    return host == 0 ? ATTN_OK : ATTN_ERR_DEVICE_TIMEOUT;
+}
+
+attn_status_t attn_fwd_dense(const void* q, const void* k, const void* v, void* o, float* lse,
+                             int B, int Lq, int Lk, int Hq, int Hkv, int D,
+                             const int64_t* sq, const int64_t* sk, const int64_t* sv,
+                             float softmax_scale, int mask, int dtype, const float* dq,
+                             const float* dk, const float* dv, attn_stream_t stream) {
+    if (!q || !k || !v || !o || !sq || !sk || !sv) return ATTN_ERR_INVALID_ARG;
+    if (B < 0 || Lq < 0 || Lk < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
+    if (!dtype_ok(dtype)) return ATTN_ERR_INVALID_ARG;
+    if (mask != ATTN_MASK_NONE && mask != ATTN_MASK_CAUSAL) {
+        return mask == ATTN_MASK_PATCH ? ATTN_ERR_UNSUPPORTED : ATTN_ERR_INVALID_ARG;
+    }
+    if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+    if (dtype == ATTN_FP8_E4M3 && (D != 128)) return ATTN_ERR_UNSUPPORTED;
+    if (dtype == ATTN_FP8_E4M3 && (!dq || !dk || !dv)) return ATTN_ERR_INVALID_ARG;
+    const int E = elem_bytes(dtype);
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return ATTN_ERR_INVALID_ARG;
+    for (int i = 0; i < 3; ++i) {
+        if (sq[i] <= 0 || sk[i] <= 0 || sv[i] <= 0) return ATTN_ERR_INVALID_ARG;
+        if ((sq[i] * E) % 16 || (sk[i] * E) % 16 || (sv[i] * E) % 16) return ATTN_ERR_INVALID_ARG;
+    }
+    if (sq[2] < D || sk[2] < D || sv[2] < D) return ATTN_ERR_INVALID_ARG;
+    if (Lq > (1 << 30) || Lk > (1 << 30)) return ATTN_ERR_UNSUPPORTED;
+    const attn_status_t dvs = current_device_ok(nullptr);
+    if (dvs != ATTN_OK) return dvs;
+    if (B == 0 || Lq == 0) return ATTN_OK;
+
+    const int chunk = 128 / E;
+    CUtensorMap mq, mk, mv;
+    const uint64_t dq4[4] = {(uint64_t)D, (uint64_t)Hq, (uint64_t)Lq, (uint64_t)B};
+    const uint64_t sq3[3] = {(uint64_t)(sq[2] * E), (uint64_t)(sq[1] * E), (uint64_t)(sq[0] * E)};
+    const uint32_t bq[4] = {(uint32_t)chunk, 1, (uint32_t)kBM, 1};
+    const uint64_t dk4[4] = {(uint64_t)D, (uint64_t)Hkv, (uint64_t)std::max(Lk, 1), (uint64_t)B};
+    const uint64_t sk3[3] = {(uint64_t)(sk[2] * E), (uint64_t)(sk[1] * E), (uint64_t)(sk[0] * E)};
+    const uint64_t sv3[3] = {(uint64_t)(sv[2] * E), (uint64_t)(sv[1] * E), (uint64_t)(sv[0] * E)};
+    const uint32_t bkv[4] = {(uint32_t)chunk, 1, (uint32_t)kBN, 1};
+    attn_status_t s;
+    if ((s = get_map(&mq, q, dtype, dq4, sq3, bq)) != ATTN_OK) return s;
+    if ((s = get_map(&mk, k, dtype, dk4, sk3, bkv)) != ATTN_OK) return s;
+    if ((s = get_map(&mv, v, dtype, dk4, sv3, bkv)) != ATTN_OK) return s;
+
+    PrefillArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.B = B;
+    a.Hq = Hq;
+    a.Hkv = Hkv;
+    a.group = Hq / Hkv;
+    a.mask = mask;
+    a.varlen = 0;
+    a.paged = 0;
+    a.Lq = Lq;
+    a.Lk = Lk;
+    a.scale = resolve_scale(softmax_scale, D);
+    a.descale_q = dq;
+    a.descale_k = dk;
+    a.descale_v = dv;
+    a.o = static_cast<__nv_bfloat16*>(o);
+    a.lse = lse;
+    a.o_stride_row = (long long)Hq * D;
+    a.o_stride_b = (long long)Lq * Hq * D;
+    a.lse_stride_h = Lq;
+    a.lse_stride_b = (long long)Hq * Lq;
+    long long grid;
+    unit_grid(a, Lq, &grid);
+    return launch_prefill(D, dtype, mq, mk, mv, a, grid, static_cast<cudaStream_t>(stream));
+}
+
+attn_status_t attn_fwd_varlen_paged(
+    const void* q, const void* k_cache, const void* v_cache, const int32_t* block_table,
+    int max_blocks_per_seq, int num_blocks, int block_size, const int32_t* cu_seqlens_q,
+    const int32_t* cu_seqlens_k, const int32_t* seqused_k, int B, int total_q, int total_k,
+    int max_seqlen_q, int Hq, int Hkv, int D, float softmax_scale, int mask,
+    const int32_t* patch_kv_range, int dtype, const float* dq, const float* dk, const float* dv,
+    void* o, float* lse, void* workspace, size_t workspace_bytes, attn_stream_t stream) {
+    (void)workspace;
+    (void)workspace_bytes;
+    if (!q || !k_cache || !v_cache || !o || !cu_seqlens_q) return ATTN_ERR_INVALID_ARG;
+    if (B < 0 || total_q < 0 || max_seqlen_q < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0)
+        return ATTN_ERR_INVALID_ARG;
+    if (!dtype_ok(dtype)) return ATTN_ERR_INVALID_ARG;
+    if (mask < ATTN_MASK_NONE || mask > ATTN_MASK_PATCH) return ATTN_ERR_INVALID_ARG;
+    if (mask == ATTN_MASK_PATCH && !patch_kv_range) return ATTN_ERR_INVALID_ARG;
+    if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+    if (dtype == ATTN_FP8_E4M3 && D != 128) return ATTN_ERR_UNSUPPORTED;
+    if (dtype == ATTN_FP8_E4M3 && (!dq || !dk || !dv)) return ATTN_ERR_INVALID_ARG;
+    const bool paged = block_table != nullptr;
+    if (paged) {
+        if (block_size != kPageRows) return ATTN_ERR_UNSUPPORTED;
+        if (num_blocks <= 0 || max_blocks_per_seq <= 0) return ATTN_ERR_INVALID_ARG;
+        if ((long long)num_blocks * block_size >= (1LL << 31)) return ATTN_ERR_UNSUPPORTED;
+        if (!seqused_k && !cu_seqlens_k) return ATTN_ERR_INVALID_ARG;
+    } else {
+        if (!cu_seqlens_k || total_k < 0) return ATTN_ERR_INVALID_ARG;
+    }
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o))
+        return ATTN_ERR_INVALID_ARG;
+    const int E = elem_bytes(dtype);
+    if ((D * E) % 16) return ATTN_ERR_INVALID_ARG;
+    const attn_status_t dvs = current_device_ok(nullptr);
+    if (dvs != ATTN_OK) return dvs;
+    if (B == 0 || total_q == 0 || max_seqlen_q == 0) return ATTN_OK;
+
+    const int chunk = 128 / E;
+    CUtensorMap mq, mk, mv;
+    const uint64_t rowq = (uint64_t)Hq * D * E;
+    const uint64_t dq4[4] = {(uint64_t)D, (uint64_t)Hq, (uint64_t)total_q, 1};
+    const uint64_t sq3[3] = {(uint64_t)D * E, rowq, rowq * (uint64_t)total_q};
+    const uint32_t bq[4] = {(uint32_t)chunk, 1, (uint32_t)kBM, 1};
+    const uint64_t rowk = (uint64_t)Hkv * D * E;
+    const uint64_t nrows = paged ? (uint64_t)num_blocks * block_size : (uint64_t)std::max(total_k, 1);
+    const uint64_t dk4[4] = {(uint64_t)D, (uint64_t)Hkv, nrows, 1};
+    const uint64_t sk3[3] = {(uint64_t)D * E, rowk, rowk * nrows};
+    const uint32_t bkv[4] = {(uint32_t)chunk, 1, (uint32_t)(paged ? kPageRows : kBN), 1};
+    attn_status_t s;
+    if ((s = get_map(&mq, q, dtype, dq4, sq3, bq)) != ATTN_OK) return s;
+    if ((s = get_map(&mk, k_cache, dtype, dk4, sk3, bkv)) != ATTN_OK) return s;
+    if ((s = get_map(&mv, v_cache, dtype, dk4, sk3, bkv)) != ATTN_OK) return s;
+
+    PrefillArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.B = B;
+    a.Hq = Hq;
+    a.Hkv = Hkv;
+    a.group = Hq / Hkv;
+    a.mask = mask;
+    a.varlen = 1;
+    a.paged = paged ? 1 : 0;
+    a.cu_q = cu_seqlens_q;
+    a.cu_k = cu_seqlens_k;
+    a.seqused_k = seqused_k;
+    a.block_table = block_table;
+    a.max_blocks = max_blocks_per_seq;
+    a.patch = patch_kv_range;
+    a.scale = resolve_scale(softmax_scale, D);
+    a.descale_q = dq;
+    a.descale_k = dk;
+    a.descale_v = dv;
+    a.o = static_cast<__nv_bfloat16*>(o);
+    a.lse = lse;
+    a.o_stride_row = (long long)Hq * D;
+    a.o_stride_b = 0;
+    a.lse_stride_h = total_q;
+    a.lse_stride_b = 0;
+    long long grid;
+    unit_grid(a, max_seqlen_q, &grid);
+    return launch_prefill(D, dtype, mq, mk, mv, a, grid, static_cast<cudaStream_t>(stream));
+}
+
+// Split-KV heuristic: enough CTAs to fill every SM about twice with sequences
+// of the maximum length, and at most ~512 keys per split for balance across
+// ragged lengths; tokens per split is a multiple of the 64-key stage.
+static void decode_splits(int B, int Hkv, int max_tokens, int requested, int* num_splits,
+                          int* tps) {
+    max_tokens = std::max(max_tokens, 1);
+    int ns;
+    if (requested > 0) {
+        ns = requested;
+    } else {
+        const int for_balance = (max_tokens + 511) / 512;
+        const int for_fill = (2 * 148 * 2 + B * Hkv - 1) / std::max(B * Hkv, 1);
+        ns = std::max(for_balance, for_fill);
+    }
+    ns = std::max(1, std::min(ns, (max_tokens + kDecStageTok - 1) / kDecStageTok));
+    int t = (max_tokens + ns - 1) / ns;
+    t = (t + kDecStageTok - 1) / kDecStageTok * kDecStageTok;
+    *tps = t;
+    *num_splits = (max_tokens + t - 1) / t;
+}
+
+size_t attn_decode_workspace_size(int B, int Hq, int Hkv, int D, int max_blocks_per_seq,
+                                  int block_size, int num_splits) {
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || max_blocks_per_seq <= 0 || block_size <= 0)
+        return 0;
+    int ns, tps;
+    decode_splits(B, Hkv, max_blocks_per_seq * block_size, num_splits, &ns, &tps);
+    if (ns <= 1) return 16;
+    return (size_t)ns * B * Hq * (D + 1) * sizeof(float) + 16;
+}
+
+attn_status_t attn_decode_paged(const void* q, const void* k_cache, const void* v_cache,
+                                const int32_t* block_table, int max_blocks_per_seq, int num_blocks,
+                                int block_size, const int32_t* seqused_k, int B, int Hq, int Hkv,
+                                int D, float softmax_scale, int num_splits, int dtype,
+                                const float* dq, const float* dk, const float* dv, void* o,
+                                float* lse, void* workspace, size_t workspace_bytes,
+                                attn_stream_t stream) {
+    (void)dq;
+    (void)dk;
+    (void)dv;
+    if (!q || !k_cache || !v_cache || !block_table || !seqused_k || !o) return ATTN_ERR_INVALID_ARG;
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
+    if (num_blocks <= 0 || max_blocks_per_seq <= 0) return ATTN_ERR_INVALID_ARG;
+    if (!dtype_ok(dtype)) return ATTN_ERR_INVALID_ARG;
+    if (dtype != ATTN_BF16) return ATTN_ERR_UNSUPPORTED;
+    if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+    if (block_size != kPageRows) return ATTN_ERR_UNSUPPORTED;
+    if (Hq / Hkv > kDecRows) return ATTN_ERR_UNSUPPORTED;
+    if ((long long)num_blocks * block_size >= (1LL << 31)) return ATTN_ERR_UNSUPPORTED;
+    if ((long long)max_blocks_per_seq * block_size >= (1LL << 30)) return ATTN_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o))
+        return ATTN_ERR_INVALID_ARG;
+    int ns, tps;
+    decode_splits(B, Hkv, max_blocks_per_seq * block_size, num_splits, &ns, &tps);
+    const size_t need = attn_decode_workspace_size(B, Hq, Hkv, D, max_blocks_per_seq, block_size,
+                                                   num_splits);
+    if (ns > 1) {
+        if (!workspace || !aligned16(workspace)) return ATTN_ERR_INVALID_ARG;
+        if (workspace_bytes < need) return ATTN_ERR_WORKSPACE_TOO_SMALL;
+    }
+    const attn_status_t dvs = current_device_ok(nullptr);
+    if (dvs != ATTN_OK) return dvs;
+    if (B == 0) return ATTN_OK;
+
+    CUtensorMap mk, mv;
+    const uint64_t rowk = (uint64_t)Hkv * D * 2;
+    const uint64_t nrows = (uint64_t)num_blocks * block_size;
+    const uint64_t dk4[4] = {(uint64_t)D, (uint64_t)Hkv, nrows, 1};
+    const uint64_t sk3[3] = {(uint64_t)D * 2, rowk, rowk * nrows};
+    const uint32_t bkv[4] = {64, 1, (uint32_t)kPageRows, 1};
+    attn_status_t s;
+    if ((s = get_map(&mk, k_cache, ATTN_BF16, dk4, sk3, bkv)) != ATTN_OK) return s;
+    if ((s = get_map(&mv, v_cache, ATTN_BF16, dk4, sk3, bkv)) != ATTN_OK) return s;
+
+    DecodeArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.B = B;
+    a.Hq = Hq;
+    a.Hkv = Hkv;
+    a.group = Hq / Hkv;
+    a.q = static_cast<const __nv_bfloat16*>(q);
+    a.block_table = block_table;
+    a.max_blocks = max_blocks_per_seq;
+    a.seqused_k = seqused_k;
+    a.tokens_per_split = tps;
+    a.num_splits = ns;
+    a.scale = resolve_scale(softmax_scale, D);
+    a.o = static_cast<__nv_bfloat16*>(o);
+    a.lse = lse;
+    a.direct = ns == 1 ? 1 : 0;
+    if (ns > 1) {
+        a.o_part = static_cast<float*>(workspace);
+        a.lse_part = a.o_part + (size_t)ns * B * Hq * D;
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const dim3 grid(ns, Hkv, B);
+    if (D == 128) {
+        static std::atomic<bool> done{false};
+        if (!done.load()) {
+            if ((s = set_smem(decode_split_kernel<128>, DecodeCfg<128>::SMEM_BYTES)) != ATTN_OK) return s;
+            done.store(true);
+        }
+        decode_split_kernel<128><<<grid, kDecThreads, DecodeCfg<128>::SMEM_BYTES, st>>>(mk, mv, a);
+        if ((s = launch_status()) != ATTN_OK) return s;
+        if (ns > 1)
+            decode_combine_kernel<128><<<B * Hq, 128, 0, st>>>(a.o_part, a.lse_part, seqused_k, B, Hq,
+                                                                ns, tps, max_blocks_per_seq * block_size,
+                                                                a.o, lse);
+    } else {
+        static std::atomic<bool> done{false};
+        if (!done.load()) {
+            if ((s = set_smem(decode_split_kernel<64>, DecodeCfg<64>::SMEM_BYTES)) != ATTN_OK) return s;
+            done.store(true);
+        }
+        decode_split_kernel<64><<<grid, kDecThreads, DecodeCfg<64>::SMEM_BYTES, st>>>(mk, mv, a);
+        if ((s = launch_status()) != ATTN_OK) return s;
+        if (ns > 1)
+            decode_combine_kernel<64><<<B * Hq, 64, 0, st>>>(a.o_part, a.lse_part, seqused_k, B, Hq,
+                                                              ns, tps, max_blocks_per_seq * block_size,
+                                                              a.o, lse);
+    }
+    return launch_status();
+}
+
+}  // extern "C"

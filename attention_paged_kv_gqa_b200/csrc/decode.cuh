@@ -1,0 +1,352 @@
+// decode.cuh -- paged GQA decode on sm_100a: one query token per sequence,
+// key range split across CTAs (split-KV), then an LSE-weighted combine.
+//
+// The work is HBM-bound (about 4 flop per byte of K/V at group size 4), so the
+// kernel is built around the memory path: a producer warp fetches each 16-token
+// page of K and V straight from the paged cache through block_table with TMA
+// (128-byte swizzle, no gather pass), several stages deep; four consumer warps
+// each own 16 keys of a 64-key stage and keep their own online-softmax state,
+// merged once at the end.  The tiny per-stage contractions (G query heads x 16
+// keys x D) run on the warp-level tensor-core MMA, which keeps the consumer
+// warps far from being the bottleneck.
+//
+// The partial results of a split are (O_s normalised, LSE_s) in fp32; the
+// combine kernel merges them as LSE = ln sum_s exp(LSE_s),
+// O = sum_s exp(LSE_s - LSE) O_s.  Paging and the packed-free page walk follow
+// "[CUDA] PagedAttention: add SM<80 fp16 fallback via memory-efficient
+// attention" (Implementation; the fp32 accumulator buffer idea); seqused_k
+// follows "Rope dim" (the varlen arguments).
+#pragma once
+
+#include "prefill.cuh"
+
+namespace attn {
+
+constexpr int kDecThreads = 160;      // warps 0-3 consumers, warp 4 producer
+constexpr int kDecStageTok = 64;      // keys per stage (4 pages)
+constexpr int kDecRows = 16;          // MMA rows = query heads of one KV group (padded)
+
+struct DecodeArgs {
+    int B, Hq, Hkv, group;
+    const __nv_bfloat16* q;   // [B][Hq][D]
+    const int* block_table;
+    int max_blocks;
+    const int* seqused_k;
+    int tokens_per_split;     // multiple of kDecStageTok
+    int num_splits;
+    float scale;
+    float* o_part;            // [splits][B][Hq][D]
+    float* lse_part;          // [splits][B][Hq]
+    __nv_bfloat16* o;         // [B][Hq][D]  (direct mode)
+    float* lse;               // [B][Hq]     (direct mode, nullable)
+    int direct;               // 1: single split, write the final result
+};
+
+template <int D>
+struct DecodeCfg {
+    static constexpr int ROWB = D * 2;
+    static constexpr int NCHUNK = ROWB / 128;
+    static constexpr int STAGE_K = kDecStageTok * ROWB;
+    static constexpr int STAGE = 2 * STAGE_K;              // K then V
+    static constexpr int NS = (D == 128) ? 3 : 6;
+    static constexpr int MERGE_BYTES = 4 * kDecRows * (D + 2) * 4;
+    static constexpr int BODY = (NS * STAGE > MERGE_BYTES) ? NS * STAGE : MERGE_BYTES;
+    static constexpr int SMEM_BYTES = 1024 + BODY + 256;
+};
+
+// Byte offset of element (row, col) of a [rows][D] bf16 tile stored as
+// 128-byte swizzled columns of `rows` rows each (the TMA SWIZZLE_128B layout).
+template <int D>
+__device__ __forceinline__ uint32_t swz_off(int row, int col, int rows) {
+    const int c = col >> 6;               // 64 bf16 per 128-byte column
+    const int piece = (col & 63) >> 3;    // 16-byte piece
+    return c * rows * 128 + row * 128 + ((piece ^ (row & 7)) << 4) + ((col & 7) << 1);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kDecThreads, 2)
+    decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                        const DecodeArgs a) {
+    using C = DecodeCfg<D>;
+    constexpr int NS = C::NS;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = align1024(smem_raw);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::BODY);
+    uint64_t* empty = full + NS;
+
+    const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int L = min(max(a.seqused_k[b], 0), a.max_blocks * kPageRows);
+    const int t_begin = split * a.tokens_per_split;
+    const int t_end = min(L, t_begin + a.tokens_per_split);
+    if (t_begin >= t_end && !(a.direct && split == 0)) return;   // empty split: combine skips it
+    const int nstage = (t_end > t_begin) ? (t_end - t_begin + kDecStageTok - 1) / kDecStageTok : 0;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < NS; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], 4);
+        }
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    if (warp == 4) {
+        // ---------------------------------------------------- producer: page gather (a3)
+        if (lane == 0) {
+            prefetch_tmap(&tmK);
+            prefetch_tmap(&tmV);
+        }
+        const uint64_t pol = policy_evict_first();
+        const int slot0 = t_begin / kPageRows;
+        int window = -1;      // index of the 32-slot window held in `pg`
+        int pg = 0;
+        int issued = 0;
+        for (int s = 0; s < nstage; ++s, ++issued) {
+            const int st = s % NS;
+            const uint32_t ph = (s / NS) & 1;
+            const int sbase = slot0 + s * (kDecStageTok / kPageRows);
+            const int w = (sbase - slot0) / 32;
+            if (w != window) {
+                window = w;
+                const int slot = slot0 + w * 32 + lane;
+                pg = (slot * kPageRows < t_end && slot < a.max_blocks)
+                         ? a.block_table[(long long)b * a.max_blocks + slot] : 0;
+            }
+            int pages[4];
+#pragma unroll
+            for (int p = 0; p < 4; ++p) pages[p] = __shfl_sync(0xffffffffu, pg, (sbase - slot0) % 32 + p);
+            bool ok = mbar_wait(&empty[st], ph ^ 1, kErrDecEmpty);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+            if (lane == 0) {
+                int npv = 0;
+#pragma unroll
+                for (int p = 0; p < 4; ++p) npv += ((sbase + p) * kPageRows < t_end) ? 1 : 0;
+                mbar_arrive_expect_tx(&full[st], 2 * npv * kPageRows * C::ROWB);
+                uint8_t* dk = smem + st * C::STAGE;
+                uint8_t* dv = dk + C::STAGE_K;
+#pragma unroll
+                for (int p = 0; p < 4; ++p) {
+                    if ((sbase + p) * kPageRows >= t_end) continue;
+#pragma unroll
+                    for (int c = 0; c < C::NCHUNK; ++c) {
+                        const int off = c * kDecStageTok * 128 + p * kPageRows * 128;
+                        tma_load_4d_hint(&tmK, &full[st], dk + off, c * 64, g, pages[p] * kPageRows, 0, pol);
+                        tma_load_4d_hint(&tmV, &full[st], dv + off, c * 64, g, pages[p] * kPageRows, 0, pol);
+                    }
+                }
+            }
+        }
+        if (lane == 0) {
+            for (int st = 0; st < NS && st < issued; ++st) {
+                const int last = st + ((issued - 1 - st) / NS) * NS;
+                mbar_wait(&full[st], (last / NS) & 1, kErrDecFull);
+            }
+        }
+    } else {
+        // ---------------------------------------------------- consumers (a4-a6 for one token)
+        const int gid = lane >> 2, t4 = lane & 3;
+        const float sl2 = a.scale * kLog2e;
+        // Q fragments (rows = the G query heads of KV head g; rows >= G are zero).
+        uint32_t qa[D / 16][4];
+        {
+            const __nv_bfloat16* qb = a.q + ((long long)b * a.Hq + (long long)g * a.group) * D;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const int c0 = kk * 16 + 2 * t4;
+                auto ld = [&](int row, int col) -> uint32_t {
+                    if (row >= a.group) return 0u;
+                    return *reinterpret_cast<const uint32_t*>(qb + (long long)row * D + col);
+                };
+                qa[kk][0] = ld(gid, c0);
+                qa[kk][1] = ld(gid + 8, c0);
+                qa[kk][2] = ld(gid, c0 + 8);
+                qa[kk][3] = ld(gid + 8, c0 + 8);
+            }
+        }
+        float o[D / 8][4];
+#pragma unroll
+        for (int i = 0; i < D / 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.0f;
+        float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.0f, l1 = 0.0f;   // rows gid, gid+8
+        bool ok = true;
+        for (int s = 0; s < nstage; ++s) {
+            const int st = s % NS;
+            ok = mbar_wait(&full[st], (s / NS) & 1, kErrDecFull);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+            const int tok0 = t_begin + s * kDecStageTok + warp * 16;   // this warp's 16 keys
+            uint8_t* sk = smem + st * C::STAGE;
+            uint8_t* sv = sk + C::STAGE_K;
+            const int lrow0 = warp * 16;                                  // row within the stage
+            if (tok0 < t_end) {
+                if (tok0 + 16 > t_end) {
+                    // Zero the V rows past the end of the sequence (not data of it).
+                    for (int i = lane; i < 16 * (D / 8); i += 32) {
+                        const int rr = i / (D / 8), cc = (i % (D / 8)) * 8;
+                        if (tok0 + rr >= t_end)
+                            *reinterpret_cast<uint4*>(sv + swz_off<D>(lrow0 + rr, cc, kDecStageTok)) =
+                                make_uint4(0, 0, 0, 0);
+                    }
+                    __syncwarp();
+                }
+                // S = Q K^T for 16 keys: two n-tiles of 8 keys.
+                float sc[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}};
+                const uint32_t skb = smem_u32(sk);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const int mi = lane >> 3, ri = lane & 7;
+                    const int row = lrow0 + (mi >> 1) * 8 + ri;
+                    const int col = kk * 16 + (mi & 1) * 8;
+                    uint32_t b0, b1, b2, b3;
+                    ldmatrix_x4(skb + swz_off<D>(row, col, kDecStageTok), b0, b1, b2, b3);
+                    mma_bf16_16816(sc[0], qa[kk], b0, b1);
+                    mma_bf16_16816(sc[1], qa[kk], b2, b3);
+                }
+                // mask keys past the end, online softmax per row
+                float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const int kv = tok0 + nt * 8 + 2 * t4 + e;
+                        if (kv >= t_end) { sc[nt][e] = -INFINITY; sc[nt][2 + e] = -INFINITY; }
+                        mx0 = fmaxf(mx0, sc[nt][e]);
+                        mx1 = fmaxf(mx1, sc[nt][2 + e]);
+                    }
+                mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+                mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+                mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+                mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+                const float mn0 = fmaxf(m0, mx0 * sl2), mn1 = fmaxf(m1, mx1 * sl2);
+                // m = -inf (nothing seen yet) -> alpha 0; both -inf -> 1 (avoid -inf - -inf)
+                const float al0 = (mn0 == -INFINITY) ? 1.0f : ex2(m0 - mn0);
+                const float al1 = (mn1 == -INFINITY) ? 1.0f : ex2(m1 - mn1);
+                m0 = mn0;
+                m1 = mn1;
+                l0 *= al0;
+                l1 *= al1;
+#pragma unroll
+                for (int i = 0; i < D / 8; ++i) {
+                    o[i][0] *= al0;
+                    o[i][1] *= al0;
+                    o[i][2] *= al1;
+                    o[i][3] *= al1;
+                }
+                const float mu0 = (m0 == -INFINITY) ? 0.0f : m0;
+                const float mu1 = (m1 == -INFINITY) ? 0.0f : m1;
+                float p[2][4];
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt) {
+                    p[nt][0] = ex2(fmaf(sc[nt][0], sl2, -mu0));
+                    p[nt][1] = ex2(fmaf(sc[nt][1], sl2, -mu0));
+                    p[nt][2] = ex2(fmaf(sc[nt][2], sl2, -mu1));
+                    p[nt][3] = ex2(fmaf(sc[nt][3], sl2, -mu1));
+                    l0 += p[nt][0] + p[nt][1];
+                    l1 += p[nt][2] + p[nt][3];
+                }
+                uint32_t pa[4];
+                pa[0] = pack_bf16(p[0][0], p[0][1]);
+                pa[1] = pack_bf16(p[0][2], p[0][3]);
+                pa[2] = pack_bf16(p[1][0], p[1][1]);
+                pa[3] = pack_bf16(p[1][2], p[1][3]);
+                // O += P V over the 16 keys
+                const uint32_t svb = smem_u32(sv);
+#pragma unroll
+                for (int nd = 0; nd < D / 8; nd += 2) {
+                    const int mi = lane >> 3, ri = lane & 7;
+                    const int row = lrow0 + (mi & 1) * 8 + ri;
+                    const int col = nd * 8 + (mi >> 1) * 8;
+                    uint32_t b0, b1, b2, b3;
+                    ldmatrix_x4_trans(svb + swz_off<D>(row, col, kDecStageTok), b0, b1, b2, b3);
+                    mma_bf16_16816(o[nd], pa, b0, b1);
+                    mma_bf16_16816(o[nd + 1], pa, b2, b3);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[st]);
+        }
+        // row sums: reduce over the quad
+        l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+        l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+        l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+        l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+
+        // ---------------------------------------------------- merge the 4 warps
+        asm volatile("bar.sync 1, 128;" ::: "memory");   // all consumers done with the stages
+        float* mo = reinterpret_cast<float*>(smem);                 // [4][16][D]
+        float* mm = mo + 4 * kDecRows * D;                          // [4][16]
+        float* ml = mm + 4 * kDecRows;                              // [4][16]
+#pragma unroll
+        for (int i = 0; i < D / 8; ++i) {
+            const int col = i * 8 + 2 * t4;
+            mo[(warp * kDecRows + gid) * D + col] = o[i][0];
+            mo[(warp * kDecRows + gid) * D + col + 1] = o[i][1];
+            mo[(warp * kDecRows + gid + 8) * D + col] = o[i][2];
+            mo[(warp * kDecRows + gid + 8) * D + col + 1] = o[i][3];
+        }
+        if (t4 == 0) {
+            mm[warp * kDecRows + gid] = m0;
+            mm[warp * kDecRows + gid + 8] = m1;
+            ml[warp * kDecRows + gid] = l0;
+            ml[warp * kDecRows + gid + 8] = l1;
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        const int G = a.group;
+        for (int idx = threadIdx.x; idx < G * D; idx += 128) {
+            const int row = idx / D, col = idx % D;
+            float M = -INFINITY;
+#pragma unroll
+            for (int w = 0; w < 4; ++w) M = fmaxf(M, mm[w * kDecRows + row]);
+            float acc = 0.0f, l = 0.0f;
+            if (M != -INFINITY) {
+#pragma unroll
+                for (int w = 0; w < 4; ++w) {
+                    const float f = ex2(mm[w * kDecRows + row] - M);
+                    acc += f * mo[(w * kDecRows + row) * D + col];
+                    l += f * ml[w * kDecRows + row];
+                }
+            }
+            const int h = g * G + row;
+            const float on = (l > 0.0f) ? acc / l : 0.0f;
+            const float lse = (l > 0.0f) ? (M + log2f(l)) * kLn2 : -INFINITY;
+            if (a.direct) {
+                a.o[((long long)b * a.Hq + h) * D + col] = __float2bfloat16_rn(on);
+                if (col == 0 && a.lse) a.lse[(long long)b * a.Hq + h] = lse;
+            } else {
+                const long long base = ((long long)split * a.B + b) * a.Hq + h;
+                a.o_part[base * D + col] = on;
+                if (col == 0) a.lse_part[base] = lse;
+            }
+        }
+    }
+}
+
+// Merge of the split partials (a9): one block per (sequence, query head).
+template <int D>
+__global__ void __launch_bounds__(D)
+    decode_combine_kernel(const float* __restrict__ o_part, const float* __restrict__ lse_part,
+                          const int* __restrict__ seqused_k, int B, int Hq, int num_splits,
+                          int tokens_per_split, int max_tokens, __nv_bfloat16* __restrict__ o, float* __restrict__ lse) {
+    const int bh = blockIdx.x;
+    const int b = bh / Hq;
+    const int d = threadIdx.x;
+    const int L = min(max(seqused_k[b], 0), max_tokens);
+    const int ns = min(num_splits, (L + tokens_per_split - 1) / tokens_per_split);
+    float M = -INFINITY;
+    for (int s = 0; s < ns; ++s) M = fmaxf(M, lse_part[(long long)s * B * Hq + bh]);
+    float acc = 0.0f, out_lse = -INFINITY;
+    if (M != -INFINITY) {
+        float W = 0.0f;
+        for (int s = 0; s < ns; ++s) W += __expf(lse_part[(long long)s * B * Hq + bh] - M);
+        out_lse = M + __logf(W);
+        for (int s = 0; s < ns; ++s) {
+            const float w = __expf(lse_part[(long long)s * B * Hq + bh] - out_lse);
+            acc += w * o_part[((long long)s * B * Hq + bh) * D + d];
+        }
+    }
+    o[(long long)bh * D + d] = __float2bfloat16_rn(acc);
+    if (lse && d == 0) lse[bh] = out_lse;
+}
+
+}  // namespace attn

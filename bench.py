@@ -1,0 +1,461 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 attention library on its seeded synthetic workloads.
+
+Primary line (one JSON object on stdout, rank 0):
+  paged GQA decode, bf16: B=32 sequences x 1 query token, Hq=32, Hkv=8, D=128,
+  16-token pages, kv lengths ~ U[1, 8192], random block table over a
+  20000-page pool.  value = algorithmic K/V (+Q, O, LSE, block-table) bytes per
+  step / device time per step, in GB/s; one step = one attn_decode_paged call
+  (split-KV kernel + combine kernel).
+Carried in the same line:
+  "prefill":     varlen paged GQA prefill, causal, 16 seqs, L ~ U[64, 4096],
+                 Hq=32, Hkv=8, D=128 -> TFLOP/s (4*D*allowed pairs per head)
+  "prefill_fp8": fp8 e4m3 dense causal B=4, H=16, L=4096, D=128 -> TFLOP/s,
+                 with the bf16 kernel on the same data beside it.
+
+Timing: W warm-up steps, then K steps each bracketed by CUDA events on the
+launching stream, a 256 MiB L2 flush between steps outside the events, and a
+barrier + synchronize on both sides of the timed region; max over ranks.
+N > 1 runs N independent replicas (one process per GPU; no collective on the
+data path).  --impl reference times the fp64 CPU oracle instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "attn fwd TFLOP/s (prefill) & paged-decode KV GB/s on 1 B200, % of roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--no-prefill", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--seed", type=int, default=0)
+    return p.parse_args()
+
+
+# --------------------------------------------------------------------------- plumbing
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+class Clocks:
+    """Samples SM clocks and throttle reasons with nvidia-smi during a timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not self.path:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+def time_steps(step_fn, steps, warmup, world, flush):
+    """Per-step device times (ms) with CUDA events on the current stream, L2 flushed between steps."""
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        step_fn()
+    barrier(world)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    for s, e in ev:
+        flush.zero_()
+        s.record(stream)
+        step_fn()
+        e.record(stream)
+    barrier(world)
+    return [s.elapsed_time(e) for s, e in ev]
+
+
+# --------------------------------------------------------------------------- algorithmic work
+def decode_bytes(t, Hq, Hkv, D):
+    lens = t["seqused_k"].numpy().astype(np.int64)
+    B = len(lens)
+    kv = int(lens.sum()) * Hkv * D * 2 * 2
+    pages = int(((lens + 15) // 16).sum()) * 4
+    return kv + B * Hq * D * 2 * 2 + B * Hq * 4 + pages + B * 4
+
+
+def causal_flops(lens, Hq, D):
+    lens = np.asarray(lens, np.int64)
+    return float(4 * D * Hq * (lens * (lens + 1) // 2).sum())
+
+
+# --------------------------------------------------------------------------- CPU oracle legs
+def oracle_decode_sample(w, target_tokens=8192, offset=0):
+    """Runs the fp64 oracle on a bounded sample of the decode batch; returns (seconds, bytes)."""
+    import oracle
+    t = w.tensors
+    lens = t["seqused_k"].numpy()
+    B = len(lens)
+    idx, tok = [], 0
+    for i in range(B):
+        b = (offset + i) % B
+        idx.append(b)
+        tok += int(lens[b])
+        if tok >= target_tokens:
+            break
+    q = t["q"][idx]
+    k_parts, v_parts, bt_rows, maxp = [], [], [], 0
+    base = 0
+    for b in idx:
+        n = (int(lens[b]) + 15) // 16
+        pages = t["block_table"][b, :n].long()
+        k_parts.append(t["k_cache"][pages])
+        v_parts.append(t["v_cache"][pages])
+        bt_rows.append(torch.arange(base, base + n, dtype=torch.int32))
+        base += n
+        maxp = max(maxp, n)
+    bt = torch.zeros(len(idx), max(maxp, 1), dtype=torch.int32)
+    for i, r in enumerate(bt_rows):
+        bt[i, :len(r)] = r
+    kc = torch.cat(k_parts) if k_parts else t["k_cache"][:1]
+    vc = torch.cat(v_parts) if v_parts else t["v_cache"][:1]
+    su = t["seqused_k"][idx]
+    nthreads = os.cpu_count() or 1
+    t0 = time.perf_counter()
+    oracle.attn_decode(q, kc, vc, bt, su, scale=w.params["scale"], nthreads=nthreads)
+    dt = time.perf_counter() - t0
+    sub = {"seqused_k": su}
+    return dt, decode_bytes(sub, w.params["Hq"], w.params["Hkv"], w.params["D"]), len(idx), int(su.sum())
+
+
+def cpu_model():
+    try:
+        out = subprocess.run(["lscpu"], capture_output=True, text=True).stdout
+        for line in out.splitlines():
+            if line.startswith("Model name"):
+                return line.split(":", 1)[1].strip()
+    except Exception:
+        pass
+    return "unknown"
+
+
+# --------------------------------------------------------------------------- arms
+def run_reference(args, rank, world):
+    """The oracle, as it stands, on the host cores (rank 0 only)."""
+    if rank != 0:
+        return
+    from attention_paged_kv_gqa_b200 import workloads as W
+    w = W.paged_decode(seed=args.seed)
+    for i in range(args.warmup):
+        oracle_decode_sample(w, offset=i)
+    secs, nbytes, toks = 0.0, 0, 0
+    for i in range(args.steps):
+        dt, nb, _, tk = oracle_decode_sample(w, offset=args.warmup + i)
+        secs += dt
+        nbytes += nb
+        toks += tk
+    value = nbytes / secs / 1e9
+    cores = os.cpu_count() or 1
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(secs / args.steps * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "paged_gqa_decode_bf16 (B=32, Hq=32, Hkv=8, D=128, 16-token pages, "
+                               "L~U[1,8192], 20000-page pool); each step a sample of whole sequences "
+                               "totalling >= 8192 keys", "parallelism": "replicas"},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": "%d steps, %d keys in total, all 32 heads" % (args.steps, toks),
+                         "cpu": cpu_model()},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, rank, world, local):
+    from attention_paged_kv_gqa_b200 import binding as A
+    from attention_paged_kv_gqa_b200 import workloads as W
+    dev = torch.device("cuda", local if world > 1 else 0)
+    st = A.attn_check_device(dev.index)
+    if st != 0:
+        raise RuntimeError("device check failed: " + A.status_string(st))
+    peaks, peak_kind = load_peaks()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    # ---------------- decode (primary)
+    w = W.paged_decode(seed=args.seed)
+    t = w.tensors
+    P = w.params
+    d = {k: v.to(dev) for k, v in t.items()}
+    ws = torch.empty(max(A.attn_decode_workspace_size(P["B"], P["Hq"], P["Hkv"], P["D"],
+                                                      P["max_blocks_per_seq"]), 16),
+                     dtype=torch.uint8, device=dev)
+    o = torch.empty(P["B"], P["Hq"], P["D"], dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(P["B"], P["Hq"], dtype=torch.float32, device=dev)
+
+    def dec_step():
+        A.attn_decode_paged(d["q"], d["k_cache"], d["v_cache"], d["block_table"], d["seqused_k"],
+                            scale=P["scale"], out=o, lse=lse, workspace=ws)
+
+    nbytes = decode_bytes(t, P["Hq"], P["Hkv"], P["D"])
+    with Clocks(dev.index) as clk:
+        times = time_steps(dec_step, args.steps, args.warmup, world, flush)
+    clocks = clk.summary()
+    ms = statistics.mean(times)
+    ms_max = max_over_ranks(sum(times), world) / args.steps
+    value = nbytes * world / (ms_max * 1e-3) / 1e9
+    kernel_gbs = nbytes / (ms * 1e-3) / 1e9
+    ns = 1 if A.attn_decode_workspace_size(P["B"], P["Hq"], P["Hkv"], P["D"],
+                                           P["max_blocks_per_seq"]) <= 16 else 2
+
+    # end to end through the binding with host buffers: q, block_table, seqused_k in
+    # (pinned), O and LSE out; the paged cache is resident device state.
+    qh = t["q"].pin_memory()
+    bth = t["block_table"].pin_memory()
+    suh = t["seqused_k"].pin_memory()
+    oh = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    lh = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    qd, btd, sud = torch.empty_like(d["q"]), torch.empty_like(d["block_table"]), torch.empty_like(d["seqused_k"])
+
+    def e2e_step():
+        qd.copy_(qh, non_blocking=True)
+        btd.copy_(bth, non_blocking=True)
+        sud.copy_(suh, non_blocking=True)
+        A.attn_decode_paged(qd, d["k_cache"], d["v_cache"], btd, sud, scale=P["scale"], out=o,
+                            lse=lse, workspace=ws)
+        oh.copy_(o, non_blocking=True)
+        lh.copy_(lse, non_blocking=True)
+
+    e2e_times = time_steps(e2e_step, args.steps, args.warmup, world, flush)
+    e2e_ms = max_over_ranks(sum(e2e_times), world) / args.steps
+    h2d = qh.numel() * 2 + bth.numel() * 4 + suh.numel() * 4
+    d2h = oh.numel() * 2 + lh.numel() * 4
+
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_max, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic: seeded N(0,1) bf16 q/k/v, uniform kv lengths, permuted page pool",
+        "config": {"workload": "paged_gqa_decode_bf16: B=32 x 1 query token, Hq=32, Hkv=8, "
+                               "D=128, 16-token pages, kv len ~ U[1,8192] (seed %d: %d keys), "
+                               "20000-page pool" % (args.seed, int(t["seqused_k"].sum())),
+                   "global_batch": P["B"] * world, "seq_len": int(t["seqused_k"].max()),
+                   "parallelism": "replicas" if world > 1 else "single",
+                   "l2": "256 MiB L2 flush between timed steps (and %.0f MB of K/V per step)"
+                         % (nbytes / 1e6),
+                   "bytes_per_step": nbytes},
+        "roofline": {"bound": "hbm", "achieved": round(kernel_gbs, 1),
+                     "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": round(kernel_gbs / peaks["hbm_gbs"], 4), "traffic": None,
+                     "kernel": "decode_split_kernel<128> + decode_combine_kernel<128> (one call)",
+                     "peak_kind": peak_kind},
+        "e2e": {"value": round(nbytes * world / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": round(e2e_ms, 5),
+                "note": "paged K/V cache resident on the device; q, block_table, seqused_k "
+                        "copied in and O, LSE copied out every step"},
+        "gpu_launches": args.steps * ns,
+        "clocks": clocks,
+    }
+
+    # ---------------- prefill (carried in the same line)
+    if not args.no_prefill:
+        del d
+        wp = W.varlen_paged_prefill(seed=args.seed)
+        tp, Pp = wp.tensors, wp.params
+        dp = {k: v.to(dev) for k, v in tp.items()}
+        op = torch.empty(Pp["total_q"], Pp["Hq"], Pp["D"], dtype=torch.bfloat16, device=dev)
+        lp = torch.empty(Pp["Hq"], Pp["total_q"], dtype=torch.float32, device=dev)
+
+        def pf_step():
+            A.attn_fwd_varlen_paged(dp["q"], dp["k_cache"], dp["v_cache"],
+                                    cu_seqlens_q=dp["cu_seqlens_q"], max_seqlen_q=Pp["max_seqlen_q"],
+                                    block_table=dp["block_table"], seqused_k=dp["seqused_k"],
+                                    mask=A.MASK_CAUSAL, scale=Pp["scale"], out=op, lse=lp)
+
+        pt = time_steps(pf_step, args.steps, args.warmup, world, flush)
+        pms = statistics.mean(pt)
+        flops = causal_flops(tp["seqused_k"].numpy(), Pp["Hq"], Pp["D"])
+        tf = flops / (pms * 1e-3) / 1e12
+        line["prefill"] = {
+            "workload": "varlen_paged_gqa_prefill_causal_bf16: 16 seqs, q len = kv len ~ "
+                        "U[64,4096] (seed %d: %d tokens), Hq=32, Hkv=8, D=128, 16-token pages"
+                        % (args.seed, Pp["total_q"]),
+            "value": round(tf, 2), "unit": "TFLOP/s", "ms_per_step": round(pms, 5),
+            "flops_per_step": flops,
+            "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": peaks["bf16_tflops"],
+                         "unit": "TFLOP/s", "frac": round(tf / peaks["bf16_tflops"], 4),
+                         "traffic": None, "kernel": "prefill_kernel<128,bf16>",
+                         "peak_kind": peak_kind},
+        }
+        line["gpu_launches"] += 0   # prefill runs outside the primary timed region
+        del dp
+
+        w8 = W.fp8_dense_causal(seed=args.seed)
+        t8 = w8.tensors
+        d8 = {k: v.to(dev) for k, v in t8.items()}
+        o8 = torch.empty(4, 4096, 16, 128, dtype=torch.bfloat16, device=dev)
+        l8 = torch.empty(4, 16, 4096, dtype=torch.float32, device=dev)
+
+        def f8_step():
+            A.attn_fwd_dense(d8["q_fp8"], d8["k_fp8"], d8["v_fp8"], causal=True,
+                             scale=w8.params["scale"], descale_q=d8["descale_q"],
+                             descale_k=d8["descale_k"], descale_v=d8["descale_v"], out=o8, lse=l8)
+
+        def b16_step():
+            A.attn_fwd_dense(d8["q"], d8["k"], d8["v"], causal=True, scale=w8.params["scale"],
+                             out=o8, lse=l8)
+
+        f8ms = statistics.mean(time_steps(f8_step, args.steps, args.warmup, world, flush))
+        b16ms = statistics.mean(time_steps(b16_step, args.steps, args.warmup, world, flush))
+        fl8 = causal_flops([4096] * 4, 16, 128)
+        fp8_peak = 2.0 * peaks["bf16_tflops"]
+        line["prefill_fp8"] = {
+            "workload": "fp8_e4m3_dense_causal: B=4, H=16, L=4096, D=128, per-tensor descale",
+            "value": round(fl8 / (f8ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+            "ms_per_step": round(f8ms, 5),
+            "bf16_same_data": {"value": round(fl8 / (b16ms * 1e-3) / 1e12, 2),
+                               "ms_per_step": round(b16ms, 5),
+                               "fp8_time_over_bf16_time": round(f8ms / b16ms, 4)},
+            "roofline": {"bound": "tensor", "achieved": round(fl8 / (f8ms * 1e-3) / 1e12, 1),
+                         "peak": fp8_peak, "unit": "TFLOP/s",
+                         "frac": round(fl8 / (f8ms * 1e-3) / 1e12 / fp8_peak, 4), "traffic": None,
+                         "kernel": "prefill_kernel<128,fp8>",
+                         "peak_kind": peak_kind + " bf16 x 2 (nominal fp8/bf16 ratio)"},
+        }
+        del d8
+
+    # ---------------- CPU baseline: the oracle on rank 0 at N=1, a bounded sample
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        secs, nb, nseq, tok = 0.0, 0, 0, 0
+        t_start = time.perf_counter()
+        i = 0
+        while time.perf_counter() - t_start < 10.0 and i < 32:
+            dt, b_, n_, tk = oracle_decode_sample(w, target_tokens=8192, offset=i * 3)
+            secs += dt
+            nb += b_
+            nseq += n_
+            tok += tk
+            i += 1
+        line["cpu_baseline"] = {"value": round(nb / secs / 1e9, 4), "unit": "GB/s",
+                                "cores": os.cpu_count() or 1, "kind": "oracle",
+                                "sample": "%d oracle calls over %d whole sequences (%d keys, all "
+                                          "32 heads) of the decode batch" % (i, nseq, tok),
+                                "cpu": cpu_model()}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    rank, world, local = dist_setup(args.gpus)
+    try:
+        if args.impl == "reference":
+            run_reference(args, rank, world)
+        else:
+            run_ours(args, rank, world, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

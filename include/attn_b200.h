@@ -1,0 +1,174 @@
+/*
+ * attn_b200.h -- C ABI of libattn_b200.so: fused scaled-dot-product attention
+ * forward with log-sum-exp output on NVIDIA B200 (sm_100a).
+ *
+ *   O   = softmax(scale * Q K^T + mask) V
+ *   LSE = ln sum_{allowed j} exp(scale * q . k_j)        (natural log, scale included)
+ *
+ * Definition: the FlexAttention forward ("[FlexAttention] Enforce Q,K,V memory
+ * layouts for fp8 flex attention", pytorch commit 7e16cb99, flex_attention
+ * docstring: shapes (B,Hq,L,E) / (B,Hkv,S,E), default scale 1/sqrt(E),
+ * enable_gqa) with the log-sum-exp output and possibly fully masked rows of its
+ * lowering ("Cross Attention does not work on CPU and older GPUs", BLT issue 6:
+ * OUTPUT_LOGSUMEXP True, ROWS_GUARANTEED_SAFE False).  Varlen batches, the paged
+ * KV cache and grouped-query heads follow "[CUDA] PagedAttention: add SM<80
+ * fp16 fallback via memory-efficient attention" (onnxruntime PR 28200,
+ * Implementation steps 2-3: block_table walk, [total_tokens, num_heads,
+ * head_size] packing addressed by cumulative sequence lengths); seqused_k
+ * follows "Rope dim" (vllm-project/flash-attention PR 172, the varlen
+ * arguments).  fp8 e4m3 operands follow the FlexAttention fp8 commit above
+ * (float8_e4m3fn, both GEMMs in the query dtype).
+ *
+ * Conventions shared by every call:
+ *  - Ownership: the caller owns every buffer.  All tensor pointers are DEVICE
+ *    pointers (e.g. from torch); scalars are passed by value.  The library never
+ *    allocates device memory per call, never synchronises the stream and never
+ *    reads device data on the host: calls are asynchronous on `stream`.
+ *  - Errors: argument errors are returned synchronously before anything is
+ *    launched.  A launch failure (cudaGetLastError) returns ATTN_ERR_CUDA.
+ *    No call prints, traps or aborts.
+ *  - Device check: each call first checks (once per device, then cached) that
+ *    the current device is compute capability 10.0 and that this library's
+ *    kernel image loads on it (ATTN_ERR_NO_KERNEL_IMAGE otherwise) -- the
+ *    check is made at call time, not deferred to the first launch.
+ *  - softmax_scale <= 0 selects the default 1/sqrt(head_dim).
+ *  - Element types: ATTN_BF16 tensors are bfloat16; ATTN_FP8_E4M3 tensors are
+ *    float8_e4m3fn codes whose real values are code * descale, with the three
+ *    descales given as DEVICE pointers to one fp32 each (no host sync).  The
+ *    output O is always bfloat16; LSE is fp32.
+ *  - Alignment: every tensor pointer and every row stride must be a multiple
+ *    of 16 bytes (the TMA rule), otherwise ATTN_ERR_INVALID_ARG.
+ *  - Supported: head_dim in {64, 128}; paged block_size == 16.  Anything else
+ *    returns ATTN_ERR_UNSUPPORTED.  num_heads_q must be a multiple of
+ *    num_heads_kv.
+ *  - Masks: ATTN_MASK_CAUSAL allows key j for query i iff j <= i + (Lk - Lq)
+ *    (bottom-right aligned; equal to q_idx >= kv_idx when Lq == Lk).
+ *    ATTN_MASK_PATCH allows key j for query i iff start_i <= j < end_i, with the
+ *    sequence-local interval [start_i, end_i) given per query.  A query with no
+ *    allowed key gets O = 0 and LSE = -inf.
+ *  - Stream: `stream` is a cudaStream_t (NULL = legacy default stream).
+ */
+#ifndef ATTN_B200_H
+#define ATTN_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    ATTN_OK = 0,
+    ATTN_ERR_INVALID_ARG = 1,        /* null/misaligned pointer, bad size or stride */
+    ATTN_ERR_UNSUPPORTED = 2,        /* valid but not implemented (head_dim, block_size, ...) */
+    ATTN_ERR_NO_KERNEL_IMAGE = 3,    /* device is not sm_100 or the image does not load */
+    ATTN_ERR_TMA_ENCODE = 4,         /* cuTensorMapEncodeTiled rejected a descriptor */
+    ATTN_ERR_WORKSPACE_TOO_SMALL = 5,
+    ATTN_ERR_CUDA = 6,               /* a CUDA runtime call or a launch failed */
+    ATTN_ERR_DEVICE_TIMEOUT = 7      /* a kernel gave up on a bounded wait (see attn_device_error) */
+} attn_status_t;
+
+typedef enum { ATTN_MASK_NONE = 0, ATTN_MASK_CAUSAL = 1, ATTN_MASK_PATCH = 2 } attn_mask_t;
+typedef enum { ATTN_BF16 = 0, ATTN_FP8_E4M3 = 1 } attn_dtype_t;
+
+/* A cudaStream_t, passed as an opaque pointer so this header needs no CUDA header. */
+typedef void *attn_stream_t;
+
+/*
+ * Checks that `device` is a compute-capability 10.0 GPU and that this
+ * library's kernels load on it.  Returns ATTN_OK, ATTN_ERR_NO_KERNEL_IMAGE or
+ * ATTN_ERR_CUDA (no driver / no such device).  Lesson of "FA3 loader reports
+ * success on Blackwell (sm_120) then dies at first kernel launch" (nanochat
+ * issue 820, Cause): check the architecture at load time, not at first launch.
+ */
+attn_status_t attn_check_device(int device);
+
+/* Static, NUL-terminated description of a status code (never NULL). */
+const char *attn_status_string(attn_status_t status);
+
+/*
+ * Reads and clears the device-side error word of the current device: 0 when
+ * no kernel gave up on a bounded wait since the last read, otherwise a code
+ * naming the wait.  Synchronises `stream` (a debugging aid, not for hot loops).
+ */
+attn_status_t attn_device_error(int *code_out, attn_stream_t stream);
+
+/*
+ * Dense attention forward.
+ *   q  [B, Lq, Hq, D], k/v [B, Lk, Hkv, D] with element strides given per
+ *      tensor as strides[3] = {batch, token, head}; the head_dim stride is 1.
+ *   o  [B, Lq, Hq, D] bf16, contiguous.   lse [B, Hq, Lq] fp32, contiguous, or NULL.
+ *   mask: ATTN_MASK_NONE or ATTN_MASK_CAUSAL (PATCH needs the varlen call).
+ *   descale_*: fp8 only (device fp32 scalars), ignored for bf16.
+ */
+attn_status_t attn_fwd_dense(
+    const void *q, const void *k, const void *v, void *o, float *lse,
+    int B, int Lq, int Lk, int num_heads_q, int num_heads_kv, int head_dim,
+    const int64_t *strides_q, const int64_t *strides_k, const int64_t *strides_v,
+    float softmax_scale, int mask, int dtype,
+    const float *descale_q, const float *descale_k, const float *descale_v,
+    attn_stream_t stream);
+
+/*
+ * Varlen attention forward over packed queries and a paged (or packed) KV store.
+ *   q            [total_q, Hq, D], contiguous; sequence b owns rows
+ *                cu_seqlens_q[b] .. cu_seqlens_q[b+1]-1 (cu_seqlens_q: int32 [B+1]).
+ *   k_cache/v_cache
+ *     paged  (block_table != NULL): [num_blocks, block_size, Hkv, D], contiguous;
+ *            key j of sequence b is row j % block_size of page
+ *            block_table[b * max_blocks_per_seq + j / block_size].
+ *     packed (block_table == NULL): [total_k, Hkv, D], contiguous; sequence b owns
+ *            rows cu_seqlens_k[b] .. ; cu_seqlens_k required.
+ *   seqused_k    int32 [B] keys used per sequence, or NULL (then the
+ *                difference of cu_seqlens_k, which is then required).
+ *   max_seqlen_q upper bound of the per-sequence query lengths (sizes the grid).
+ *   patch_kv_range int32 [total_q, 2], PATCH only: per-query [start, end).
+ *   o            [total_q, Hq, D] bf16.   lse [Hq, total_q] fp32 or NULL.
+ *   workspace    unused by this version; may be NULL with workspace_bytes 0.
+ * Page indices outside [0, num_blocks) read zeros (TMA bounds fill); the
+ * caller must keep block_table entries for the used pages valid.
+ */
+attn_status_t attn_fwd_varlen_paged(
+    const void *q, const void *k_cache, const void *v_cache,
+    const int32_t *block_table, int max_blocks_per_seq, int num_blocks, int block_size,
+    const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k, const int32_t *seqused_k,
+    int B, int total_q, int total_k, int max_seqlen_q,
+    int num_heads_q, int num_heads_kv, int head_dim,
+    float softmax_scale, int mask, const int32_t *patch_kv_range,
+    int dtype, const float *descale_q, const float *descale_k, const float *descale_v,
+    void *o, float *lse, void *workspace, size_t workspace_bytes, attn_stream_t stream);
+
+/*
+ * Bytes of workspace attn_decode_paged needs for these sizes (fp32 partial O
+ * and LSE per split).  num_splits <= 0 means "as chosen automatically for
+ * max_blocks_per_seq".  Returns 0 for invalid sizes.
+ */
+size_t attn_decode_workspace_size(int B, int num_heads_q, int num_heads_kv, int head_dim,
+                                  int max_blocks_per_seq, int block_size, int num_splits);
+
+/*
+ * Paged decode: one query token per sequence, split-KV with an LSE-weighted
+ * combine.  Non-causal over the sequence's cached keys.
+ *   q            [B, Hq, D] bf16, contiguous.
+ *   k_cache/v_cache, block_table, block_size: as in attn_fwd_varlen_paged.
+ *   seqused_k    int32 [B], keys cached per sequence (0 gives O = 0, LSE = -inf).
+ *   num_splits   key-range splits per sequence; <= 0 chooses automatically.
+ *   o            [B, Hq, D] bf16.   lse [B, Hq] fp32 or NULL.
+ *   workspace    >= attn_decode_workspace_size(...) bytes of device memory,
+ *                16-byte aligned; its contents on entry do not matter.
+ * Supported: bf16, head_dim in {64, 128}, Hq/Hkv <= 16.
+ */
+attn_status_t attn_decode_paged(
+    const void *q, const void *k_cache, const void *v_cache, const int32_t *block_table,
+    int max_blocks_per_seq, int num_blocks, int block_size, const int32_t *seqused_k,
+    int B, int num_heads_q, int num_heads_kv, int head_dim, float softmax_scale,
+    int num_splits, int dtype,
+    const float *descale_q, const float *descale_k, const float *descale_v,
+    void *o, float *lse, void *workspace, size_t workspace_bytes, attn_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_B200_H */

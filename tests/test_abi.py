@@ -1,0 +1,108 @@
+"""The C-ABI library loads on a machine without a GPU, exports every declared
+entry point, and rejects bad arguments before touching the device."""
+import ctypes
+import re
+from pathlib import Path
+
+import pytest
+
+from attention_paged_kv_gqa_b200 import build as B
+from attention_paged_kv_gqa_b200 import binding
+
+ROOT = Path(__file__).resolve().parents[1]
+
+
+@pytest.fixture(scope="module")
+def L():
+    B.build()
+    return binding.lib()
+
+
+def declared_entry_points():
+    names = set()
+    for h in (ROOT / "include").glob("*.h"):
+        text = h.read_text()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names |= set(re.findall(r"\b(attn_[a-z0-9_]+)\s*\(", text))
+    return sorted(names)
+
+
+def test_header_declares_the_boundary():
+    names = declared_entry_points()
+    for n in ("attn_fwd_dense", "attn_fwd_varlen_paged", "attn_decode_paged",
+              "attn_decode_workspace_size", "attn_check_device", "attn_status_string"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(L):
+    for n in declared_entry_points():
+        assert hasattr(L, n), n
+
+
+def test_status_strings(L):
+    for s in range(0, 8):
+        assert binding.status_string(s)
+    assert binding.status_string(0) == "ok"
+
+
+def test_device_check_without_gpu_is_an_error_not_a_crash(L):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("has a GPU")
+    assert L.attn_check_device(0) != 0
+
+
+def _strides():
+    return (ctypes.c_int64 * 3)(128 * 2 * 64, 2 * 64, 64)
+
+
+def test_null_pointers_rejected_before_launch(L):
+    st = L.attn_fwd_dense(None, None, None, None, None, 1, 128, 128, 2, 2, 64, _strides(),
+                          _strides(), _strides(), 0.0, 1, 0, None, None, None, None)
+    assert st == 1
+
+
+def test_bad_group_and_head_dim(L):
+    p = ctypes.c_void_p(1 << 20)
+    st = L.attn_fwd_dense(p, p, p, p, None, 1, 128, 128, 3, 2, 64, _strides(), _strides(),
+                          _strides(), 0.0, 1, 0, None, None, None, None)
+    assert st == 1                     # Hq % Hkv != 0
+    st = L.attn_fwd_dense(p, p, p, p, None, 1, 128, 128, 2, 2, 96, _strides(), _strides(),
+                          _strides(), 0.0, 1, 0, None, None, None, None)
+    assert st == 2                     # head_dim 96 unsupported
+
+
+def test_misaligned_pointer_and_fp8_without_descale(L):
+    p = ctypes.c_void_p(1 << 20)
+    bad = ctypes.c_void_p((1 << 20) + 8)
+    st = L.attn_fwd_dense(bad, p, p, p, None, 1, 128, 128, 2, 2, 64, _strides(), _strides(),
+                          _strides(), 0.0, 1, 0, None, None, None, None)
+    assert st == 1
+    s128 = (ctypes.c_int64 * 3)(128 * 2 * 128, 2 * 128, 128)
+    st = L.attn_fwd_dense(p, p, p, p, None, 1, 128, 128, 2, 2, 128, s128, s128, s128, 0.0, 1, 1,
+                          None, None, None, None)
+    assert st == 1
+
+
+def test_paged_block_size_and_patch_requirements(L):
+    p = ctypes.c_void_p(1 << 20)
+    cu = ctypes.c_void_p(1 << 21)
+    # block_size 32 -> unsupported
+    st = L.attn_fwd_varlen_paged(p, p, p, p, 4, 100, 32, cu, None, cu, 1, 16, 0, 16, 2, 2, 64,
+                                 0.0, 1, None, 0, None, None, None, p, None, None, 0, None)
+    assert st == 2
+    # patch mask without ranges -> invalid
+    st = L.attn_fwd_varlen_paged(p, p, p, p, 4, 100, 16, cu, None, cu, 1, 16, 0, 16, 2, 2, 64,
+                                 0.0, 2, None, 0, None, None, None, p, None, None, 0, None)
+    assert st == 1
+
+
+def test_decode_workspace_size_and_limits(L):
+    n = L.attn_decode_workspace_size(32, 32, 8, 128, 512, 16, 0)
+    assert n > 0 and n % 4 == 0
+    assert L.attn_decode_workspace_size(0, 32, 8, 128, 512, 16, 0) == 0
+    p = ctypes.c_void_p(1 << 20)
+    # group of 32 query heads per KV head is beyond the decode kernel's 16 rows
+    st = L.attn_decode_paged(p, p, p, p, 4, 100, 16, p, 1, 32, 1, 128, 0.0, 1, 0, None, None,
+                             None, p, None, p, 1 << 20, None)
+    assert st == 2
