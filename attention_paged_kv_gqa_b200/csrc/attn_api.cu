@@ -67,6 +67,21 @@ attn_status_t current_device_ok(int* dev_out) {
     return s == 1 ? ATTN_OK : static_cast<attn_status_t>(s - 100);
 }
 
+int sm_count(int dev) {
+    static std::atomic<int> cache[kMaxDevices];
+    if (dev >= 0 && dev < kMaxDevices) {
+        int v = cache[dev].load(std::memory_order_relaxed);
+        if (v > 0) return v;
+    }
+    int n = 148;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+        cudaGetLastError();
+        n = 148;
+    }
+    if (dev >= 0 && dev < kMaxDevices) cache[dev].store(n, std::memory_order_relaxed);
+    return n;
+}
+
 // ------------------------------------------------------------------ TMA descriptors
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -181,11 +196,14 @@ template <int D, bool FP8>
 attn_status_t launch_prefill_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                                const PrefillArgs& a, long long grid, cudaStream_t stream) {
     using Cfg = PrefillCfg<D, FP8>;
-    static std::atomic<bool> attr_done{false};
-    if (!attr_done.load()) {
+    static std::atomic<uint64_t> attr_mask{0};   // one bit per device
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const uint64_t bit = 1ull << (dev & 63);
+    if (!(attr_mask.load() & bit)) {
         const attn_status_t s = set_smem(prefill_kernel<D, FP8>, Cfg::SMEM_BYTES);
         if (s != ATTN_OK) return s;
-        attr_done.store(true);
+        attr_mask.fetch_or(bit);
     }
     prefill_kernel<D, FP8><<<static_cast<unsigned>(grid), kPrefillThreads, Cfg::SMEM_BYTES, stream>>>(
         mq, mk, mv, a);
@@ -209,6 +227,71 @@ void unit_grid(PrefillArgs& a, int max_seqlen_q, long long* grid) {
     a.NH = a.pair_heads ? a.Hq / 2 : a.Hq;
     a.NQ = a.pair_heads ? nqt : (nqt + 1) / 2;
     *grid = static_cast<long long>(a.NQ) * a.B * a.NH;
+}
+
+// Stage-ring depth and CTAs per SM for the decode kernel: two CTAs per SM
+// when at least two 64-key stages fit in half of the SM's shared memory,
+// otherwise one CTA with as many stages as fit.
+template <int D>
+bool decode_geometry(int G, int B, int* ns_out, int* ctas_per_sm, int* smem_out) {
+    using Cfg = DecodeCfg<D>;
+    const int half = (228 * 1024 - 2 * 1024) / 2;
+    const int whole = 227 * 1024;
+    for (int per_sm : {2, 1}) {
+        const int cap = per_sm == 2 ? half : whole;
+        int ns = 0;
+        while (ns < 16 && Cfg::smem_bytes(G, B, ns + 1) <= cap) ++ns;
+        if (ns >= 2) {
+            *ns_out = ns;
+            *ctas_per_sm = per_sm;
+            *smem_out = Cfg::smem_bytes(G, B, ns);
+            return true;
+        }
+    }
+    return false;
+}
+
+template <int D>
+attn_status_t launch_decode(const CUtensorMap& mk, const CUtensorMap& mv, DecodeArgs a,
+                            int sms, long long items_max, cudaStream_t st, const int32_t* seqused_k,
+                            int max_tokens) {
+    static std::atomic<uint64_t> attr_mask{0};   // one bit per device
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const uint64_t bit = 1ull << (dev & 63);
+    if (!(attr_mask.load() & bit)) {
+        const attn_status_t s = set_smem(decode_split_kernel<D>, 227 * 1024);
+        if (s != ATTN_OK) return s;
+        attr_mask.fetch_or(bit);
+    }
+    int ns = 0, per_sm = 0, smem = 0;
+    if (!decode_geometry<D>(a.group, a.B, &ns, &per_sm, &smem)) return ATTN_ERR_UNSUPPORTED;
+    a.nstages = ns;
+    const int grid = (int)std::min<long long>((long long)sms * per_sm, std::max<long long>(items_max, 1));
+    decode_split_kernel<D><<<grid, kDecThreads, smem, st>>>(mk, mv, a);
+    attn_status_t s = launch_status();
+    if (s != ATTN_OK || a.direct) return s;
+    // The combine kernel is launched as a programmatic dependent of the split
+    // kernel: it is scheduled while the split grid runs and waits on the grid
+    // dependency before reading the partials.
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(a.B * a.Hq);
+    cfg.blockDim = dim3(D);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, decode_combine_kernel<D>, (const float*)a.o_part,
+                           (const float*)a.lse_part, (const int*)seqused_k, a.B, a.Hq, a.num_splits,
+                           a.tokens_per_split, max_tokens, a.o, a.lse) != cudaSuccess) {
+        cudaGetLastError();
+        return ATTN_ERR_CUDA;
+    }
+    return ATTN_OK;
 }
 
 }  // namespace
@@ -421,6 +504,7 @@ static void decode_splits(int B, int Hkv, int max_tokens, int requested, int* nu
         ns = std::max(for_balance, for_fill);
     }
     ns = std::max(1, std::min(ns, (max_tokens + kDecStageTok - 1) / kDecStageTok));
+    ns = std::min(ns, kMaxSplits);
     int t = (max_tokens + ns - 1) / ns;
     t = (t + kDecStageTok - 1) / kDecStageTok * kDecStageTok;
     *tps = t;
@@ -455,6 +539,7 @@ attn_status_t attn_decode_paged(const void* q, const void* k_cache, const void* 
     if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
     if (block_size != kPageRows) return ATTN_ERR_UNSUPPORTED;
     if (Hq / Hkv > kDecRows) return ATTN_ERR_UNSUPPORTED;
+    if (B > kDecMaxSeqs) return ATTN_ERR_UNSUPPORTED;
     if ((long long)num_blocks * block_size >= (1LL << 31)) return ATTN_ERR_UNSUPPORTED;
     if ((long long)max_blocks_per_seq * block_size >= (1LL << 30)) return ATTN_ERR_UNSUPPORTED;
     if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o))
@@ -467,7 +552,8 @@ attn_status_t attn_decode_paged(const void* q, const void* k_cache, const void* 
         if (!workspace || !aligned16(workspace)) return ATTN_ERR_INVALID_ARG;
         if (workspace_bytes < need) return ATTN_ERR_WORKSPACE_TOO_SMALL;
     }
-    const attn_status_t dvs = current_device_ok(nullptr);
+    int dev = 0;
+    const attn_status_t dvs = current_device_ok(&dev);
     if (dvs != ATTN_OK) return dvs;
     if (B == 0) return ATTN_OK;
 
@@ -502,32 +588,14 @@ attn_status_t attn_decode_paged(const void* q, const void* k_cache, const void* 
         a.lse_part = a.o_part + (size_t)ns * B * Hq * D;
     }
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const dim3 grid(ns, Hkv, B);
-    if (D == 128) {
-        static std::atomic<bool> done{false};
-        if (!done.load()) {
-            if ((s = set_smem(decode_split_kernel<128>, DecodeCfg<128>::SMEM_BYTES)) != ATTN_OK) return s;
-            done.store(true);
-        }
-        decode_split_kernel<128><<<grid, kDecThreads, DecodeCfg<128>::SMEM_BYTES, st>>>(mk, mv, a);
-        if ((s = launch_status()) != ATTN_OK) return s;
-        if (ns > 1)
-            decode_combine_kernel<128><<<B * Hq, 128, 0, st>>>(a.o_part, a.lse_part, seqused_k, B, Hq,
-                                                                ns, tps, max_blocks_per_seq * block_size,
-                                                                a.o, lse);
-    } else {
-        static std::atomic<bool> done{false};
-        if (!done.load()) {
-            if ((s = set_smem(decode_split_kernel<64>, DecodeCfg<64>::SMEM_BYTES)) != ATTN_OK) return s;
-            done.store(true);
-        }
-        decode_split_kernel<64><<<grid, kDecThreads, DecodeCfg<64>::SMEM_BYTES, st>>>(mk, mv, a);
-        if ((s = launch_status()) != ATTN_OK) return s;
-        if (ns > 1)
-            decode_combine_kernel<64><<<B * Hq, 64, 0, st>>>(a.o_part, a.lse_part, seqused_k, B, Hq,
-                                                              ns, tps, max_blocks_per_seq * block_size,
-                                                              a.o, lse);
-    }
+    const long long items_max = (long long)B * Hkv * ns;
+    if (D == 128)
+        s = launch_decode<128>(mk, mv, a, sm_count(dev), items_max, st, seqused_k,
+                               max_blocks_per_seq * block_size);
+    else
+        s = launch_decode<64>(mk, mv, a, sm_count(dev), items_max, st, seqused_k,
+                              max_blocks_per_seq * block_size);
+    if (s != ATTN_OK) return s;
     return launch_status();
 }
 

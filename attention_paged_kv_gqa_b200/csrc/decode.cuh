@@ -25,6 +25,7 @@ namespace attn {
 constexpr int kDecThreads = 160;      // warps 0-3 consumers, warp 4 producer
 constexpr int kDecStageTok = 64;      // keys per stage (4 pages)
 constexpr int kDecRows = 16;          // MMA rows = query heads of one KV group (padded)
+constexpr int kDecMaxSeqs = 4096;     // sequences per call (on-device item table in smem)
 
 struct DecodeArgs {
     int B, Hq, Hkv, group;
@@ -40,6 +41,7 @@ struct DecodeArgs {
     __nv_bfloat16* o;         // [B][Hq][D]  (direct mode)
     float* lse;               // [B][Hq]     (direct mode, nullable)
     int direct;               // 1: single split, write the final result
+    int nstages;              // stage ring depth (runtime: sized from G and B)
 };
 
 template <int D>
@@ -48,10 +50,18 @@ struct DecodeCfg {
     static constexpr int NCHUNK = ROWB / 128;
     static constexpr int STAGE_K = kDecStageTok * ROWB;
     static constexpr int STAGE = 2 * STAGE_K;              // K then V
-    static constexpr int NS = (D == 128) ? 3 : 6;
-    static constexpr int MERGE_BYTES = 4 * kDecRows * (D + 2) * 4;
-    static constexpr int BODY = (NS * STAGE > MERGE_BYTES) ? NS * STAGE : MERGE_BYTES;
-    static constexpr int SMEM_BYTES = 1024 + BODY + 256;
+    static_assert(STAGE % 1024 == 0, "stages stay 1024-byte aligned for the 128-byte swizzle");
+    // Shared memory after the stage ring, for group size G and B sequences:
+    // merge area [4][G][D] f32 + m, l [4][16] f32; tables prefix [B+1] and
+    // lengths [B] int32 (16-byte rounded); then 2*NS mbarriers.
+    __host__ __device__ static constexpr int merge_bytes(int G) { return 4 * G * D * 4 + 2 * 4 * kDecRows * 4; }
+    __host__ __device__ static constexpr int table_bytes(int B) { return ((2 * B + 1) * 4 + 15) / 16 * 16; }
+    __host__ __device__ static constexpr int tail_bytes(int G, int B, int ns) {
+        return merge_bytes(G) + table_bytes(B) + 2 * ns * 8;
+    }
+    __host__ __device__ static constexpr int smem_bytes(int G, int B, int ns) {
+        return 1024 + ns * STAGE + tail_bytes(G, B, ns);
+    }
 };
 
 // Byte offset of element (row, col) of a [rows][D] bf16 tile stored as
@@ -63,25 +73,87 @@ __device__ __forceinline__ uint32_t swz_off(int row, int col, int rows) {
     return c * rows * 128 + row * 128 + ((piece ^ (row & 7)) << 4) + ((col & 7) << 1);
 }
 
+// Work item -> (sequence, split, kv head) through the per-sequence split counts.
+struct DecItem {
+    int b, split, g, t_begin, t_end;
+};
+
+// Sequence of L keys -> ceil(L / tps) splits of nearly equal size (multiples
+// of the stage), so the work items of one sequence are balanced.
+__host__ __device__ __forceinline__ int dec_nsplit(int L, int tps) { return (L + tps - 1) / tps; }
+
+__device__ __forceinline__ DecItem dec_item(int item, const int* prefix, int B, int Hkv, int tps,
+                                            const int* lens) {
+    DecItem it;
+    it.g = item % Hkv;
+    const int r = item / Hkv;
+    int lo = 0, hi = B;           // largest b with prefix[b] <= r
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (prefix[mid] <= r) lo = mid; else hi = mid;
+    }
+    it.b = lo;
+    it.split = r - prefix[lo];
+    const int L = lens[lo];
+    const int n = max(dec_nsplit(L, tps), 1);
+    int sz = (L + n - 1) / n;
+    sz = (sz + kDecStageTok - 1) / kDecStageTok * kDecStageTok;
+    it.t_begin = it.split * sz;
+    it.t_end = min(L, it.t_begin + sz);
+    return it;
+}
+
+// Persistent split-KV decode: one CTA per SM walks the work items
+// blockIdx.x, blockIdx.x + gridDim.x, ...; the producer warp streams the pages
+// of consecutive items through one stage ring without draining between them.
 template <int D>
 __global__ void __launch_bounds__(kDecThreads, 2)
     decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                         const DecodeArgs a) {
     using C = DecodeCfg<D>;
-    constexpr int NS = C::NS;
+    const int NS = a.nstages;
+    const int G = a.group;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::BODY);
+    float* mo = reinterpret_cast<float*>(smem + NS * C::STAGE);       // [4][G][D]
+    float* mm = mo + 4 * G * D;                                        // [4][16]
+    float* ml = mm + 4 * kDecRows;                                     // [4][16]
+    int* prefix = reinterpret_cast<int*>(ml + 4 * kDecRows);           // [B+1] split-count prefix
+    int* lenv = prefix + (a.B + 1);                                    // [B] keys per sequence
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + NS * C::STAGE + C::merge_bytes(G) +
+                                                 C::table_bytes(a.B));
     uint64_t* empty = full + NS;
 
-    const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int L = min(max(a.seqused_k[b], 0), a.max_blocks * kPageRows);
-    const int t_begin = split * a.tokens_per_split;
-    const int t_end = min(L, t_begin + a.tokens_per_split);
-    if (t_begin >= t_end && !(a.direct && split == 0)) return;   // empty split: combine skips it
-    const int nstage = (t_end > t_begin) ? (t_end - t_begin + kDecStageTok - 1) / kDecStageTok : 0;
+    // Let the combine kernel launch now; it waits for this grid's results itself.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int tps = a.tokens_per_split;
+    const int cap = a.max_blocks * kPageRows;
+    // Split counts per sequence and their exclusive prefix sum (warp 0).
+    if (warp == 0) {
+        int run = 0;
+        for (int base = 0; base < a.B; base += 32) {
+            const int b = base + lane;
+            int cnt = 0;
+            if (b < a.B) {
+                const int L = min(max(a.seqused_k[b], 0), cap);
+                cnt = dec_nsplit(L, tps);
+                if (a.direct && cnt == 0) cnt = 1;    // a zero-length row is still written
+            }
+            int incl = cnt;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += v;
+            }
+            if (b < a.B) prefix[b] = run + incl - cnt;
+            run += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (lane == 0) prefix[a.B] = run;
+    }
+    for (int b = threadIdx.x; b < a.B; b += kDecThreads)
+        lenv[b] = min(max(a.seqused_k[b], 0), cap);
     if (threadIdx.x == 0) {
         for (int i = 0; i < NS; ++i) {
             mbar_init(&full[i], 1);
@@ -90,6 +162,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
         fence_mbar_init();
     }
     __syncthreads();
+    const int total = prefix[a.B] * a.Hkv;
 
     if (warp == 4) {
         // ---------------------------------------------------- producer: page gather (a3)
@@ -98,49 +171,57 @@ __global__ void __launch_bounds__(kDecThreads, 2)
             prefetch_tmap(&tmV);
         }
         const uint64_t pol = policy_evict_first();
-        const int slot0 = t_begin / kPageRows;
-        int window = -1;      // index of the 32-slot window held in `pg`
-        int pg = 0;
-        int issued = 0;
-        for (int s = 0; s < nstage; ++s, ++issued) {
-            const int st = s % NS;
-            const uint32_t ph = (s / NS) & 1;
-            const int sbase = slot0 + s * (kDecStageTok / kPageRows);
-            const int w = (sbase - slot0) / 32;
-            if (w != window) {
-                window = w;
-                const int slot = slot0 + w * 32 + lane;
-                pg = (slot * kPageRows < t_end && slot < a.max_blocks)
-                         ? a.block_table[(long long)b * a.max_blocks + slot] : 0;
-            }
-            int pages[4];
+        int ctr = 0;       // stages filled so far (ring position and phase)
+        bool ok = true;
+        for (int item = blockIdx.x; ok && item < total; item += gridDim.x) {
+            const DecItem it = dec_item(item, prefix, a.B, a.Hkv, tps, lenv);
+            const int nstage = (it.t_end > it.t_begin)
+                                   ? (it.t_end - it.t_begin + kDecStageTok - 1) / kDecStageTok : 0;
+            const int slot0 = it.t_begin / kPageRows;
+            int window = -1, pg = 0;
+            for (int s = 0; s < nstage; ++s, ++ctr) {
+                const int st = ctr % NS;
+                const uint32_t ph = (ctr / NS) & 1;
+                const int sbase = slot0 + s * (kDecStageTok / kPageRows);
+                const int w = (sbase - slot0) / 32;
+                if (w != window) {
+                    window = w;
+                    const int slot = slot0 + w * 32 + lane;
+                    pg = (slot * kPageRows < it.t_end && slot < a.max_blocks)
+                             ? a.block_table[(long long)it.b * a.max_blocks + slot] : 0;
+                }
+                int pages[4];
 #pragma unroll
-            for (int p = 0; p < 4; ++p) pages[p] = __shfl_sync(0xffffffffu, pg, (sbase - slot0) % 32 + p);
-            bool ok = mbar_wait(&empty[st], ph ^ 1, kErrDecEmpty);
-            ok = __all_sync(0xffffffffu, ok);
-            if (!ok) break;
-            if (lane == 0) {
-                int npv = 0;
+                for (int p = 0; p < 4; ++p) pages[p] = __shfl_sync(0xffffffffu, pg, (sbase - slot0) % 32 + p);
+                ok = mbar_wait(&empty[st], ph ^ 1, kErrDecEmpty);
+                ok = __all_sync(0xffffffffu, ok);
+                if (!ok) break;
+                if (lane == 0) {
+                    int npv = 0;
 #pragma unroll
-                for (int p = 0; p < 4; ++p) npv += ((sbase + p) * kPageRows < t_end) ? 1 : 0;
-                mbar_arrive_expect_tx(&full[st], 2 * npv * kPageRows * C::ROWB);
-                uint8_t* dk = smem + st * C::STAGE;
-                uint8_t* dv = dk + C::STAGE_K;
+                    for (int p = 0; p < 4; ++p) npv += ((sbase + p) * kPageRows < it.t_end) ? 1 : 0;
+                    mbar_arrive_expect_tx(&full[st], 2 * npv * kPageRows * C::ROWB);
+                    uint8_t* dk = smem + st * C::STAGE;
+                    uint8_t* dv = dk + C::STAGE_K;
 #pragma unroll
-                for (int p = 0; p < 4; ++p) {
-                    if ((sbase + p) * kPageRows >= t_end) continue;
+                    for (int p = 0; p < 4; ++p) {
+                        if ((sbase + p) * kPageRows >= it.t_end) continue;
 #pragma unroll
-                    for (int c = 0; c < C::NCHUNK; ++c) {
-                        const int off = c * kDecStageTok * 128 + p * kPageRows * 128;
-                        tma_load_4d_hint(&tmK, &full[st], dk + off, c * 64, g, pages[p] * kPageRows, 0, pol);
-                        tma_load_4d_hint(&tmV, &full[st], dv + off, c * 64, g, pages[p] * kPageRows, 0, pol);
+                        for (int c = 0; c < C::NCHUNK; ++c) {
+                            const int off = c * kDecStageTok * 128 + p * kPageRows * 128;
+                            tma_load_4d_hint(&tmK, &full[st], dk + off, c * 64, it.g,
+                                             pages[p] * kPageRows, 0, pol);
+                            tma_load_4d_hint(&tmV, &full[st], dv + off, c * 64, it.g,
+                                             pages[p] * kPageRows, 0, pol);
+                        }
                     }
                 }
             }
         }
+        // Every copy started must land before the CTA exits.
         if (lane == 0) {
-            for (int st = 0; st < NS && st < issued; ++st) {
-                const int last = st + ((issued - 1 - st) / NS) * NS;
+            for (int st = 0; st < NS && st < ctr; ++st) {
+                const int last = st + ((ctr - 1 - st) / NS) * NS;
                 mbar_wait(&full[st], (last / NS) & 1, kErrDecFull);
             }
         }
@@ -148,205 +229,229 @@ __global__ void __launch_bounds__(kDecThreads, 2)
         // ---------------------------------------------------- consumers (a4-a6 for one token)
         const int gid = lane >> 2, t4 = lane & 3;
         const float sl2 = a.scale * kLog2e;
-        // Q fragments (rows = the G query heads of KV head g; rows >= G are zero).
-        uint32_t qa[D / 16][4];
-        {
-            const __nv_bfloat16* qb = a.q + ((long long)b * a.Hq + (long long)g * a.group) * D;
-#pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-                const int c0 = kk * 16 + 2 * t4;
-                auto ld = [&](int row, int col) -> uint32_t {
-                    if (row >= a.group) return 0u;
-                    return *reinterpret_cast<const uint32_t*>(qb + (long long)row * D + col);
-                };
-                qa[kk][0] = ld(gid, c0);
-                qa[kk][1] = ld(gid + 8, c0);
-                qa[kk][2] = ld(gid, c0 + 8);
-                qa[kk][3] = ld(gid + 8, c0 + 8);
-            }
-        }
-        float o[D / 8][4];
-#pragma unroll
-        for (int i = 0; i < D / 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.0f;
-        float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.0f, l1 = 0.0f;   // rows gid, gid+8
+        int ctr = 0;
         bool ok = true;
-        for (int s = 0; s < nstage; ++s) {
-            const int st = s % NS;
-            ok = mbar_wait(&full[st], (s / NS) & 1, kErrDecFull);
-            ok = __all_sync(0xffffffffu, ok);
-            if (!ok) break;
-            const int tok0 = t_begin + s * kDecStageTok + warp * 16;   // this warp's 16 keys
-            uint8_t* sk = smem + st * C::STAGE;
-            uint8_t* sv = sk + C::STAGE_K;
-            const int lrow0 = warp * 16;                                  // row within the stage
-            if (tok0 < t_end) {
-                if (tok0 + 16 > t_end) {
-                    // Zero the V rows past the end of the sequence (not data of it).
-                    for (int i = lane; i < 16 * (D / 8); i += 32) {
-                        const int rr = i / (D / 8), cc = (i % (D / 8)) * 8;
-                        if (tok0 + rr >= t_end)
-                            *reinterpret_cast<uint4*>(sv + swz_off<D>(lrow0 + rr, cc, kDecStageTok)) =
-                                make_uint4(0, 0, 0, 0);
-                    }
-                    __syncwarp();
-                }
-                // S = Q K^T for 16 keys: two n-tiles of 8 keys.
-                float sc[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}};
-                const uint32_t skb = smem_u32(sk);
+        for (int item = blockIdx.x; item < total; item += gridDim.x) {
+            const DecItem it = dec_item(item, prefix, a.B, a.Hkv, tps, lenv);
+            const int nstage = (it.t_end > it.t_begin)
+                                   ? (it.t_end - it.t_begin + kDecStageTok - 1) / kDecStageTok : 0;
+            // Q fragments (rows = the G query heads of KV head g; rows >= G are zero).
+            uint32_t qa[D / 16][4];
+            {
+                const __nv_bfloat16* qb = a.q + ((long long)it.b * a.Hq + (long long)it.g * G) * D;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const int mi = lane >> 3, ri = lane & 7;
-                    const int row = lrow0 + (mi >> 1) * 8 + ri;
-                    const int col = kk * 16 + (mi & 1) * 8;
-                    uint32_t b0, b1, b2, b3;
-                    ldmatrix_x4(skb + swz_off<D>(row, col, kDecStageTok), b0, b1, b2, b3);
-                    mma_bf16_16816(sc[0], qa[kk], b0, b1);
-                    mma_bf16_16816(sc[1], qa[kk], b2, b3);
+                    const int c0 = kk * 16 + 2 * t4;
+                    auto ld = [&](int row, int col) -> uint32_t {
+                        if (row >= G) return 0u;
+                        return __ldg(reinterpret_cast<const unsigned int*>(qb + (long long)row * D + col));
+                    };
+                    qa[kk][0] = ld(gid, c0);
+                    qa[kk][1] = ld(gid + 8, c0);
+                    qa[kk][2] = ld(gid, c0 + 8);
+                    qa[kk][3] = ld(gid + 8, c0 + 8);
                 }
-                // mask keys past the end, online softmax per row
-                float mx0 = -INFINITY, mx1 = -INFINITY;
+            }
+            float o[D / 8][4];
 #pragma unroll
-                for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        const int kv = tok0 + nt * 8 + 2 * t4 + e;
-                        if (kv >= t_end) { sc[nt][e] = -INFINITY; sc[nt][2 + e] = -INFINITY; }
-                        mx0 = fmaxf(mx0, sc[nt][e]);
-                        mx1 = fmaxf(mx1, sc[nt][2 + e]);
+            for (int i = 0; i < D / 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.0f;
+            float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.0f, l1 = 0.0f;   // rows gid, gid+8
+            for (int s = 0; s < nstage; ++s, ++ctr) {
+                const int st = ctr % NS;
+                if (ok) {
+                    ok = mbar_wait(&full[st], (ctr / NS) & 1, kErrDecFull);
+                    ok = __all_sync(0xffffffffu, ok);
+                }
+                const int tok0 = it.t_begin + s * kDecStageTok + warp * 16;   // this warp's 16 keys
+                uint8_t* sk = smem + st * C::STAGE;
+                uint8_t* sv = sk + C::STAGE_K;
+                const int lrow0 = warp * 16;
+                if (ok && tok0 < it.t_end) {
+                    if (tok0 + 16 > it.t_end) {
+                        // Zero the V rows past the end of the sequence (not data of it).
+                        for (int i = lane; i < 16 * (D / 8); i += 32) {
+                            const int rr = i / (D / 8), cc = (i % (D / 8)) * 8;
+                            if (tok0 + rr >= it.t_end)
+                                *reinterpret_cast<uint4*>(sv + swz_off<D>(lrow0 + rr, cc, kDecStageTok)) =
+                                    make_uint4(0, 0, 0, 0);
+                        }
+                        __syncwarp();
                     }
-                mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
-                mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
-                mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-                mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-                const float mn0 = fmaxf(m0, mx0 * sl2), mn1 = fmaxf(m1, mx1 * sl2);
-                // m = -inf (nothing seen yet) -> alpha 0; both -inf -> 1 (avoid -inf - -inf)
-                const float al0 = (mn0 == -INFINITY) ? 1.0f : ex2(m0 - mn0);
-                const float al1 = (mn1 == -INFINITY) ? 1.0f : ex2(m1 - mn1);
-                m0 = mn0;
-                m1 = mn1;
-                l0 *= al0;
-                l1 *= al1;
+                    // S = Q K^T for 16 keys: two n-tiles of 8 keys.
+                    float sc[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}};
+                    const uint32_t skb = smem_u32(sk);
 #pragma unroll
-                for (int i = 0; i < D / 8; ++i) {
-                    o[i][0] *= al0;
-                    o[i][1] *= al0;
-                    o[i][2] *= al1;
-                    o[i][3] *= al1;
-                }
-                const float mu0 = (m0 == -INFINITY) ? 0.0f : m0;
-                const float mu1 = (m1 == -INFINITY) ? 0.0f : m1;
-                float p[2][4];
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const int mi = lane >> 3, ri = lane & 7;
+                        const int row = lrow0 + (mi >> 1) * 8 + ri;
+                        const int col = kk * 16 + (mi & 1) * 8;
+                        uint32_t b0, b1, b2, b3;
+                        ldmatrix_x4(skb + swz_off<D>(row, col, kDecStageTok), b0, b1, b2, b3);
+                        mma_bf16_16816(sc[0], qa[kk], b0, b1);
+                        mma_bf16_16816(sc[1], qa[kk], b2, b3);
+                    }
+                    float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
-                for (int nt = 0; nt < 2; ++nt) {
-                    p[nt][0] = ex2(fmaf(sc[nt][0], sl2, -mu0));
-                    p[nt][1] = ex2(fmaf(sc[nt][1], sl2, -mu0));
-                    p[nt][2] = ex2(fmaf(sc[nt][2], sl2, -mu1));
-                    p[nt][3] = ex2(fmaf(sc[nt][3], sl2, -mu1));
-                    l0 += p[nt][0] + p[nt][1];
-                    l1 += p[nt][2] + p[nt][3];
-                }
-                uint32_t pa[4];
-                pa[0] = pack_bf16(p[0][0], p[0][1]);
-                pa[1] = pack_bf16(p[0][2], p[0][3]);
-                pa[2] = pack_bf16(p[1][0], p[1][1]);
-                pa[3] = pack_bf16(p[1][2], p[1][3]);
-                // O += P V over the 16 keys
-                const uint32_t svb = smem_u32(sv);
+                    for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-                for (int nd = 0; nd < D / 8; nd += 2) {
-                    const int mi = lane >> 3, ri = lane & 7;
-                    const int row = lrow0 + (mi & 1) * 8 + ri;
-                    const int col = nd * 8 + (mi >> 1) * 8;
-                    uint32_t b0, b1, b2, b3;
-                    ldmatrix_x4_trans(svb + swz_off<D>(row, col, kDecStageTok), b0, b1, b2, b3);
-                    mma_bf16_16816(o[nd], pa, b0, b1);
-                    mma_bf16_16816(o[nd + 1], pa, b2, b3);
+                        for (int e = 0; e < 2; ++e) {
+                            const int kv = tok0 + nt * 8 + 2 * t4 + e;
+                            if (kv >= it.t_end) { sc[nt][e] = -INFINITY; sc[nt][2 + e] = -INFINITY; }
+                            mx0 = fmaxf(mx0, sc[nt][e]);
+                            mx1 = fmaxf(mx1, sc[nt][2 + e]);
+                        }
+                    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+                    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+                    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+                    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+                    const float mn0 = fmaxf(m0, mx0 * sl2), mn1 = fmaxf(m1, mx1 * sl2);
+                    // m = -inf (nothing seen yet) -> alpha 0; both -inf -> 1
+                    const float al0 = (mn0 == -INFINITY) ? 1.0f : ex2(m0 - mn0);
+                    const float al1 = (mn1 == -INFINITY) ? 1.0f : ex2(m1 - mn1);
+                    m0 = mn0;
+                    m1 = mn1;
+                    l0 *= al0;
+                    l1 *= al1;
+#pragma unroll
+                    for (int i = 0; i < D / 8; ++i) {
+                        o[i][0] *= al0;
+                        o[i][1] *= al0;
+                        o[i][2] *= al1;
+                        o[i][3] *= al1;
+                    }
+                    const float mu0 = (m0 == -INFINITY) ? 0.0f : m0;
+                    const float mu1 = (m1 == -INFINITY) ? 0.0f : m1;
+                    float p[2][4];
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt) {
+                        p[nt][0] = ex2(fmaf(sc[nt][0], sl2, -mu0));
+                        p[nt][1] = ex2(fmaf(sc[nt][1], sl2, -mu0));
+                        p[nt][2] = ex2(fmaf(sc[nt][2], sl2, -mu1));
+                        p[nt][3] = ex2(fmaf(sc[nt][3], sl2, -mu1));
+                        l0 += p[nt][0] + p[nt][1];
+                        l1 += p[nt][2] + p[nt][3];
+                    }
+                    uint32_t pa[4];
+                    pa[0] = pack_bf16(p[0][0], p[0][1]);
+                    pa[1] = pack_bf16(p[0][2], p[0][3]);
+                    pa[2] = pack_bf16(p[1][0], p[1][1]);
+                    pa[3] = pack_bf16(p[1][2], p[1][3]);
+                    const uint32_t svb = smem_u32(sv);
+#pragma unroll
+                    for (int nd = 0; nd < D / 8; nd += 2) {
+                        const int mi = lane >> 3, ri = lane & 7;
+                        const int row = lrow0 + (mi & 1) * 8 + ri;
+                        const int col = nd * 8 + (mi >> 1) * 8;
+                        uint32_t b0, b1, b2, b3;
+                        ldmatrix_x4_trans(svb + swz_off<D>(row, col, kDecStageTok), b0, b1, b2, b3);
+                        mma_bf16_16816(o[nd], pa, b0, b1);
+                        mma_bf16_16816(o[nd + 1], pa, b2, b3);
+                    }
                 }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[st]);
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[st]);
-        }
-        // row sums: reduce over the quad
-        l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
-        l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
-        l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
-        l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+            // row sums over the quad
+            l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+            l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+            l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+            l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
 
-        // ---------------------------------------------------- merge the 4 warps
-        asm volatile("bar.sync 1, 128;" ::: "memory");   // all consumers done with the stages
-        float* mo = reinterpret_cast<float*>(smem);                 // [4][16][D]
-        float* mm = mo + 4 * kDecRows * D;                          // [4][16]
-        float* ml = mm + 4 * kDecRows;                              // [4][16]
+            // ------------------------------------------------ merge the 4 warps (own smem area)
+            asm volatile("bar.sync 1, 128;" ::: "memory");   // previous item's readers are done
 #pragma unroll
-        for (int i = 0; i < D / 8; ++i) {
-            const int col = i * 8 + 2 * t4;
-            mo[(warp * kDecRows + gid) * D + col] = o[i][0];
-            mo[(warp * kDecRows + gid) * D + col + 1] = o[i][1];
-            mo[(warp * kDecRows + gid + 8) * D + col] = o[i][2];
-            mo[(warp * kDecRows + gid + 8) * D + col + 1] = o[i][3];
-        }
-        if (t4 == 0) {
-            mm[warp * kDecRows + gid] = m0;
-            mm[warp * kDecRows + gid + 8] = m1;
-            ml[warp * kDecRows + gid] = l0;
-            ml[warp * kDecRows + gid + 8] = l1;
-        }
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        const int G = a.group;
-        for (int idx = threadIdx.x; idx < G * D; idx += 128) {
-            const int row = idx / D, col = idx % D;
-            float M = -INFINITY;
-#pragma unroll
-            for (int w = 0; w < 4; ++w) M = fmaxf(M, mm[w * kDecRows + row]);
-            float acc = 0.0f, l = 0.0f;
-            if (M != -INFINITY) {
-#pragma unroll
-                for (int w = 0; w < 4; ++w) {
-                    const float f = ex2(mm[w * kDecRows + row] - M);
-                    acc += f * mo[(w * kDecRows + row) * D + col];
-                    l += f * ml[w * kDecRows + row];
+            for (int i = 0; i < D / 8; ++i) {
+                const int col = i * 8 + 2 * t4;
+                if (gid < G) {
+                    *reinterpret_cast<float2*>(&mo[(warp * G + gid) * D + col]) =
+                        make_float2(o[i][0], o[i][1]);
+                }
+                if (gid + 8 < G) {
+                    *reinterpret_cast<float2*>(&mo[(warp * G + gid + 8) * D + col]) =
+                        make_float2(o[i][2], o[i][3]);
                 }
             }
-            const int h = g * G + row;
-            const float on = (l > 0.0f) ? acc / l : 0.0f;
-            const float lse = (l > 0.0f) ? (M + log2f(l)) * kLn2 : -INFINITY;
-            if (a.direct) {
-                a.o[((long long)b * a.Hq + h) * D + col] = __float2bfloat16_rn(on);
-                if (col == 0 && a.lse) a.lse[(long long)b * a.Hq + h] = lse;
-            } else {
-                const long long base = ((long long)split * a.B + b) * a.Hq + h;
-                a.o_part[base * D + col] = on;
-                if (col == 0) a.lse_part[base] = lse;
+            if (t4 == 0) {
+                mm[warp * kDecRows + gid] = m0;
+                mm[warp * kDecRows + gid + 8] = m1;
+                ml[warp * kDecRows + gid] = l0;
+                ml[warp * kDecRows + gid + 8] = l1;
+            }
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            for (int idx = threadIdx.x; idx < G * D; idx += 128) {
+                const int row = idx / D, col = idx % D;
+                float M = -INFINITY;
+#pragma unroll
+                for (int w = 0; w < 4; ++w) M = fmaxf(M, mm[w * kDecRows + row]);
+                float acc = 0.0f, l = 0.0f;
+                if (M != -INFINITY) {
+#pragma unroll
+                    for (int w = 0; w < 4; ++w) {
+                        const float f = ex2(mm[w * kDecRows + row] - M);
+                        acc += f * mo[(w * G + row) * D + col];
+                        l += f * ml[w * kDecRows + row];
+                    }
+                }
+                const int h = it.g * G + row;
+                const float on = (l > 0.0f) ? acc / l : 0.0f;
+                const float lse = (l > 0.0f) ? (M + log2f(l)) * kLn2 : -INFINITY;
+                if (a.direct) {
+                    a.o[((long long)it.b * a.Hq + h) * D + col] = __float2bfloat16_rn(on);
+                    if (col == 0 && a.lse) a.lse[(long long)it.b * a.Hq + h] = lse;
+                } else {
+                    const long long base = ((long long)it.split * a.B + it.b) * a.Hq + h;
+                    a.o_part[base * D + col] = on;
+                    if (col == 0) a.lse_part[base] = lse;
+                }
             }
         }
     }
 }
 
 // Merge of the split partials (a9): one block per (sequence, query head).
+// Warp 0 reads every split's LSE at once and turns them into weights
+// w_s = exp(LSE_s - LSE) in shared memory; then each thread (one per d) sums
+// w_s * O_s[d] with all of its loads in flight together.
+constexpr int kMaxSplits = 256;
+
 template <int D>
 __global__ void __launch_bounds__(D)
     decode_combine_kernel(const float* __restrict__ o_part, const float* __restrict__ lse_part,
                           const int* __restrict__ seqused_k, int B, int Hq, int num_splits,
-                          int tokens_per_split, int max_tokens, __nv_bfloat16* __restrict__ o, float* __restrict__ lse) {
+                          int tokens_per_split, int max_tokens, __nv_bfloat16* __restrict__ o,
+                          float* __restrict__ lse) {
+    __shared__ float w_s[kMaxSplits];
+    __shared__ float lse_s;
+    // Launched early (programmatic dependent launch): wait here for the split grid.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int bh = blockIdx.x;
     const int b = bh / Hq;
     const int d = threadIdx.x;
     const int L = min(max(seqused_k[b], 0), max_tokens);
     const int ns = min(num_splits, (L + tokens_per_split - 1) / tokens_per_split);
-    float M = -INFINITY;
-    for (int s = 0; s < ns; ++s) M = fmaxf(M, lse_part[(long long)s * B * Hq + bh]);
-    float acc = 0.0f, out_lse = -INFINITY;
-    if (M != -INFINITY) {
+    const long long stride = (long long)B * Hq;
+    if (threadIdx.x < 32) {
+        const int lane = threadIdx.x;
+        float M = -INFINITY;
+        for (int s = lane; s < ns; s += 32) M = fmaxf(M, lse_part[s * stride + bh]);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
         float W = 0.0f;
-        for (int s = 0; s < ns; ++s) W += __expf(lse_part[(long long)s * B * Hq + bh] - M);
-        out_lse = M + __logf(W);
-        for (int s = 0; s < ns; ++s) {
-            const float w = __expf(lse_part[(long long)s * B * Hq + bh] - out_lse);
-            acc += w * o_part[((long long)s * B * Hq + bh) * D + d];
-        }
+        if (M != -INFINITY)
+            for (int s = lane; s < ns; s += 32) W += __expf(lse_part[s * stride + bh] - M);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) W += __shfl_xor_sync(0xffffffffu, W, off);
+        const float out_lse = (M != -INFINITY && W > 0.0f) ? M + __logf(W) : -INFINITY;
+        for (int s = lane; s < ns; s += 32)
+            w_s[s] = (out_lse == -INFINITY) ? 0.0f : __expf(lse_part[s * stride + bh] - out_lse);
+        if (lane == 0) lse_s = out_lse;
     }
+    __syncthreads();
+    float acc = 0.0f;
+#pragma unroll 8
+    for (int s = 0; s < ns; ++s) acc += w_s[s] * o_part[(s * stride + bh) * D + d];
     o[(long long)bh * D + d] = __float2bfloat16_rn(acc);
-    if (lse && d == 0) lse[bh] = out_lse;
+    if (lse && d == 0) lse[bh] = lse_s;
 }
 
 }  // namespace attn

@@ -470,14 +470,14 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             tc_fence_after();
             float s[kBN];
             {
-                uint32_t u[32];
+                // All four column blocks in flight, one wait.
+                uint32_t u[kBN];
 #pragma unroll
-                for (int c4 = 0; c4 < kBN / 32; ++c4) {
-                    tmem_ld32(tS + c4 * 32, u);
-                    tmem_wait_ld();
+                for (int c4 = 0; c4 < kBN / 32; ++c4)
+                    tmem_ld32(tS + c4 * 32, *reinterpret_cast<uint32_t(*)[32]>(&u[c4 * 32]));
+                tmem_wait_ld();
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) s[c4 * 32 + c] = __uint_as_float(u[c]);
-                }
+                for (int c = 0; c < kBN; ++c) s[c] = __uint_as_float(u[c]);
             }
             const int kbase = j * kBN;
             if (kbase < klo || kbase + kBN > khi) {
@@ -487,9 +487,19 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                     s[c] = (kv >= klo && kv < khi) ? s[c] : -INFINITY;
                 }
             }
-            float mx = -INFINITY;
+            // Row max as 8 independent chains (short dependency depth).
+            float mx;
+            {
+                float m8[8];
 #pragma unroll
-            for (int c = 0; c < kBN; ++c) mx = fmaxf(mx, s[c]);
+                for (int i = 0; i < 8; ++i) m8[i] = s[i];
+#pragma unroll
+                for (int c = 8; c < kBN; c += 8)
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) m8[i] = fmaxf(m8[i], s[c + i]);
+                mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                           fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+            }
             const float m_new = fmaxf(m_run, mx * sl2);
             const bool want = m_new > m_run + kRescaleThreshold;
             float alpha = 1.0f;
@@ -499,7 +509,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                 m_run = m_new;
             }
             const float mu = (m_run == -INFINITY) ? 0.0f : m_run;
-            float sum = 0.0f;
+            float sums[4] = {0.0f, 0.0f, 0.0f, 0.0f};
             __syncwarp();
             // P overwrites the first columns of S in TMEM, 32 keys at a time.
 #pragma unroll
@@ -512,7 +522,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                         const float p1 = ex2(fmaf(s[c4 * 32 + 4 * c + 1], sl2, -mu));
                         const float p2 = ex2(fmaf(s[c4 * 32 + 4 * c + 2], sl2, -mu));
                         const float p3 = ex2(fmaf(s[c4 * 32 + 4 * c + 3], sl2, -mu));
-                        sum += (p0 + p1) + (p2 + p3);
+                        sums[0] += p0;
+                        sums[1] += p1;
+                        sums[2] += p2;
+                        sums[3] += p3;
                         pk[c] = pack_e4m3x4(p0, p1, p2, p3);
                     }
                     tmem_st8(tS + c4 * 8, pk);
@@ -522,12 +535,14 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                     for (int c = 0; c < 16; ++c) {
                         const float p0 = ex2(fmaf(s[c4 * 32 + 2 * c + 0], sl2, -mu));
                         const float p1 = ex2(fmaf(s[c4 * 32 + 2 * c + 1], sl2, -mu));
-                        sum += p0 + p1;
+                        sums[(2 * c) & 3] += p0;
+                        sums[(2 * c + 1) & 3] += p1;
                         pk[c] = pack_bf16(p0, p1);
                     }
                     tmem_st16(tS + c4 * 16, pk);
                 }
             }
+            const float sum = (sums[0] + sums[1]) + (sums[2] + sums[3]);
             if (jj > 0 && __any_sync(0xffffffffu, want)) {
                 // O holds the sum over earlier tiles (their P.V MMAs completed
                 // before this tile's S was committed); rescale this row.

@@ -48,6 +48,9 @@ def parse_args():
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-prefill", action="store_true")
+    p.add_argument("--workload", choices=["all", "decode", "prefill", "fp8"], default="all",
+                   help="run only one workload (profiling runs); the JSON line then carries "
+                        "only what ran")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--seed", type=int, default=0)
     return p.parse_args()
@@ -279,6 +282,22 @@ def run_ours(args, rank, world, local):
     peaks, peak_kind = load_peaks()
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
 
+    line = {"metric": METRIC, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16"}
+    if args.workload in ("all", "decode"):
+        w = run_decode(args, A, W, dev, world, flush, peaks, peak_kind, line)
+    if args.workload in ("all", "prefill") and not args.no_prefill:
+        run_prefill(args, A, W, dev, world, flush, peaks, peak_kind, line)
+    if args.workload in ("all", "fp8") and not args.no_prefill:
+        run_fp8(args, A, W, dev, world, flush, peaks, peak_kind, line)
+    if args.workload in ("all", "decode") and rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_decode(args, A, W, dev, world, flush, peaks, peak_kind, line):
     # ---------------- decode (primary)
     w = W.paged_decode(seed=args.seed)
     t = w.tensors
@@ -328,10 +347,8 @@ def run_ours(args, rank, world, local):
     h2d = qh.numel() * 2 + bth.numel() * 4 + suh.numel() * 4
     d2h = oh.numel() * 2 + lh.numel() * 4
 
-    line = {
-        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_max, 5),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+    line.update({
+        "value": round(value, 2), "ms_per_step": round(ms_max, 5),
         "data": "synthetic: seeded N(0,1) bf16 q/k/v, uniform kv lengths, permuted page pool",
         "config": {"workload": "paged_gqa_decode_bf16: B=32 x 1 query token, Hq=32, Hkv=8, "
                                "D=128, 16-token pages, kv len ~ U[1,8192] (seed %d: %d keys), "
@@ -353,94 +370,95 @@ def run_ours(args, rank, world, local):
                         "copied in and O, LSE copied out every step"},
         "gpu_launches": args.steps * ns,
         "clocks": clocks,
-    }
+    })
+    return w
 
+
+def run_prefill(args, A, W, dev, world, flush, peaks, peak_kind, line):
     # ---------------- prefill (carried in the same line)
-    if not args.no_prefill:
-        del d
-        wp = W.varlen_paged_prefill(seed=args.seed)
-        tp, Pp = wp.tensors, wp.params
-        dp = {k: v.to(dev) for k, v in tp.items()}
-        op = torch.empty(Pp["total_q"], Pp["Hq"], Pp["D"], dtype=torch.bfloat16, device=dev)
-        lp = torch.empty(Pp["Hq"], Pp["total_q"], dtype=torch.float32, device=dev)
+    wp = W.varlen_paged_prefill(seed=args.seed)
+    tp, Pp = wp.tensors, wp.params
+    dp = {k: v.to(dev) for k, v in tp.items()}
+    op = torch.empty(Pp["total_q"], Pp["Hq"], Pp["D"], dtype=torch.bfloat16, device=dev)
+    lp = torch.empty(Pp["Hq"], Pp["total_q"], dtype=torch.float32, device=dev)
 
-        def pf_step():
-            A.attn_fwd_varlen_paged(dp["q"], dp["k_cache"], dp["v_cache"],
-                                    cu_seqlens_q=dp["cu_seqlens_q"], max_seqlen_q=Pp["max_seqlen_q"],
-                                    block_table=dp["block_table"], seqused_k=dp["seqused_k"],
-                                    mask=A.MASK_CAUSAL, scale=Pp["scale"], out=op, lse=lp)
+    def pf_step():
+        A.attn_fwd_varlen_paged(dp["q"], dp["k_cache"], dp["v_cache"],
+                                cu_seqlens_q=dp["cu_seqlens_q"], max_seqlen_q=Pp["max_seqlen_q"],
+                                block_table=dp["block_table"], seqused_k=dp["seqused_k"],
+                                mask=A.MASK_CAUSAL, scale=Pp["scale"], out=op, lse=lp)
 
-        pt = time_steps(pf_step, args.steps, args.warmup, world, flush)
-        pms = statistics.mean(pt)
-        flops = causal_flops(tp["seqused_k"].numpy(), Pp["Hq"], Pp["D"])
-        tf = flops / (pms * 1e-3) / 1e12
-        line["prefill"] = {
-            "workload": "varlen_paged_gqa_prefill_causal_bf16: 16 seqs, q len = kv len ~ "
-                        "U[64,4096] (seed %d: %d tokens), Hq=32, Hkv=8, D=128, 16-token pages"
-                        % (args.seed, Pp["total_q"]),
-            "value": round(tf, 2), "unit": "TFLOP/s", "ms_per_step": round(pms, 5),
-            "flops_per_step": flops,
-            "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": peaks["bf16_tflops"],
-                         "unit": "TFLOP/s", "frac": round(tf / peaks["bf16_tflops"], 4),
-                         "traffic": None, "kernel": "prefill_kernel<128,bf16>",
-                         "peak_kind": peak_kind},
-        }
-        line["gpu_launches"] += 0   # prefill runs outside the primary timed region
-        del dp
+    pt = time_steps(pf_step, args.steps, args.warmup, world, flush)
+    pms = statistics.mean(pt)
+    flops = causal_flops(tp["seqused_k"].numpy(), Pp["Hq"], Pp["D"])
+    tf = flops / (pms * 1e-3) / 1e12
+    line["prefill"] = {
+        "workload": "varlen_paged_gqa_prefill_causal_bf16: 16 seqs, q len = kv len ~ "
+                    "U[64,4096] (seed %d: %d tokens), Hq=32, Hkv=8, D=128, 16-token pages"
+                    % (args.seed, Pp["total_q"]),
+        "value": round(tf, 2), "unit": "TFLOP/s", "ms_per_step": round(pms, 5),
+        "flops_per_step": flops,
+        "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": peaks["bf16_tflops"],
+                     "unit": "TFLOP/s", "frac": round(tf / peaks["bf16_tflops"], 4),
+                     "traffic": None, "kernel": "prefill_kernel<128,bf16>",
+                     "peak_kind": peak_kind},
+    }
+    del dp
 
-        w8 = W.fp8_dense_causal(seed=args.seed)
-        t8 = w8.tensors
-        d8 = {k: v.to(dev) for k, v in t8.items()}
-        o8 = torch.empty(4, 4096, 16, 128, dtype=torch.bfloat16, device=dev)
-        l8 = torch.empty(4, 16, 4096, dtype=torch.float32, device=dev)
 
-        def f8_step():
-            A.attn_fwd_dense(d8["q_fp8"], d8["k_fp8"], d8["v_fp8"], causal=True,
-                             scale=w8.params["scale"], descale_q=d8["descale_q"],
-                             descale_k=d8["descale_k"], descale_v=d8["descale_v"], out=o8, lse=l8)
+def run_fp8(args, A, W, dev, world, flush, peaks, peak_kind, line):
+    w8 = W.fp8_dense_causal(seed=args.seed)
+    t8 = w8.tensors
+    d8 = {k: v.to(dev) for k, v in t8.items()}
+    o8 = torch.empty(4, 4096, 16, 128, dtype=torch.bfloat16, device=dev)
+    l8 = torch.empty(4, 16, 4096, dtype=torch.float32, device=dev)
 
-        def b16_step():
-            A.attn_fwd_dense(d8["q"], d8["k"], d8["v"], causal=True, scale=w8.params["scale"],
-                             out=o8, lse=l8)
+    def f8_step():
+        A.attn_fwd_dense(d8["q_fp8"], d8["k_fp8"], d8["v_fp8"], causal=True,
+                         scale=w8.params["scale"], descale_q=d8["descale_q"],
+                         descale_k=d8["descale_k"], descale_v=d8["descale_v"], out=o8, lse=l8)
 
-        f8ms = statistics.mean(time_steps(f8_step, args.steps, args.warmup, world, flush))
-        b16ms = statistics.mean(time_steps(b16_step, args.steps, args.warmup, world, flush))
-        fl8 = causal_flops([4096] * 4, 16, 128)
-        fp8_peak = 2.0 * peaks["bf16_tflops"]
-        line["prefill_fp8"] = {
-            "workload": "fp8_e4m3_dense_causal: B=4, H=16, L=4096, D=128, per-tensor descale",
-            "value": round(fl8 / (f8ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
-            "ms_per_step": round(f8ms, 5),
-            "bf16_same_data": {"value": round(fl8 / (b16ms * 1e-3) / 1e12, 2),
-                               "ms_per_step": round(b16ms, 5),
-                               "fp8_time_over_bf16_time": round(f8ms / b16ms, 4)},
-            "roofline": {"bound": "tensor", "achieved": round(fl8 / (f8ms * 1e-3) / 1e12, 1),
-                         "peak": fp8_peak, "unit": "TFLOP/s",
-                         "frac": round(fl8 / (f8ms * 1e-3) / 1e12 / fp8_peak, 4), "traffic": None,
-                         "kernel": "prefill_kernel<128,fp8>",
-                         "peak_kind": peak_kind + " bf16 x 2 (nominal fp8/bf16 ratio)"},
-        }
-        del d8
+    def b16_step():
+        A.attn_fwd_dense(d8["q"], d8["k"], d8["v"], causal=True, scale=w8.params["scale"],
+                         out=o8, lse=l8)
 
-    # ---------------- CPU baseline: the oracle on rank 0 at N=1, a bounded sample
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        secs, nb, nseq, tok = 0.0, 0, 0, 0
-        t_start = time.perf_counter()
-        i = 0
-        while time.perf_counter() - t_start < 10.0 and i < 32:
-            dt, b_, n_, tk = oracle_decode_sample(w, target_tokens=8192, offset=i * 3)
-            secs += dt
-            nb += b_
-            nseq += n_
-            tok += tk
-            i += 1
-        line["cpu_baseline"] = {"value": round(nb / secs / 1e9, 4), "unit": "GB/s",
-                                "cores": os.cpu_count() or 1, "kind": "oracle",
-                                "sample": "%d oracle calls over %d whole sequences (%d keys, all "
-                                          "32 heads) of the decode batch" % (i, nseq, tok),
-                                "cpu": cpu_model()}
-    if rank == 0:
-        print(json.dumps(line), flush=True)
+    f8ms = statistics.mean(time_steps(f8_step, args.steps, args.warmup, world, flush))
+    b16ms = statistics.mean(time_steps(b16_step, args.steps, args.warmup, world, flush))
+    fl8 = causal_flops([4096] * 4, 16, 128)
+    fp8_peak = 2.0 * peaks["bf16_tflops"]
+    line["prefill_fp8"] = {
+        "workload": "fp8_e4m3_dense_causal: B=4, H=16, L=4096, D=128, per-tensor descale",
+        "value": round(fl8 / (f8ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+        "ms_per_step": round(f8ms, 5),
+        "bf16_same_data": {"value": round(fl8 / (b16ms * 1e-3) / 1e12, 2),
+                           "ms_per_step": round(b16ms, 5),
+                           "fp8_time_over_bf16_time": round(f8ms / b16ms, 4)},
+        "roofline": {"bound": "tensor", "achieved": round(fl8 / (f8ms * 1e-3) / 1e12, 1),
+                     "peak": fp8_peak, "unit": "TFLOP/s",
+                     "frac": round(fl8 / (f8ms * 1e-3) / 1e12 / fp8_peak, 4), "traffic": None,
+                     "kernel": "prefill_kernel<128,fp8>",
+                     "peak_kind": peak_kind + " bf16 x 2 (nominal fp8/bf16 ratio)"},
+    }
+    del d8
+
+
+def cpu_baseline(w):
+    """The oracle on rank 0 at N=1, a bounded sample (about 10 s) of the decode batch."""
+    secs, nb, nseq, tok = 0.0, 0, 0, 0
+    t_start = time.perf_counter()
+    i = 0
+    while time.perf_counter() - t_start < 10.0 and i < 32:
+        dt, b_, n_, tk = oracle_decode_sample(w, target_tokens=8192, offset=i * 3)
+        secs += dt
+        nb += b_
+        nseq += n_
+        tok += tk
+        i += 1
+    return {"value": round(nb / secs / 1e9, 4), "unit": "GB/s",
+            "cores": os.cpu_count() or 1, "kind": "oracle",
+            "sample": "%d oracle calls over %d whole sequences (%d keys, all "
+                      "32 heads) of the decode batch" % (i, nseq, tok),
+            "cpu": cpu_model()}
 
 
 def main():
