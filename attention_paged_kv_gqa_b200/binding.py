@@ -47,6 +47,8 @@ def lib():
         L.attn_status_string.restype = ctypes.c_char_p
         L.attn_device_error.argtypes = [ctypes.POINTER(I), P]
         L.attn_device_error.restype = I
+        L.attn_selftest_exp2.argtypes = [P, P, I, I, P]
+        L.attn_selftest_exp2.restype = I
         L.attn_fwd_dense.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P, P, P, F, I, I, P, P, P, P]
         L.attn_fwd_dense.restype = I
         L.attn_fwd_varlen_paged.argtypes = [P, P, P, P, I, I, I, P, P, P, I, I, I, I, I, I, I,
@@ -110,6 +112,14 @@ def attn_device_error(stream=None) -> int:
     if st not in (0, 7):
         _check(st, "attn_device_error")
     return code.value
+
+
+def attn_selftest_exp2(x, degree=3, stream=None):
+    """The prefill softmax's FMA-pipe exp2 applied to a device fp32 tensor."""
+    y = torch.empty_like(x)
+    _check(lib().attn_selftest_exp2(_ptr(x), _ptr(y), x.numel(), int(degree), _stream(stream)),
+           "attn_selftest_exp2")
+    return y
 
 
 def attn_fwd_dense(q, k, v, *, causal=False, scale=None, descale_q=None, descale_k=None,

@@ -38,6 +38,21 @@ constexpr int kPageRows = 16;      // paged KV: tokens per page
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only when the max grows by > 2^8
 constexpr float kLn2 = 0.69314718055994531f;
 constexpr float kLog2e = 1.44269504088896341f;
+// Of every 8 softmax exponentials, this many are evaluated by a polynomial on
+// the FMA pipe (exp2_fma) and the rest by the MUFU unit, so that the two run
+// side by side instead of the MUFU unit bounding the tile.
+#ifndef ATTN_EXP2_EMU_OF_8
+#define ATTN_EXP2_EMU_OF_8 0
+#endif
+constexpr int kEmuOf8 = ATTN_EXP2_EMU_OF_8;
+
+// exp2 of element e of a row (e is a constant after unrolling): MUFU or the
+// FMA polynomial.
+template <bool FP8>
+__device__ __forceinline__ float row_exp2(int e, float x) {
+    if ((e & 7) >= 8 - kEmuOf8) return exp2_fma<FP8 ? 2 : 3>(x);
+    return ex2(x);
+}
 
 enum : int { kMaskNone = 0, kMaskCausal = 1, kMaskPatch = 2 };
 
@@ -487,18 +502,17 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                     s[c] = (kv >= klo && kv < khi) ? s[c] : -INFINITY;
                 }
             }
-            // Row max as 8 independent chains (short dependency depth).
+            // Row max: 8 independent chains of three-input max.
             float mx;
             {
                 float m8[8];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) m8[i] = s[i];
+                for (int i = 0; i < 8; ++i) m8[i] = fmaxf(s[i], s[8 + i]);
 #pragma unroll
-                for (int c = 8; c < kBN; c += 8)
+                for (int c = 16; c < kBN; c += 16)
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) m8[i] = fmaxf(m8[i], s[c + i]);
-                mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                           fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+                    for (int i = 0; i < 8; ++i) m8[i] = fmax3(m8[i], s[c + i], s[c + 8 + i]);
+                mx = fmaxf(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], fmax3(m8[5], m8[6], m8[7])));
             }
             const float m_new = fmaxf(m_run, mx * sl2);
             const bool want = m_new > m_run + kRescaleThreshold;
@@ -518,10 +532,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                     uint32_t pk[8];
 #pragma unroll
                     for (int c = 0; c < 8; ++c) {
-                        const float p0 = ex2(fmaf(s[c4 * 32 + 4 * c + 0], sl2, -mu));
-                        const float p1 = ex2(fmaf(s[c4 * 32 + 4 * c + 1], sl2, -mu));
-                        const float p2 = ex2(fmaf(s[c4 * 32 + 4 * c + 2], sl2, -mu));
-                        const float p3 = ex2(fmaf(s[c4 * 32 + 4 * c + 3], sl2, -mu));
+                        const float p0 = row_exp2<FP8>(4 * c + 0, fmaf(s[c4 * 32 + 4 * c + 0], sl2, -mu));
+                        const float p1 = row_exp2<FP8>(4 * c + 1, fmaf(s[c4 * 32 + 4 * c + 1], sl2, -mu));
+                        const float p2 = row_exp2<FP8>(4 * c + 2, fmaf(s[c4 * 32 + 4 * c + 2], sl2, -mu));
+                        const float p3 = row_exp2<FP8>(4 * c + 3, fmaf(s[c4 * 32 + 4 * c + 3], sl2, -mu));
                         sums[0] += p0;
                         sums[1] += p1;
                         sums[2] += p2;
@@ -533,8 +547,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                     uint32_t pk[16];
 #pragma unroll
                     for (int c = 0; c < 16; ++c) {
-                        const float p0 = ex2(fmaf(s[c4 * 32 + 2 * c + 0], sl2, -mu));
-                        const float p1 = ex2(fmaf(s[c4 * 32 + 2 * c + 1], sl2, -mu));
+                        const float p0 = row_exp2<FP8>(2 * c + 0, fmaf(s[c4 * 32 + 2 * c + 0], sl2, -mu));
+                        const float p1 = row_exp2<FP8>(2 * c + 1, fmaf(s[c4 * 32 + 2 * c + 1], sl2, -mu));
                         sums[(2 * c) & 3] += p0;
                         sums[(2 * c + 1) & 3] += p1;
                         pk[c] = pack_bf16(p0, p1);

@@ -352,3 +352,18 @@ def test_config_fp8_dense_causal_full():
                 assert np.max(np.abs(oo[b, i] - ref_o[0])) <= tol_o, (name, b, i)
                 if tol_l is not None:
                     assert np.max(np.abs(ll[b, :, i] - ref_l[:, 0])) <= tol_l, (name, b, i)
+
+
+# ---------------------------------------------------------------------------- building blocks
+@pytest.mark.parametrize("degree,bound", [(3, 1.0e-4), (2, 2.0e-3)])
+def test_fma_pipe_exp2_error_bound(degree, bound):
+    """The softmax's polynomial exp2 stays within its fitted relative-error bound of 2^x."""
+    x = torch.linspace(-60.0, 8.0, 1 << 20, dtype=torch.float32)
+    y = A.attn_selftest_exp2(x.to(DEV), degree=degree).cpu().double()
+    ref = torch.exp2(x.double())
+    rel = ((y - ref).abs() / ref).max().item()
+    assert rel <= bound, rel
+    tiny = A.attn_selftest_exp2(torch.tensor([-float("inf"), -500.0, -125.5, -125.0], device=DEV),
+                                degree).cpu()
+    assert tiny[0] == 0 and tiny[1] == 0 and tiny[2] == 0     # masked scores contribute nothing
+    assert 0 < tiny[3] < 2.0 ** -124
