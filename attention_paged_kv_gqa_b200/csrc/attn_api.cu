@@ -300,6 +300,40 @@ __global__ void exp2_selftest_kernel(const float* __restrict__ x, float* __restr
     if (i < n) y[i] = degree >= 3 ? exp2_fma<3>(x[i]) : exp2_fma<2>(x[i]);
 }
 
+template <int D>
+attn_status_t launch_decode_pages(const CUtensorMap& mk, const CUtensorMap& mv, const DecodePagesArgs& a,
+                                  int grid, cudaStream_t st, __nv_bfloat16* o, float* lse) {
+    static std::atomic<uint64_t> attr_mask{0};   // one bit per device
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const uint64_t bit = 1ull << (dev & 63);
+    if (!(attr_mask.load() & bit)) {
+        const attn_status_t s = set_smem(decode_pages_kernel<D>, 227 * 1024);
+        if (s != ATTN_OK) return s;
+        attr_mask.fetch_or(bit);
+    }
+    const int smem = DecodePagesCfg<D>::smem_bytes(a.Hkv, a.B, a.nstages);
+    decode_pages_kernel<D><<<grid, 32 * (a.Hkv + 1), smem, st>>>(mk, mv, a);
+    attn_status_t s = launch_status();
+    if (s != ATTN_OK) return s;
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(a.B * a.Hq);
+    cfg.blockDim = dim3(D);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, decode_pages_combine_kernel<D>, (const float*)a.o_part,
+                           (const float*)a.lse_part, (const int*)a.meta, a.B, a.Hq, o, lse) != cudaSuccess) {
+        cudaGetLastError();
+        return ATTN_ERR_CUDA;
+    }
+    return ATTN_OK;
+}
+
 }  // namespace
 
 // ==================================================================== C ABI
@@ -526,10 +560,43 @@ static void decode_splits(int B, int Hkv, int max_tokens, int requested, int* nu
     *num_splits = (max_tokens + t - 1) / t;
 }
 
+static int decode_pages_stages(int D, int Hkv, int B) {
+    const int cap = 227 * 1024;
+    int ns = 0;
+    if (D == 128)
+        while (ns < 8 && DecodePagesCfg<128>::smem_bytes(Hkv, B, ns + 1) <= cap) ++ns;
+    else
+        while (ns < 8 && DecodePagesCfg<64>::smem_bytes(Hkv, B, ns + 1) <= cap) ++ns;
+    return ns;
+}
+
+// The page-stream kernel serves the automatic split choice whenever a whole
+// page of all KV heads fits a stage twice over; an explicit num_splits selects
+// the per-(sequence, split, KV head) kernel.
+static bool use_page_stream(int B, int Hq, int Hkv, int D, int num_splits) {
+    return num_splits <= 0 && Hkv <= kPgMaxWarps && Hq / Hkv <= kDecRows && B <= kDecMaxSeqs &&
+           decode_pages_stages(D, Hkv, B) >= 2;
+}
+
+static int current_sm_count_or(int fallback) {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+        cudaGetLastError();
+        return fallback;
+    }
+    return n;
+}
+
 size_t attn_decode_workspace_size(int B, int Hq, int Hkv, int D, int max_blocks_per_seq,
                                   int block_size, int num_splits) {
     if (B <= 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || max_blocks_per_seq <= 0 || block_size <= 0)
         return 0;
+    if (use_page_stream(B, Hq, Hkv, D, num_splits)) {
+        // partial slots (grid + B), their LSEs, then the page prefix table
+        const size_t slots = (size_t)current_sm_count_or(1024) + B;
+        return slots * Hq * (D + 1) * sizeof(float) + (size_t)(B + 2) * sizeof(int) + 64;
+    }
     int ns, tps;
     decode_splits(B, Hkv, max_blocks_per_seq * block_size, num_splits, &ns, &tps);
     if (ns <= 1) return 16;
@@ -563,7 +630,7 @@ attn_status_t attn_decode_paged(const void* q, const void* k_cache, const void* 
     decode_splits(B, Hkv, max_blocks_per_seq * block_size, num_splits, &ns, &tps);
     const size_t need = attn_decode_workspace_size(B, Hq, Hkv, D, max_blocks_per_seq, block_size,
                                                    num_splits);
-    if (ns > 1) {
+    if (ns > 1 && !use_page_stream(B, Hq, Hkv, D, num_splits)) {
         if (!workspace || !aligned16(workspace)) return ATTN_ERR_INVALID_ARG;
         if (workspace_bytes < need) return ATTN_ERR_WORKSPACE_TOO_SMALL;
     }
@@ -573,6 +640,41 @@ attn_status_t attn_decode_paged(const void* q, const void* k_cache, const void* 
     if (B == 0) return ATTN_OK;
 
     CUtensorMap mk, mv;
+    cudaStream_t stp = static_cast<cudaStream_t>(stream);
+    if (use_page_stream(B, Hq, Hkv, D, num_splits)) {
+        // {d, token, head, page} view: one box = a whole page's 128-byte column
+        CUtensorMap pk, pv;
+        const uint64_t rowk = (uint64_t)Hkv * D * 2;
+        const uint64_t pd[4] = {(uint64_t)D, (uint64_t)kPageRows, (uint64_t)Hkv, (uint64_t)num_blocks};
+        const uint64_t ps[3] = {rowk, (uint64_t)D * 2, rowk * kPageRows};
+        const uint32_t pbox[4] = {64, (uint32_t)kPageRows, (uint32_t)Hkv, 1};
+        attn_status_t s;
+        if ((s = get_map(&pk, k_cache, ATTN_BF16, pd, ps, pbox)) != ATTN_OK) return s;
+        if ((s = get_map(&pv, v_cache, ATTN_BF16, pd, ps, pbox)) != ATTN_OK) return s;
+        const int grid = sm_count(dev);
+        const size_t slots = (size_t)grid + B;
+        const size_t need_pg = slots * Hq * (D + 1) * sizeof(float) + (size_t)(B + 2) * sizeof(int);
+        if (!workspace || !aligned16(workspace)) return ATTN_ERR_INVALID_ARG;
+        if (workspace_bytes < need_pg) return ATTN_ERR_WORKSPACE_TOO_SMALL;
+        DecodePagesArgs pa;
+        std::memset(&pa, 0, sizeof(pa));
+        pa.B = B;
+        pa.Hq = Hq;
+        pa.Hkv = Hkv;
+        pa.group = Hq / Hkv;
+        pa.q = static_cast<const __nv_bfloat16*>(q);
+        pa.block_table = block_table;
+        pa.max_blocks = max_blocks_per_seq;
+        pa.seqused_k = seqused_k;
+        pa.scale = resolve_scale(softmax_scale, D);
+        pa.o_part = static_cast<float*>(workspace);
+        pa.lse_part = pa.o_part + slots * Hq * D;
+        pa.meta = reinterpret_cast<int*>(pa.lse_part + slots * Hq);
+        pa.nstages = decode_pages_stages(D, Hkv, B);
+        if (D == 128) return launch_decode_pages<128>(pk, pv, pa, grid, stp, static_cast<__nv_bfloat16*>(o), lse);
+        return launch_decode_pages<64>(pk, pv, pa, grid, stp, static_cast<__nv_bfloat16*>(o), lse);
+    }
+
     const uint64_t rowk = (uint64_t)Hkv * D * 2;
     const uint64_t nrows = (uint64_t)num_blocks * block_size;
     const uint64_t dk4[4] = {(uint64_t)D, (uint64_t)Hkv, nrows, 1};

@@ -26,6 +26,7 @@ constexpr int kDecThreads = 160;      // warps 0-3 consumers, warp 4 producer
 constexpr int kDecStageTok = 64;      // keys per stage (4 pages)
 constexpr int kDecRows = 16;          // MMA rows = query heads of one KV group (padded)
 constexpr int kDecMaxSeqs = 4096;     // sequences per call (on-device item table in smem)
+constexpr int kMaxSplits = 256;       // partials merged per (sequence, head)
 
 struct DecodeArgs {
     int B, Hq, Hkv, group;
@@ -408,11 +409,361 @@ __global__ void __launch_bounds__(kDecThreads, 2)
     }
 }
 
+// ---------------------------------------------------------------------------
+// Page-stream decode: the whole batch's pages, in sequence order, are cut into
+// one contiguous, equal share per CTA (one CTA per SM).  Each page is fetched
+// whole -- all KV heads of its 16 tokens, 16 * Hkv * D * 2 contiguous bytes --
+// by two TMA boxes per tensor through a {d, token, head, page} view, which
+// streams DRAM far faster than one head's 128-byte rows at a head-count stride.
+// Consumer warp h owns KV head h (its G query heads) and keeps that head's
+// online softmax; where a sequence ends or the CTA's share ends it writes the
+// partial (O_s normalised, LSE_s) of (this CTA, that sequence) to slot
+// CTA + sequence, so at most grid + B slots exist.  The combine kernel merges,
+// for each sequence, the slots of the CTAs whose share covered it.
+constexpr int kPgMaxWarps = 8;         // consumer warps (KV heads) of the page-stream kernel
+
+struct DecodePagesArgs {
+    int B, Hq, Hkv, group;
+    const __nv_bfloat16* q;   // [B][Hq][D]
+    const int* block_table;
+    int max_blocks;
+    const int* seqused_k;
+    float scale;
+    float* o_part;            // [grid + B][Hq][D]
+    float* lse_part;          // [grid + B][Hq]
+    int* meta;                // [B + 1] page prefix, then pages per CTA (written by CTA 0)
+    int nstages;
+};
+
+template <int D>
+struct DecodePagesCfg {
+    static constexpr int ROWB = D * 2;
+    static constexpr int NCHUNK = ROWB / 128;
+    // stage = one page of K and V for all heads: 2 * 16 * Hkv * D * 2 bytes
+    __host__ __device__ static constexpr int stage_bytes(int Hkv) { return 2 * kPageRows * Hkv * ROWB; }
+    __host__ __device__ static constexpr int table_bytes(int B) { return ((2 * B + 2) * 4 + 15) / 16 * 16; }
+    __host__ __device__ static constexpr int smem_bytes(int Hkv, int B, int ns) {
+        return 1024 + ns * stage_bytes(Hkv) + table_bytes(B) + 2 * ns * 8;
+    }
+};
+
+template <int D>
+__global__ void __launch_bounds__(32 * (kPgMaxWarps + 1), 1)
+    decode_pages_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                        const DecodePagesArgs a) {
+    using C = DecodePagesCfg<D>;
+    const int NS = a.nstages;
+    const int Hkv = a.Hkv, G = a.group;
+    const int SB = C::stage_bytes(Hkv);
+    const int rows = kPageRows * Hkv;            // rows of one 128-byte column of a stage tensor
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = align1024(smem_raw);
+    int* prefix = reinterpret_cast<int*>(smem + NS * SB);   // [B+1] pages before sequence b
+    int* lenv = prefix + (a.B + 1);                          // [B] keys of sequence b
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + NS * SB + C::table_bytes(a.B));
+    uint64_t* empty = full + NS;
+
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int cap = a.max_blocks * kPageRows;
+    if (warp == 0) {
+        int run = 0;
+        for (int base = 0; base < a.B; base += 32) {
+            const int b = base + lane;
+            int cnt = 0;
+            if (b < a.B) {
+                const int L = min(max(a.seqused_k[b], 0), cap);
+                lenv[b] = L;
+                cnt = (L + kPageRows - 1) / kPageRows;
+            }
+            int incl = cnt;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += v;
+            }
+            if (b < a.B) prefix[b] = run + incl - cnt;
+            run += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (lane == 0) prefix[a.B] = run;
+    }
+    if (threadIdx.x == 32) {
+        for (int i = 0; i < NS; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], Hkv);
+        }
+        fence_mbar_init();
+    }
+    __syncthreads();
+    const int P = prefix[a.B];
+    const int ppc = (P + gridDim.x - 1) / gridDim.x;
+    const int p0 = min(P, blockIdx.x * ppc), p1 = min(P, p0 + ppc);
+    if (blockIdx.x == 0) {
+        for (int b = threadIdx.x; b <= a.B; b += blockDim.x) a.meta[b] = prefix[b];
+        if (threadIdx.x == 0) a.meta[a.B + 1] = ppc;
+    }
+    // sequence containing global page g: largest b with prefix[b] <= g
+    auto seq_of = [&](int g) {
+        int lo = 0, hi = a.B;
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (prefix[mid] <= g) lo = mid; else hi = mid;
+        }
+        return lo;
+    };
+    const int npages = p1 - p0;
+
+    if (warp == Hkv) {
+        // ------------------------------------------------------------ producer: whole pages (a3)
+        if (lane == 0) {
+            prefetch_tmap(&tmK);
+            prefetch_tmap(&tmV);
+        }
+        const uint64_t pol = policy_evict_first();
+        int issued = 0;
+        for (int base = 0; base < npages; base += 32) {
+            // this lane's page of the next 32
+            const int g = p0 + base + lane;
+            int phys = 0;
+            if (base + lane < npages) {
+                const int b = seq_of(g);
+                const int slot = g - prefix[b];
+                phys = a.block_table[(long long)b * a.max_blocks + slot];
+            }
+            const int cnt = min(32, npages - base);
+            bool ok = true;
+            for (int i = 0; i < cnt; ++i, ++issued) {
+                const int page = __shfl_sync(0xffffffffu, phys, i);
+                const int st = issued % NS;
+                ok = mbar_wait(&empty[st], ((issued / NS) & 1) ^ 1, kErrDecEmpty);
+                ok = __all_sync(0xffffffffu, ok);
+                if (!ok) break;
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&full[st], SB);
+                    uint8_t* dk = smem + st * SB;
+                    uint8_t* dv = dk + SB / 2;
+#pragma unroll
+                    for (int c = 0; c < C::NCHUNK; ++c) {
+                        tma_load_4d_hint(&tmK, &full[st], dk + c * rows * 128, c * 64, 0, 0, page, pol);
+                        tma_load_4d_hint(&tmV, &full[st], dv + c * rows * 128, c * 64, 0, 0, page, pol);
+                    }
+                }
+            }
+            if (!ok) break;
+        }
+        if (lane == 0) {
+            for (int st = 0; st < NS && st < issued; ++st) {
+                const int last = st + ((issued - 1 - st) / NS) * NS;
+                mbar_wait(&full[st], (last / NS) & 1, kErrDecFull);
+            }
+        }
+    } else if (warp < Hkv) {
+        // ------------------------------------------------------------ consumer warp = KV head
+        const int h = warp;
+        const int gid = lane >> 2, t4 = lane & 3;
+        const float sl2 = a.scale * kLog2e;
+        uint32_t qa[D / 16][4];
+        float o[D / 8][4];
+        float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.0f, l1 = 0.0f;
+        int b = -1, b_end = 0, L = 0;
+        auto load_q = [&](int bb) {
+            const __nv_bfloat16* qb = a.q + ((long long)bb * a.Hq + (long long)h * G) * D;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const int c0 = kk * 16 + 2 * t4;
+                auto ld = [&](int row, int col) -> uint32_t {
+                    if (row >= G) return 0u;
+                    return __ldg(reinterpret_cast<const unsigned int*>(qb + (long long)row * D + col));
+                };
+                qa[kk][0] = ld(gid, c0);
+                qa[kk][1] = ld(gid + 8, c0);
+                qa[kk][2] = ld(gid, c0 + 8);
+                qa[kk][3] = ld(gid + 8, c0 + 8);
+            }
+        };
+        auto reset = [&]() {
+#pragma unroll
+            for (int i = 0; i < D / 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.0f;
+            m0 = m1 = -INFINITY;
+            l0 = l1 = 0.0f;
+        };
+        // write the partial of (this CTA, sequence b) for this head's G query heads
+        auto flush_partial = [&]() {
+            float s0 = l0, s1 = l1;
+            s0 += __shfl_xor_sync(0xffffffffu, s0, 1);
+            s0 += __shfl_xor_sync(0xffffffffu, s0, 2);
+            s1 += __shfl_xor_sync(0xffffffffu, s1, 1);
+            s1 += __shfl_xor_sync(0xffffffffu, s1, 2);
+            const long long slot = (long long)blockIdx.x + b;
+            const float i0 = s0 > 0.0f ? 1.0f / s0 : 0.0f, i1 = s1 > 0.0f ? 1.0f / s1 : 0.0f;
+#pragma unroll
+            for (int i = 0; i < D / 8; ++i) {
+                const int col = i * 8 + 2 * t4;
+                if (gid < G)
+                    *reinterpret_cast<float2*>(&a.o_part[(slot * a.Hq + h * G + gid) * D + col]) =
+                        make_float2(o[i][0] * i0, o[i][1] * i0);
+                if (gid + 8 < G)
+                    *reinterpret_cast<float2*>(&a.o_part[(slot * a.Hq + h * G + gid + 8) * D + col]) =
+                        make_float2(o[i][2] * i1, o[i][3] * i1);
+            }
+            if (t4 == 0) {
+                if (gid < G) a.lse_part[slot * a.Hq + h * G + gid] = s0 > 0.0f ? (m0 + log2f(s0)) * kLn2 : -INFINITY;
+                if (gid + 8 < G)
+                    a.lse_part[slot * a.Hq + h * G + gid + 8] = s1 > 0.0f ? (m1 + log2f(s1)) * kLn2 : -INFINITY;
+            }
+        };
+        bool ok = true;
+        for (int i = 0; i < npages; ++i) {
+            const int g = p0 + i;
+            if (g >= b_end) {                       // next sequence (skipping empty ones)
+                if (b >= 0) flush_partial();
+                b = seq_of(g);
+                b_end = prefix[b + 1];
+                L = lenv[b];
+                load_q(b);
+                reset();
+            }
+            const int st = i % NS;
+            if (ok) {
+                ok = mbar_wait(&full[st], (i / NS) & 1, kErrDecFull);
+                ok = __all_sync(0xffffffffu, ok);
+            }
+            const int tok0 = (g - prefix[b]) * kPageRows;     // first key of this page
+            uint8_t* sk = smem + st * SB;
+            uint8_t* sv = sk + SB / 2;
+            const int r0 = h * kPageRows;                      // this head's first row in the stage
+            if (ok) {
+                if (tok0 + kPageRows > L) {
+                    // zero this head's V rows past the sequence end (not data of it)
+                    for (int e = lane; e < kPageRows * (D / 8); e += 32) {
+                        const int rr = e / (D / 8), cc = (e % (D / 8)) * 8;
+                        if (tok0 + rr >= L)
+                            *reinterpret_cast<uint4*>(sv + swz_off<D>(r0 + rr, cc, rows)) = make_uint4(0, 0, 0, 0);
+                    }
+                    __syncwarp();
+                }
+                float sc[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}};
+                const uint32_t skb = smem_u32(sk);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const int mi = lane >> 3, ri = lane & 7;
+                    const int row = r0 + (mi >> 1) * 8 + ri;
+                    const int col = kk * 16 + (mi & 1) * 8;
+                    uint32_t b0, b1, b2, b3;
+                    ldmatrix_x4(skb + swz_off<D>(row, col, rows), b0, b1, b2, b3);
+                    mma_bf16_16816(sc[0], qa[kk], b0, b1);
+                    mma_bf16_16816(sc[1], qa[kk], b2, b3);
+                }
+                float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const int kv = tok0 + nt * 8 + 2 * t4 + e;
+                        if (kv >= L) { sc[nt][e] = -INFINITY; sc[nt][2 + e] = -INFINITY; }
+                        mx0 = fmaxf(mx0, sc[nt][e]);
+                        mx1 = fmaxf(mx1, sc[nt][2 + e]);
+                    }
+                mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+                mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+                mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+                mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+                const float mn0 = fmaxf(m0, mx0 * sl2), mn1 = fmaxf(m1, mx1 * sl2);
+                const float al0 = (mn0 == -INFINITY) ? 1.0f : ex2(m0 - mn0);
+                const float al1 = (mn1 == -INFINITY) ? 1.0f : ex2(m1 - mn1);
+                m0 = mn0;
+                m1 = mn1;
+                l0 *= al0;
+                l1 *= al1;
+#pragma unroll
+                for (int k2 = 0; k2 < D / 8; ++k2) {
+                    o[k2][0] *= al0;
+                    o[k2][1] *= al0;
+                    o[k2][2] *= al1;
+                    o[k2][3] *= al1;
+                }
+                const float mu0 = (m0 == -INFINITY) ? 0.0f : m0;
+                const float mu1 = (m1 == -INFINITY) ? 0.0f : m1;
+                float pp[2][4];
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt) {
+                    pp[nt][0] = ex2(fmaf(sc[nt][0], sl2, -mu0));
+                    pp[nt][1] = ex2(fmaf(sc[nt][1], sl2, -mu0));
+                    pp[nt][2] = ex2(fmaf(sc[nt][2], sl2, -mu1));
+                    pp[nt][3] = ex2(fmaf(sc[nt][3], sl2, -mu1));
+                    l0 += pp[nt][0] + pp[nt][1];
+                    l1 += pp[nt][2] + pp[nt][3];
+                }
+                uint32_t pa[4];
+                pa[0] = pack_bf16(pp[0][0], pp[0][1]);
+                pa[1] = pack_bf16(pp[0][2], pp[0][3]);
+                pa[2] = pack_bf16(pp[1][0], pp[1][1]);
+                pa[3] = pack_bf16(pp[1][2], pp[1][3]);
+                const uint32_t svb = smem_u32(sv);
+#pragma unroll
+                for (int nd = 0; nd < D / 8; nd += 2) {
+                    const int mi = lane >> 3, ri = lane & 7;
+                    const int row = r0 + (mi & 1) * 8 + ri;
+                    const int col = nd * 8 + (mi >> 1) * 8;
+                    uint32_t b0, b1, b2, b3;
+                    ldmatrix_x4_trans(svb + swz_off<D>(row, col, rows), b0, b1, b2, b3);
+                    mma_bf16_16816(o[nd], pa, b0, b1);
+                    mma_bf16_16816(o[nd + 1], pa, b2, b3);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[st]);
+        }
+        if (b >= 0) flush_partial();
+    }
+}
+
+// Merge for the page-stream decode: for sequence b, the partials of CTAs
+// c_first .. c_last sit in slots c + b.
+template <int D>
+__global__ void __launch_bounds__(D)
+    decode_pages_combine_kernel(const float* __restrict__ o_part, const float* __restrict__ lse_part,
+                                const int* __restrict__ meta, int B, int Hq,
+                                __nv_bfloat16* __restrict__ o, float* __restrict__ lse) {
+    __shared__ float w_s[kMaxSplits];
+    __shared__ float lse_s;
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    const int bh = blockIdx.x;
+    const int b = bh / Hq, h = bh % Hq;
+    const int d = threadIdx.x;
+    const int ppc = max(meta[B + 1], 1);
+    const int pb = meta[b], pe = meta[b + 1];
+    const int c0 = pb / ppc, c1 = (pe - 1) / ppc;
+    const int ns = (pe > pb) ? min(c1 - c0 + 1, kMaxSplits) : 0;
+    if (threadIdx.x < 32) {
+        const int lane = threadIdx.x;
+        float M = -INFINITY;
+        for (int s = lane; s < ns; s += 32) M = fmaxf(M, lse_part[(long long)(c0 + s + b) * Hq + h]);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+        float W = 0.0f;
+        if (M != -INFINITY)
+            for (int s = lane; s < ns; s += 32) W += __expf(lse_part[(long long)(c0 + s + b) * Hq + h] - M);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) W += __shfl_xor_sync(0xffffffffu, W, off);
+        const float out_lse = (M != -INFINITY && W > 0.0f) ? M + __logf(W) : -INFINITY;
+        for (int s = lane; s < ns; s += 32)
+            w_s[s] = (out_lse == -INFINITY) ? 0.0f
+                                            : __expf(lse_part[(long long)(c0 + s + b) * Hq + h] - out_lse);
+        if (lane == 0) lse_s = out_lse;
+    }
+    __syncthreads();
+    float acc = 0.0f;
+#pragma unroll 4
+    for (int s = 0; s < ns; ++s) acc += w_s[s] * o_part[((long long)(c0 + s + b) * Hq + h) * D + d];
+    o[(long long)bh * D + d] = __float2bfloat16_rn(acc);
+    if (lse && d == 0) lse[bh] = lse_s;
+}
+
 // Merge of the split partials (a9): one block per (sequence, query head).
 // Warp 0 reads every split's LSE at once and turns them into weights
 // w_s = exp(LSE_s - LSE) in shared memory; then each thread (one per d) sums
 // w_s * O_s[d] with all of its loads in flight together.
-constexpr int kMaxSplits = 256;
 
 template <int D>
 __global__ void __launch_bounds__(D)

@@ -472,7 +472,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             klo = max(a.patch[2LL * (q_off + qi)], 0);
             khi = min(a.patch[2LL * (q_off + qi) + 1], Lk);
         }
-        if (!row_ok) { klo = 0; khi = 0; }
+        // Rows past the sequence end are computed like unmasked rows (their
+        // inputs are finite: the next sequence's rows or TMA zero fill) and
+        // never stored; masking them would only slow their warp down.
+        if (!row_ok) { klo = 0; khi = Lk; }
 
         float m_run = -INFINITY, l_run = 0.0f;
         const int n_t = hi_t[t] - lo_t[t];

@@ -367,3 +367,21 @@ def test_fma_pipe_exp2_error_bound(degree, bound):
                                 degree).cpu()
     assert tiny[0] == 0 and tiny[1] == 0 and tiny[2] == 0     # masked scores contribute nothing
     assert 0 < tiny[3] < 2.0 ** -124
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(32, 8), (8, 4), (4, 1), (16, 8)])
+@pytest.mark.parametrize("D", [64, 128])
+def test_decode_page_stream_many_sequences(Hq, Hkv, D):
+    """Automatic (page-stream) decode over many short and long sequences, including
+    empty ones, so CTA shares start and end inside sequences."""
+    lens = [0, 1, 5, 16, 17, 31, 300, 0, 2048, 64, 65, 1000, 7, 129, 3000, 15] * 3
+    w = W.paged_decode(B=len(lens), Hq=Hq, Hkv=Hkv, D=D, num_blocks=2000, lmax=3072, lens=lens,
+                       seed=D + Hq + Hkv)
+    t = w.tensors
+    o, lse = A.attn_decode_paged(t["q"].to(DEV), t["k_cache"].to(DEV), t["v_cache"].to(DEV),
+                                 t["block_table"].to(DEV), t["seqused_k"].to(DEV),
+                                 scale=w.params["scale"])
+    o_ref, lse_ref = oracle.attn_decode(t["q"], t["k_cache"], t["v_cache"], t["block_table"],
+                                        t["seqused_k"], scale=w.params["scale"])
+    _cmp(o, lse, o_ref, lse_ref, TOL_O_BF16, TOL_LSE_BF16, "page-stream decode")
+    _no_device_error()
