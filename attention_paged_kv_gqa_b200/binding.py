@@ -59,6 +59,8 @@ def lib():
         L.attn_decode_paged.argtypes = [P, P, P, P, I, I, I, P, I, I, I, I, F, I, I, P, P, P,
                                         P, P, P, Z, P]
         L.attn_decode_paged.restype = I
+        L.attn_decode_paged_noalloc.argtypes = [P, P, P, P, I, I, I, P, I, I, I, I, F, I, P, P, P]
+        L.attn_decode_paged_noalloc.restype = I
         _lib = L
     return _lib
 
@@ -199,3 +201,24 @@ def attn_decode_paged(q, k_cache, v_cache, block_table, seqused_k, *, scale=None
 
 def default_scale(head_dim: int) -> float:
     return 1.0 / math.sqrt(head_dim)
+
+
+def attn_decode_paged_noalloc(q, k_cache, v_cache, block_table, seqused_k, *, scale=None,
+                              out=None, lse=None, return_lse=True, stream=None):
+    """attn_decode_paged whose split-KV scratch is the library's fixed device array.
+
+    For callers that must not allocate device memory while they run: the C
+    call allocates nothing (the outputs are allocated here only when not given).
+    """
+    B, Hq, D = q.shape
+    num_blocks, block_size, Hkv = k_cache.shape[0], k_cache.shape[1], k_cache.shape[2]
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=torch.bfloat16, device=q.device)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    st = lib().attn_decode_paged_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table),
+                                         block_table.shape[1], num_blocks, block_size,
+                                         _ptr(seqused_k), B, Hq, Hkv, D, _scale(scale),
+                                         _dtype_code(q), _ptr(out), _ptr(lse), _stream(stream))
+    _check(st, "attn_decode_paged_noalloc")
+    return out, lse

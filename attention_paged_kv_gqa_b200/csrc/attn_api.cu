@@ -300,6 +300,33 @@ __global__ void exp2_selftest_kernel(const float* __restrict__ x, float* __restr
     if (i < n) y[i] = degree >= 3 ? exp2_fma<3>(x[i]) : exp2_fma<2>(x[i]);
 }
 
+// ------------------------------------------------------------------ allocation-free decode
+// Fixed device scratch for attn_decode_paged_noalloc.  Every device that loads
+// this library holds these bytes until the process exits.  Host code must not
+// pass the symbol itself to a kernel (on the host it is only a stand-in for the
+// device object); the device address is looked up once per device below.
+constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;   // 8 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+std::atomic<void*> g_noalloc_addr[kMaxDevices];
+std::mutex g_noalloc_mu;
+
+// Device address of the scratch on the current device, resolved on first use
+// (with that device current) and cached.  Returns nullptr on failure.
+void* noalloc_scratch_address(int dev) {
+    if (dev < 0 || dev >= kMaxDevices) return nullptr;
+    void* p = g_noalloc_addr[dev].load(std::memory_order_acquire);
+    if (p) return p;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    p = g_noalloc_addr[dev].load(std::memory_order_acquire);
+    if (p) return p;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    g_noalloc_addr[dev].store(p, std::memory_order_release);
+    return p;
+}
+
 template <int D>
 attn_status_t launch_decode_pages(const CUtensorMap& mk, const CUtensorMap& mv, const DecodePagesArgs& a,
                                   int grid, cudaStream_t st, __nv_bfloat16* o, float* lse) {
@@ -349,6 +376,7 @@ const char* attn_status_string(attn_status_t s) {
     case ATTN_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
     case ATTN_ERR_CUDA: return "CUDA runtime error";
     case ATTN_ERR_DEVICE_TIMEOUT: return "a kernel gave up on a bounded wait";
+    case ATTN_ERR_SCRATCH_LIMIT: return "request needs more than the library's fixed scratch (8 MiB)";
     default: return "unknown status";
     }
 }
@@ -714,6 +742,31 @@ attn_status_t attn_decode_paged(const void* q, const void* k_cache, const void* 
                               max_blocks_per_seq * block_size);
     if (s != ATTN_OK) return s;
     return launch_status();
+}
+
+attn_status_t attn_decode_paged_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                                        const int32_t* block_table, int max_blocks_per_seq,
+                                        int num_blocks, int block_size, const int32_t* seqused_k,
+                                        int B, int Hq, int Hkv, int D, float softmax_scale, int dtype,
+                                        void* o, float* lse, attn_stream_t stream) {
+    // Arguments that the shared path would reject are reported by it; here only
+    // what decides whether the fixed scratch can serve the request.
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || Hq % Hkv != 0 || max_blocks_per_seq <= 0 ||
+        block_size <= 0)
+        return ATTN_ERR_INVALID_ARG;
+    if (B == 0) return ATTN_OK;
+    if (!use_page_stream(B, Hq, Hkv, D, 0)) return ATTN_ERR_UNSUPPORTED;
+    int dev = 0;
+    const attn_status_t dvs = current_device_ok(&dev);
+    if (dvs != ATTN_OK) return dvs;
+    const size_t need = (size_t)((size_t)sm_count(dev) + B) * Hq * (D + 1) * sizeof(float) +
+                        (size_t)(B + 2) * sizeof(int);
+    if (need > kNoAllocScratchBytes) return ATTN_ERR_SCRATCH_LIMIT;
+    void* scratch = noalloc_scratch_address(dev);
+    if (!scratch) return ATTN_ERR_CUDA;
+    return attn_decode_paged(q, k_cache, v_cache, block_table, max_blocks_per_seq, num_blocks,
+                             block_size, seqused_k, B, Hq, Hkv, D, softmax_scale, 0, dtype, nullptr,
+                             nullptr, nullptr, o, lse, scratch, kNoAllocScratchBytes, stream);
 }
 
 }  // extern "C"

@@ -66,7 +66,8 @@ typedef enum {
     ATTN_ERR_TMA_ENCODE = 4,         /* cuTensorMapEncodeTiled rejected a descriptor */
     ATTN_ERR_WORKSPACE_TOO_SMALL = 5,
     ATTN_ERR_CUDA = 6,               /* a CUDA runtime call or a launch failed */
-    ATTN_ERR_DEVICE_TIMEOUT = 7      /* a kernel gave up on a bounded wait (see attn_device_error) */
+    ATTN_ERR_DEVICE_TIMEOUT = 7,     /* a kernel gave up on a bounded wait (see attn_device_error) */
+    ATTN_ERR_SCRATCH_LIMIT = 8       /* attn_decode_paged_noalloc: needs more than its fixed scratch */
 } attn_status_t;
 
 typedef enum { ATTN_MASK_NONE = 0, ATTN_MASK_CAUSAL = 1, ATTN_MASK_PATCH = 2 } attn_mask_t;
@@ -176,6 +177,35 @@ attn_status_t attn_decode_paged(
     int num_splits, int dtype,
     const float *descale_q, const float *descale_k, const float *descale_v,
     void *o, float *lse, void *workspace, size_t workspace_bytes, attn_stream_t stream);
+
+/*
+ * attn_decode_paged without any device allocation by the caller: the same
+ * paged decode (automatic split choice), with its scratch taken from a fixed
+ * 8 MiB array that this library keeps in device memory.  No counterpart on
+ * the pages; it exists for callers that cannot allocate device memory at
+ * call time -- e.g. a plug-in loaded into a host program that owns every
+ * allocation and exposes no allocator, or a latency-critical serving loop
+ * whose memory is sized once at start-up and which must not reach
+ * cudaMalloc (an implicit synchronisation) while it runs.
+ *   Arguments: as attn_decode_paged, without num_splits and workspace.
+ *   Limits: requests whose split-KV partials need more than 8 MiB (about
+ *   (SMs + B) * Hq * (head_dim + 1) * 4 bytes) return ATTN_ERR_SCRATCH_LIMIT;
+ *   shapes outside the page-stream decode (more than 8 KV heads, more than 16
+ *   query heads per KV head) return ATTN_ERR_UNSUPPORTED.
+ *   Set-up: the first call on each device looks up the scratch's device
+ *   address (cudaGetSymbolAddress) with that device current; make that first
+ *   call before any stream capture.
+ *   Sharing: every call on a device uses the same scratch and leaves its
+ *   contents behind (nothing in it needs to start zeroed).  Calls whose
+ *   kernels could overlap on the GPU (different streams without ordering)
+ *   race on it; order them on one stream or with events.
+ *   Allocation: none -- no cudaMalloc, cudaFree or allocating library call.
+ */
+attn_status_t attn_decode_paged_noalloc(
+    const void *q, const void *k_cache, const void *v_cache, const int32_t *block_table,
+    int max_blocks_per_seq, int num_blocks, int block_size, const int32_t *seqused_k,
+    int B, int num_heads_q, int num_heads_kv, int head_dim, float softmax_scale, int dtype,
+    void *o, float *lse, attn_stream_t stream);
 
 #ifdef __cplusplus
 }
