@@ -38,6 +38,34 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "attn fwd TFLOP/s (prefill) & paged-decode KV GB/s on 1 B200, % of roofline"
+
+# DRAM bytes read + written per launch of each timed kernel, from one ncu
+# capture on its bench workload (full-size launch).  They hold only for the
+# kernel sources they were taken on: when the sha256 prefix of those sources
+# differs, the roofline reports traffic null.
+KERNEL_SOURCES = ["attention_paged_kv_gqa_b200/csrc/decode.cuh",
+                  "attention_paged_kv_gqa_b200/csrc/ptx.cuh",
+                  "attention_paged_kv_gqa_b200/csrc/prefill.cuh"]
+MEASURED_TRAFFIC = {
+    "decode": {"bytes": 579_228_160, "sources": "97cd16d5854f17c1"},
+    "prefill": {"bytes": 2_085_679_264, "sources": "97cd16d5854f17c1"},
+}
+
+
+def kernel_sources_sha() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(kind):
+    rec = MEASURED_TRAFFIC.get(kind)
+    if rec is None or rec["sources"] != kernel_sources_sha():
+        return None
+    return rec["bytes"]
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -164,7 +192,7 @@ def flush_l2(flush):
     step starts cold without inheriting write-backs (a write sweep would leave
     ~126 MB of dirty lines for the next step's DRAM traffic to absorb).
     """
-    flush.sum(dtype=torch.int32)
+    flush.view(torch.int64).sum()
 
 
 def time_steps(step_fn, steps, warmup, world, flush):
@@ -370,8 +398,9 @@ def run_decode(args, A, W, dev, world, flush, peaks, peak_kind, line):
                    "bytes_per_step": nbytes},
         "roofline": {"bound": "hbm", "achieved": round(kernel_gbs, 1),
                      "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": round(kernel_gbs / peaks["hbm_gbs"], 4), "traffic": None,
-                     "kernel": "decode_split_kernel<128> + decode_combine_kernel<128> (one call)",
+                     "frac": round(kernel_gbs / peaks["hbm_gbs"], 4),
+                     "traffic": measured_traffic("decode"),
+                     "kernel": "decode_pages_kernel<128> + decode_pages_combine_kernel<128> (one call)",
                      "peak_kind": peak_kind},
         "e2e": {"value": round(nbytes * world / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
@@ -410,7 +439,7 @@ def run_prefill(args, A, W, dev, world, flush, peaks, peak_kind, line):
         "flops_per_step": flops,
         "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": peaks["bf16_tflops"],
                      "unit": "TFLOP/s", "frac": round(tf / peaks["bf16_tflops"], 4),
-                     "traffic": None, "kernel": "prefill_kernel<128,bf16>",
+                     "traffic": measured_traffic("prefill"), "kernel": "prefill_kernel<128,bf16>",
                      "peak_kind": peak_kind},
     }
     del dp
