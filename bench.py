@@ -85,17 +85,23 @@ def parse_args():
 
 
 # --------------------------------------------------------------------------- plumbing
-def dist_setup(n_gpus):
+def dist_setup(impl="ours"):
+    """Process group for N > 1 (one process per GPU).  NCCL for the CUDA arm;
+    gloo for the reference arm (CPU oracle) or when no GPU is present."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    use_cuda = torch.cuda.is_available() and impl == "ours"
     if world > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    elif torch.cuda.is_available():
+        if use_cuda:
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=120))
+    elif use_cuda:
         torch.cuda.set_device(0)
     return rank, world, local
 
@@ -104,14 +110,17 @@ def barrier(world):
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
-    torch.cuda.synchronize()
+    if torch.cuda.is_available():
+        torch.cuda.synchronize()
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """Largest value over all ranks (the slowest rank's time)."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
@@ -502,7 +511,7 @@ def cpu_baseline(w):
 
 def main():
     args = parse_args()
-    rank, world, local = dist_setup(args.gpus)
+    rank, world, local = dist_setup(args.impl)
     try:
         if args.impl == "reference":
             run_reference(args, rank, world)
