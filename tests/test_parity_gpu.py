@@ -354,6 +354,28 @@ def test_config_fp8_dense_causal_full():
                     assert np.max(np.abs(ll[b, :, i] - ref_l[:, 0])) <= tol_l, (name, b, i)
 
 
+@pytest.mark.parametrize("L", [1, 100, 129, 300, 777])
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("Hq,Hkv", [(2, 2), (4, 2), (3, 1)])
+def test_dense_fp8_small(L, causal, Hq, Hkv):
+    """fp8 e4m3 dense attention over several 128-key tiles with a ragged tail, every
+    output element against the oracle fed the dequantised values."""
+    w = W.dense(B=2, L=L, Hq=Hq, Hkv=Hkv, D=128, causal=causal, seed=11 * L + Hq)
+    t = w.tensors
+    qf, dq = W.quantize_e4m3(t["q"])
+    kf, dk = W.quantize_e4m3(t["k"])
+    vf, dv = W.quantize_e4m3(t["v"])
+    o, lse = A.attn_fwd_dense(qf.to(DEV), kf.to(DEV), vf.to(DEV), causal=causal,
+                              scale=w.params["scale"], descale_q=dq.to(DEV), descale_k=dk.to(DEV),
+                              descale_v=dv.to(DEV))
+    torch.cuda.synchronize()
+    _no_device_error()
+    o_ref, lse_ref = oracle.attn_dense(oracle.dequant_e4m3(qf, dq), oracle.dequant_e4m3(kf, dk),
+                                       oracle.dequant_e4m3(vf, dv), scale=w.params["scale"],
+                                       causal=causal)
+    _cmp(o, lse, o_ref, lse_ref, TOL_O_FP8, None, "fp8 dense L%d" % L)
+
+
 # ---------------------------------------------------------------------------- building blocks
 @pytest.mark.parametrize("degree,bound", [(3, 1.0e-4), (2, 2.0e-3)])
 def test_fma_pipe_exp2_error_bound(degree, bound):
