@@ -49,18 +49,23 @@ def build(force: bool = False) -> Path:
     return _LIB_PATH
 
 
+def bind(lib):
+    """Declares the C oracle's signatures on a loaded library handle."""
+    P = ctypes.c_void_p
+    I = ctypes.c_int
+    D = ctypes.c_double
+    lib.attn_oracle_fwd.restype = I
+    lib.attn_oracle_fwd.argtypes = [P, P, P, P, I, I, P, P, P, I, I, I, I,
+                                    D, I, P, I, D, P, P, I, I]
+    lib.attn_oracle_combine.restype = None
+    lib.attn_oracle_combine.argtypes = [P, P, I, I, I, P, P]
+    return lib
+
+
 def _load():
     global _lib
     if _lib is None:
-        lib = ctypes.CDLL(str(build()))
-        P = ctypes.c_void_p
-        I = ctypes.c_int
-        lib.attn_oracle_fwd.restype = I
-        lib.attn_oracle_fwd.argtypes = [P, P, P, P, I, I, P, P, P, I, I, I, I,
-                                        ctypes.c_double, I, P, P, P, I, I]
-        lib.attn_oracle_combine.restype = None
-        lib.attn_oracle_combine.argtypes = [P, P, I, I, I, P, P]
-        _lib = lib
+        _lib = bind(ctypes.CDLL(str(build())))
     return _lib
 
 
@@ -94,12 +99,14 @@ def default_scale(head_dim: int) -> float:
 
 def attn_varlen(q, k, v, *, cu_seqlens_q, num_heads_kv, scale, mask=MASK_NONE,
                 cu_seqlens_k=None, seqused_k=None, block_table=None, block_size=16,
-                patch_kv_range=None, nthreads=None):
+                patch_kv_range=None, window_left=-1, softcap=0.0, nthreads=None):
     """Varlen / paged attention forward in fp64.
 
     q [total_q, Hq, D]; k, v either [total_k, Hkv, D] (block_table None) or
     paged [num_blocks, block_size, Hkv, D].  Returns (O [total_q, Hq, D],
-    LSE [Hq, total_q]) as fp64 numpy arrays.
+    LSE [Hq, total_q]) as fp64 numpy arrays.  window_left >= 0 (causal mask
+    only) keeps the keys i' - window_left <= j <= i' of row i (i' = i + Lk -
+    Lq); softcap > 0 maps each scaled score s to softcap * tanh(s / softcap).
     """
     lib = _load()
     qa, ka, va = _f64(q), _f64(k), _f64(v)
@@ -117,14 +124,15 @@ def attn_varlen(q, k, v, *, cu_seqlens_q, num_heads_kv, scale, mask=MASK_NONE,
         scale = default_scale(D)
     rc = lib.attn_oracle_fwd(_ptr(qa), _ptr(ka), _ptr(va), _ptr(bt), mbps, int(block_size),
                              _ptr(cq), _ptr(ck), _ptr(su), B, Hq, int(num_heads_kv), D,
-                             float(scale), int(mask), _ptr(pr), _ptr(o), _ptr(lse),
+                             float(scale), int(mask), _ptr(pr), int(window_left),
+                             float(softcap), _ptr(o), _ptr(lse),
                              total_q, int(nthreads or os.cpu_count() or 1))
     if rc != 0:
         raise ValueError("oracle rejected its arguments (rc=%d)" % rc)
     return o, lse
 
 
-def attn_dense(q, k, v, *, scale, causal, nthreads=None):
+def attn_dense(q, k, v, *, scale, causal, window_left=-1, softcap=0.0, nthreads=None):
     """Dense [B, L, H, D] attention in fp64: returns O [B, Lq, Hq, D], LSE [B, Hq, Lq]."""
     qa, ka, va = _f64(q), _f64(k), _f64(v)
     B, Lq, Hq, D = qa.shape
@@ -134,20 +142,27 @@ def attn_dense(q, k, v, *, scale, causal, nthreads=None):
     o, lse = attn_varlen(qa.reshape(B * Lq, Hq, D), ka.reshape(B * Lk, Hkv, D),
                          va.reshape(B * Lk, Hkv, D), cu_seqlens_q=cq, cu_seqlens_k=ck,
                          num_heads_kv=Hkv, scale=scale,
-                         mask=MASK_CAUSAL if causal else MASK_NONE, nthreads=nthreads)
+                         mask=MASK_CAUSAL if causal else MASK_NONE, window_left=window_left,
+                         softcap=softcap, nthreads=nthreads)
     return o.reshape(B, Lq, Hq, D), lse.reshape(Hq, B, Lq).transpose(1, 0, 2).copy()
 
 
 def attn_decode(q, k_cache, v_cache, block_table, seqused_k, *, scale, block_size=16,
-                nthreads=None):
-    """One query token per sequence against a paged cache: O [B, Hq, D], LSE [B, Hq]."""
+                window_left=-1, softcap=0.0, nthreads=None):
+    """One query token per sequence against a paged cache: O [B, Hq, D], LSE [B, Hq].
+
+    The query is the newest cached token, so with a sliding window it sees the
+    keys Lk - 1 - window_left .. Lk - 1 (causal with Lq = 1 and the window).
+    """
     qa = _f64(q)
     B, Hq, D = qa.shape
     Hkv = k_cache.shape[2]
     cq = np.arange(B + 1, dtype=np.int32)
     o, lse = attn_varlen(qa, k_cache, v_cache, cu_seqlens_q=cq, seqused_k=seqused_k,
                          block_table=block_table, block_size=block_size,
-                         num_heads_kv=Hkv, scale=scale, mask=MASK_NONE, nthreads=nthreads)
+                         num_heads_kv=Hkv, scale=scale,
+                         mask=MASK_CAUSAL if window_left >= 0 else MASK_NONE,
+                         window_left=window_left, softcap=softcap, nthreads=nthreads)
     return o, lse.T.copy()
 
 

@@ -12,7 +12,9 @@
  *   For sequence b, query head h, query i:
  *     g      = h / (Hq / Hkv)                       grouped-query head sharing
  *     s_ij   = scale * sum_d q[i,h,d] * k[j,g,d]    explicit score row, all j < Lk_b
- *     allowed(i,j) by index (none / causal / patch)
+ *     s_ij   = c * tanh(s_ij / c)                   only with a softcap c > 0
+ *     allowed(i,j) by index (none / causal / patch; causal optionally with a
+ *                  sliding window of W keys before the diagonal)
  *     M      = max_{allowed j} s_ij
  *     p_ij   = exp(s_ij - M) for allowed j, else 0
  *     O[i,h] = sum_j p_ij v[j,g] / sum_j p_ij
@@ -38,7 +40,13 @@
  *   - causal alignment for Lq != Lk is bottom-right: j <= i + (Lk - Lq); it is
  *     the page's q_idx >= kv_idx when Lq == Lk;
  *   - the patch predicate is start_i <= j < end_i, sequence-local;
- *   - paged layout [num_blocks][block_size][Hkv][D], block_table[b][j / bs].
+ *   - paged layout [num_blocks][block_size][Hkv][D], block_table[b][j / bs];
+ *   - "local window on/off" and "softcap 0/50" (the parity matrix of "[CUDA]
+ *     PagedAttention: add SM<80 fp16 fallback via memory-efficient
+ *     attention", Testing) are read as: a causal row keeps only the keys
+ *     i' - W <= j <= i' (i' = i + Lk - Lq, W >= 0; W < 0 means no window),
+ *     and a softcap c > 0 maps each scaled score s to c * tanh(s / c)
+ *     (c = 0 means none).
  */
 #include <math.h>
 #include <stdint.h>
@@ -64,10 +72,13 @@ static const double *kv_row(const double *base, int b, int j, int g, int Hkv, in
     return base + (row * Hkv + g) * (long long)D;
 }
 
-static int allowed(int mask, int i, int j, int Lq, int Lk, const int32_t *range_i) {
+static int allowed(int mask, int i, int j, int Lq, int Lk, const int32_t *range_i,
+                   int window_left) {
     switch (mask) {
     case ORACLE_MASK_NONE: return 1;
-    case ORACLE_MASK_CAUSAL: return j <= i + (Lk - Lq);
+    case ORACLE_MASK_CAUSAL:
+        if (window_left >= 0 && j < i + (Lk - Lq) - window_left) return 0;
+        return j <= i + (Lk - Lq);
     case ORACLE_MASK_PATCH: return range_i[0] <= j && j < range_i[1];
     default: return 0;
     }
@@ -78,6 +89,7 @@ static int allowed(int mask, int i, int j, int Lq, int Lk, const int32_t *range_
  * k, v paged: [num_blocks][block_size][Hkv][D] (block_table != NULL)
  *      else : [total_k][Hkv][D] addressed by cu_seqlens_k
  * Lk_b = seqused_k[b] if seqused_k, else cu_seqlens_k[b+1] - cu_seqlens_k[b]
+ * window_left >= 0 only with the causal mask; softcap >= 0 (0: none)
  * o    [total_q][Hq][D];  lse [Hq][total_q]
  * Returns 0, or -1 for arguments it cannot interpret.
  */
@@ -86,8 +98,11 @@ int attn_oracle_fwd(const double *q, const double *k, const double *v,
                     const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
                     const int32_t *seqused_k, int B, int Hq, int Hkv, int D,
                     double scale, int mask, const int32_t *patch_kv_range,
+                    int window_left, double softcap,
                     double *o, double *lse, int total_q, int nthreads) {
     if (B < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || Hq % Hkv != 0) return -1;
+    if (window_left >= 0 && mask != ORACLE_MASK_CAUSAL) return -1;
+    if (!(softcap >= 0.0)) return -1;
     if (!seqused_k && !cu_seqlens_k) return -1;
     if (!block_table && !cu_seqlens_k) return -1;
     if (mask == ORACLE_MASK_PATCH && !patch_kv_range) return -1;
@@ -119,12 +134,13 @@ int attn_oracle_fwd(const double *q, const double *k, const double *v,
                 double acc = 0.0;
                 for (int d = 0; d < D; ++d) acc += qi[d] * kj[d];
                 s[j] = scale * acc;
+                if (softcap > 0.0) s[j] = softcap * tanh(s[j] / softcap);
             }
             /* max over the allowed keys */
             double M = -INFINITY;
             int any = 0;
             for (int j = 0; j < Lk; ++j) {
-                if (!allowed(mask, i, j, Lq, Lk, range_i)) continue;
+                if (!allowed(mask, i, j, Lq, Lk, range_i, window_left)) continue;
                 if (!any || s[j] > M) M = s[j];
                 any = 1;
             }
@@ -133,7 +149,7 @@ int attn_oracle_fwd(const double *q, const double *k, const double *v,
             /* max-subtracted softmax and the weighted sum of V rows */
             double Z = 0.0;
             for (int j = 0; j < Lk; ++j) {
-                if (!allowed(mask, i, j, Lq, Lk, range_i)) continue;
+                if (!allowed(mask, i, j, Lq, Lk, range_i, window_left)) continue;
                 const double p = exp(s[j] - M);
                 const double *vj = kv_row(v, b, j, g, Hkv, D, block_table,
                                           max_blocks_per_seq, block_size, cu_seqlens_k);

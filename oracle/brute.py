@@ -18,18 +18,23 @@ from __future__ import annotations
 import math
 
 
-def _allowed(mask: str, i: int, j: int, Lq: int, Lk: int, rng) -> bool:
+def _allowed(mask: str, i: int, j: int, Lq: int, Lk: int, rng, window) -> bool:
     if mask == "none":
         return True
     if mask == "causal":
-        return j <= i + (Lk - Lq)
+        diag = i + (Lk - Lq)
+        return j <= diag and (window < 0 or diag - j <= window)
     if mask == "patch":
         return rng[0] <= j < rng[1]
     raise ValueError(mask)
 
 
-def attention(q, k, v, scale, mask="none", patch=None):
+def attention(q, k, v, scale, mask="none", patch=None, window=-1, softcap=0.0):
     """One sequence.  q[i][h][d], k[j][g][d], v[j][g][d] as nested lists.
+
+    window >= 0 (causal only) keeps the keys at most `window` positions
+    before the row's diagonal; softcap > 0 replaces each scaled score s by
+    softcap * tanh(s / softcap).
 
     Returns (o[i][h][d], lse[h][i]) as nested lists of Python floats.
     """
@@ -43,13 +48,15 @@ def attention(q, k, v, scale, mask="none", patch=None):
         g = h // group
         for i in range(Lq):
             keys = [j for j in range(Lk)
-                    if _allowed(mask, i, j, Lq, Lk, patch[i] if patch else None)]
+                    if _allowed(mask, i, j, Lq, Lk, patch[i] if patch else None, window)]
             if not keys:
                 lse[h][i] = -math.inf
                 continue
             e = {}
             for j in keys:
                 s = scale * math.fsum(q[i][h][d] * k[j][g][d] for d in range(D))
+                if softcap > 0:
+                    s = softcap * math.tanh(s / softcap)
                 e[j] = math.exp(s)
             z = math.fsum(e.values())
             for d in range(D):

@@ -258,8 +258,123 @@ def test_split_kv_combine_reproduces_unsplit():
 
 
 # ----------------------------------------------------------------------------
+# sliding window and softcap (the "local window on/off, softcap 0/50" options)
+# ----------------------------------------------------------------------------
+
+def test_window_zero_keeps_only_the_diagonal_key():
+    """W = 0: row i sees only key i' = i + Lk - Lq, so O = v_i' exactly and LSE = s_ii'."""
+    Lq, Lk, D = 5, 9, 4
+    q, k, v = rnd((Lq, 2, D), 41), rnd((Lk, 1, D), 42), rnd((Lk, 1, D), 43)
+    o, lse = oracle.attn_varlen(q, k, v, cu_seqlens_q=cu([Lq]), cu_seqlens_k=cu([Lk]),
+                                num_heads_kv=1, scale=0.4, mask=1, window_left=0)
+    for i in range(Lq):
+        d = i + Lk - Lq
+        for h in range(2):
+            np.testing.assert_array_equal(o[i, h], v[d, 0])
+            assert lse[h, i] == pytest.approx(0.4 * float(np.dot(q[i, h], k[d, 0])), abs=1e-14)
+
+
+@pytest.mark.parametrize("W", [1, 3, 6])
+def test_window_equals_unmasked_attention_over_the_sliced_keys(W):
+    """Row i with window W == unmasked attention of query i over keys max(0, i'-W) .. i'."""
+    Lq, Lk, D = 6, 10, 5
+    q, k, v = rnd((Lq, 1, D), 44), rnd((Lk, 1, D), 45), rnd((Lk, 1, D), 46)
+    o, lse = oracle.attn_varlen(q, k, v, cu_seqlens_q=cu([Lq]), cu_seqlens_k=cu([Lk]),
+                                num_heads_kv=1, scale=0.5, mask=1, window_left=W)
+    for i in range(Lq):
+        d = i + Lk - Lq
+        a = max(0, d - W)
+        oi, li = oracle.attn_varlen(q[i:i + 1], k[a:d + 1], v[a:d + 1], cu_seqlens_q=cu([1]),
+                                    cu_seqlens_k=cu([d + 1 - a]), num_heads_kv=1, scale=0.5,
+                                    mask=0)
+        np.testing.assert_allclose(o[i], oi[0], atol=1e-14, rtol=0)
+        assert lse[0, i] == pytest.approx(li[0, 0], abs=1e-14)
+
+
+def test_window_at_least_the_length_is_plain_causal():
+    L, D = 7, 3
+    q, k, v = rnd((L, 2, D), 47), rnd((L, 1, D), 48), rnd((L, 1, D), 49)
+    kw = dict(cu_seqlens_q=cu([L]), cu_seqlens_k=cu([L]), num_heads_kv=1, scale=0.7, mask=1)
+    o0, l0 = oracle.attn_varlen(q, k, v, **kw)
+    o1, l1 = oracle.attn_varlen(q, k, v, window_left=L, **kw)
+    np.testing.assert_array_equal(o0, o1)
+    np.testing.assert_array_equal(l0, l1)
+
+
+def test_softcap_closed_form_two_keys():
+    """Scaled scores c*atanh(1/2) and 0 become c/2 and 0 (tanh(ln(3)/2) = 1/2), so
+    O = (e^(c/2) v1 + v2) / (e^(c/2) + 1) and LSE = ln(e^(c/2) + 1)."""
+    c, scale = 3.0, 0.25
+    q = np.ones((1, 1, 1))
+    k = np.array([[[c * math.log(3.0) / 2 / scale]], [[0.0]]])
+    v = np.array([[[2.0]], [[-5.0]]])
+    o, lse = oracle.attn_varlen(q, k, v, cu_seqlens_q=cu([1]), cu_seqlens_k=cu([2]),
+                                num_heads_kv=1, scale=scale, softcap=c)
+    e = math.exp(c / 2)
+    assert o[0, 0, 0] == pytest.approx((e * 2.0 - 5.0) / (e + 1), abs=1e-13)
+    assert lse[0, 0] == pytest.approx(math.log(e + 1), abs=1e-13)
+
+
+def test_softcap_limits():
+    """A cap far below every score flattens the weights (O = mean of the allowed V,
+    LSE = ln n); a cap far above them leaves the plain result."""
+    L, D = 6, 4
+    q, k, v = rnd((L, 1, D), 50) * 3, rnd((L, 1, D), 51) * 3, rnd((L, 1, D), 52)
+    kw = dict(cu_seqlens_q=cu([L]), cu_seqlens_k=cu([L]), num_heads_kv=1, scale=0.9, mask=1)
+    o, lse = oracle.attn_varlen(q, k, v, softcap=1e-9, **kw)
+    for i in range(L):
+        np.testing.assert_allclose(o[i, 0], v[:i + 1, 0].mean(axis=0), atol=1e-8, rtol=0)
+        assert lse[0, i] == pytest.approx(math.log(i + 1), abs=1e-8)
+    o0, l0 = oracle.attn_varlen(q, k, v, **kw)
+    o1, l1 = oracle.attn_varlen(q, k, v, softcap=1e9, **kw)   # |s - c tanh(s/c)| <= |s|^3/(3c^2)
+    np.testing.assert_allclose(o1, o0, atol=1e-12, rtol=0)
+    np.testing.assert_allclose(l1, l0, atol=1e-12, rtol=0)
+
+
+def test_softcap_bounds_the_lse():
+    """Capped logits lie in (-c, c), so ln n - c < LSE < ln n + c even for huge scores."""
+    L, D, c = 9, 4, 2.0
+    q, k, v = rnd((L, 1, D), 53), rnd((L, 1, D), 54), rnd((L, 1, D), 55)
+    o, lse = oracle.attn_varlen(q, k, v, cu_seqlens_q=cu([L]), cu_seqlens_k=cu([L]),
+                                num_heads_kv=1, scale=1e3, mask=0, softcap=c)
+    assert np.all(lse > math.log(L) - c) and np.all(lse < math.log(L) + c)
+    assert np.all(np.isfinite(o))
+
+
+def test_window_and_softcap_rejected_where_undefined():
+    q = rnd((2, 1, 2), 56)
+    with pytest.raises(ValueError):
+        oracle.attn_varlen(q, q, q, cu_seqlens_q=cu([2]), cu_seqlens_k=cu([2]), num_heads_kv=1,
+                           scale=1.0, mask=0, window_left=1)
+    with pytest.raises(ValueError):
+        oracle.attn_varlen(q, q, q, cu_seqlens_q=cu([2]), cu_seqlens_k=cu([2]), num_heads_kv=1,
+                           scale=1.0, mask=1, softcap=-1.0)
+
+
+# ----------------------------------------------------------------------------
 # an independent implementation on tiny inputs
 # ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+@pytest.mark.parametrize("window,softcap", [(0, 0.0), (2, 0.0), (-1, 1.5), (3, 0.8)])
+def test_brute_force_agrees_with_window_and_softcap(window, softcap, seed):
+    rng = np.random.default_rng(200 + seed)
+    Hq, Hkv, D = 2, 1, 3
+    lens_q = [int(x) for x in rng.integers(1, 9, size=2)]
+    lens_k = [max(lq, int(x)) for lq, x in zip(lens_q, rng.integers(1, 9, size=2))]
+    cq, ck = cu(lens_q), cu(lens_k)
+    q = rng.standard_normal((cq[-1], Hq, D)) * 2
+    k = rng.standard_normal((ck[-1], Hkv, D)) * 2
+    v = rng.standard_normal((ck[-1], Hkv, D))
+    o, lse = oracle.attn_varlen(q, k, v, cu_seqlens_q=cq, cu_seqlens_k=ck, num_heads_kv=Hkv,
+                                scale=0.6, mask=1, window_left=window, softcap=softcap)
+    for b in range(2):
+        ob, lb = brute.attention(q[cq[b]:cq[b + 1]].tolist(), k[ck[b]:ck[b + 1]].tolist(),
+                                 v[ck[b]:ck[b + 1]].tolist(), 0.6, "causal", None, window,
+                                 softcap)
+        np.testing.assert_allclose(o[cq[b]:cq[b + 1]], np.array(ob), atol=1e-12, rtol=0)
+        np.testing.assert_allclose(lse[:, cq[b]:cq[b + 1]], np.array(lb), atol=1e-12, rtol=0)
+
 
 @pytest.mark.parametrize("mask", ["none", "causal", "patch"])
 @pytest.mark.parametrize("seed", [0, 1, 2])
@@ -372,6 +487,18 @@ MUTATIONS = {
                             "return range_i[0] <= j && j <= range_i[1];"),
     "combine_weight": ("const double w = exp(lse_parts[(long long)s * N + n] - lse[n]);",
                        "const double w = exp(lse_parts[(long long)s * N + n] - M);"),
+    "window_off_by_one": ("if (window_left >= 0 && j < i + (Lk - Lq) - window_left) return 0;",
+                          "if (window_left >= 0 && j <= i + (Lk - Lq) - window_left) return 0;"),
+    "window_ignored": ("if (window_left >= 0 && j < i + (Lk - Lq) - window_left) return 0;", ""),
+    "window_top_left": ("if (window_left >= 0 && j < i + (Lk - Lq) - window_left) return 0;",
+                        "if (window_left >= 0 && j < i - window_left) return 0;"),
+    "softcap_ignored": ("if (softcap > 0.0) s[j] = softcap * tanh(s[j] / softcap);", ""),
+    "softcap_no_outer_factor": ("if (softcap > 0.0) s[j] = softcap * tanh(s[j] / softcap);",
+                                "if (softcap > 0.0) s[j] = tanh(s[j] / softcap);"),
+    "softcap_no_inner_division": ("if (softcap > 0.0) s[j] = softcap * tanh(s[j] / softcap);",
+                                  "if (softcap > 0.0) s[j] = softcap * tanh(s[j]);"),
+    "softcap_before_scale": ("if (softcap > 0.0) s[j] = softcap * tanh(s[j] / softcap);",
+                             "if (softcap > 0.0) s[j] = scale * softcap * tanh(acc / softcap);"),
 }
 
 PINS = [
@@ -388,6 +515,14 @@ PINS = [
     lambda: [test_brute_force_enumeration_agrees(m, s) for m in ("none", "causal", "patch")
              for s in (0, 1, 2)],
     test_golden_causal_predicate_4x4,
+    test_window_zero_keeps_only_the_diagonal_key,
+    lambda: [test_window_equals_unmasked_attention_over_the_sliced_keys(w) for w in (1, 3, 6)],
+    test_window_at_least_the_length_is_plain_causal,
+    test_softcap_closed_form_two_keys,
+    test_softcap_limits,
+    test_softcap_bounds_the_lse,
+    lambda: [test_brute_force_agrees_with_window_and_softcap(w, c, s)
+             for w, c in ((0, 0.0), (2, 0.0), (-1, 1.5), (3, 0.8)) for s in (0, 1, 2)],
 ]
 
 
@@ -400,14 +535,8 @@ def _mutated_oracle(src_text):
         subprocess.run(["gcc", "-O1", "-fopenmp", "-fPIC", "-shared", "-std=c11", str(c),
                         "-o", str(so), "-lm"], check=True)
         saved = oracle._lib
-        lib = ctypes.CDLL(str(so))
+        lib = oracle.bind(ctypes.CDLL(str(so)))
         try:
-            P, I = ctypes.c_void_p, ctypes.c_int
-            lib.attn_oracle_fwd.restype = I
-            lib.attn_oracle_fwd.argtypes = [P, P, P, P, I, I, P, P, P, I, I, I, I,
-                                            ctypes.c_double, I, P, P, P, I, I]
-            lib.attn_oracle_combine.restype = None
-            lib.attn_oracle_combine.argtypes = [P, P, I, I, I, P, P]
             oracle._lib = lib
             yield
         finally:
