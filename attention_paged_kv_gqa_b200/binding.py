@@ -49,15 +49,16 @@ def lib():
         L.attn_device_error.restype = I
         L.attn_selftest_exp2.argtypes = [P, P, I, I, P]
         L.attn_selftest_exp2.restype = I
-        L.attn_fwd_dense.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P, P, P, F, I, I, P, P, P, P]
+        L.attn_fwd_dense.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P, P, P, F, I, I, F, I,
+                                     P, P, P, P]
         L.attn_fwd_dense.restype = I
         L.attn_fwd_varlen_paged.argtypes = [P, P, P, P, I, I, I, P, P, P, I, I, I, I, I, I, I,
-                                            F, I, P, I, P, P, P, P, P, P, Z, P]
+                                            F, I, P, I, F, I, P, P, P, P, P, P, Z, P]
         L.attn_fwd_varlen_paged.restype = I
         L.attn_decode_workspace_size.argtypes = [I, I, I, I, I, I, I]
         L.attn_decode_workspace_size.restype = Z
-        L.attn_decode_paged.argtypes = [P, P, P, P, I, I, I, P, I, I, I, I, F, I, I, P, P, P,
-                                        P, P, P, Z, P]
+        L.attn_decode_paged.argtypes = [P, P, P, P, I, I, I, P, I, I, I, I, F, I, F, I, I, P, P,
+                                        P, P, P, P, Z, P]
         L.attn_decode_paged.restype = I
         L.attn_decode_paged_noalloc.argtypes = [P, P, P, P, I, I, I, P, I, I, I, I, F, I, P, P, P]
         L.attn_decode_paged_noalloc.restype = I
@@ -124,9 +125,14 @@ def attn_selftest_exp2(x, degree=3, stream=None):
     return y
 
 
-def attn_fwd_dense(q, k, v, *, causal=False, scale=None, descale_q=None, descale_k=None,
-                   descale_v=None, out=None, lse=None, return_lse=True, stream=None):
-    """q [B, Lq, Hq, D], k/v [B, Lk, Hkv, D] -> (o [B, Lq, Hq, D] bf16, lse [B, Hq, Lq] fp32)."""
+def attn_fwd_dense(q, k, v, *, causal=False, scale=None, window_left=-1, softcap=0.0,
+                   descale_q=None, descale_k=None, descale_v=None, out=None, lse=None,
+                   return_lse=True, stream=None):
+    """q [B, Lq, Hq, D], k/v [B, Lk, Hkv, D] -> (o [B, Lq, Hq, D] bf16, lse [B, Hq, Lq] fp32).
+
+    window_left >= 0 (causal only): row i keeps keys i' - window_left .. i';
+    softcap > 0: each logit s becomes softcap * tanh(s / softcap).
+    """
     B, Lq, Hq, D = q.shape
     Lk, Hkv = k.shape[1], k.shape[2]
     if out is None:
@@ -135,7 +141,8 @@ def attn_fwd_dense(q, k, v, *, causal=False, scale=None, descale_q=None, descale
         lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=q.device)
     st = lib().attn_fwd_dense(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Lq, Lk, Hq, Hkv,
                               D, _strides3(q), _strides3(k), _strides3(v), _scale(scale),
-                              MASK_CAUSAL if causal else MASK_NONE, _dtype_code(q),
+                              MASK_CAUSAL if causal else MASK_NONE, int(window_left),
+                              float(softcap), _dtype_code(q),
                               _ptr(descale_q), _ptr(descale_k), _ptr(descale_v), _stream(stream))
     _check(st, "attn_fwd_dense")
     return out, lse
@@ -143,8 +150,9 @@ def attn_fwd_dense(q, k, v, *, causal=False, scale=None, descale_q=None, descale
 
 def attn_fwd_varlen_paged(q, k_cache, v_cache, *, cu_seqlens_q, max_seqlen_q, block_table=None,
                           cu_seqlens_k=None, seqused_k=None, mask=MASK_NONE, scale=None,
-                          patch_kv_range=None, descale_q=None, descale_k=None, descale_v=None,
-                          out=None, lse=None, return_lse=True, stream=None):
+                          patch_kv_range=None, window_left=-1, softcap=0.0, descale_q=None,
+                          descale_k=None, descale_v=None, out=None, lse=None, return_lse=True,
+                          stream=None):
     """q [total_q, Hq, D]; paged k/v [num_blocks, 16, Hkv, D] (or packed [total_k, Hkv, D]).
 
     Returns (o [total_q, Hq, D] bf16, lse [Hq, total_q] fp32).
@@ -165,7 +173,7 @@ def attn_fwd_varlen_paged(q, k_cache, v_cache, *, cu_seqlens_q, max_seqlen_q, bl
         _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), mbps, num_blocks, block_size,
         _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), _ptr(seqused_k), B, total_q, total_k,
         int(max_seqlen_q), Hq, Hkv, D, _scale(scale), int(mask), _ptr(patch_kv_range),
-        _dtype_code(q), _ptr(descale_q), _ptr(descale_k), _ptr(descale_v), _ptr(out), _ptr(lse),
+        int(window_left), float(softcap), _dtype_code(q), _ptr(descale_q), _ptr(descale_k), _ptr(descale_v), _ptr(out), _ptr(lse),
         None, 0, _stream(stream))
     _check(st, "attn_fwd_varlen_paged")
     return out, lse
@@ -178,8 +186,13 @@ def attn_decode_workspace_size(B, num_heads_q, num_heads_kv, head_dim, max_block
 
 
 def attn_decode_paged(q, k_cache, v_cache, block_table, seqused_k, *, scale=None, num_splits=0,
-                      out=None, lse=None, workspace=None, return_lse=True, stream=None):
-    """q [B, Hq, D] against a paged cache -> (o [B, Hq, D] bf16, lse [B, Hq] fp32)."""
+                      window_left=-1, softcap=0.0, out=None, lse=None, workspace=None,
+                      return_lse=True, stream=None):
+    """q [B, Hq, D] against a paged cache -> (o [B, Hq, D] bf16, lse [B, Hq] fp32).
+
+    The query is the newest cached token; window_left >= 0 keeps the keys
+    L-1-window_left .. L-1; softcap > 0 caps the logits as in the prefill calls.
+    """
     B, Hq, D = q.shape
     num_blocks, block_size, Hkv = k_cache.shape[0], k_cache.shape[1], k_cache.shape[2]
     mbps = block_table.shape[1]
@@ -192,7 +205,8 @@ def attn_decode_paged(q, k_cache, v_cache, block_table, seqused_k, *, scale=None
         workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=q.device)
     st = lib().attn_decode_paged(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), mbps,
                                  num_blocks, block_size, _ptr(seqused_k), B, Hq, Hkv, D,
-                                 _scale(scale), int(num_splits), _dtype_code(q), None, None, None,
+                                 _scale(scale), int(window_left), float(softcap), int(num_splits),
+                                 _dtype_code(q), None, None, None,
                                  _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(),
                                  _stream(stream))
     _check(st, "attn_decode_paged")

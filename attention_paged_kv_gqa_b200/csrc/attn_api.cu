@@ -41,7 +41,7 @@ attn_status_t check_device_uncached(int device) {
     cudaGetDevice(&prev);
     if (prev != device) cudaSetDevice(device);
     cudaFuncAttributes fa;
-    const cudaError_t e = cudaFuncGetAttributes(&fa, prefill_kernel<128, false>);
+    const cudaError_t e = cudaFuncGetAttributes(&fa, prefill_kernel<128, false, false>);
     if (prev != device && prev >= 0) cudaSetDevice(prev);
     if (e != cudaSuccess) {
         cudaGetLastError();
@@ -192,7 +192,7 @@ attn_status_t launch_status() {
 }
 
 // ------------------------------------------------------------------ prefill dispatch
-template <int D, bool FP8>
+template <int D, bool FP8, bool CAP>
 attn_status_t launch_prefill_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                                const PrefillArgs& a, long long grid, cudaStream_t stream) {
     using Cfg = PrefillCfg<D, FP8>;
@@ -201,11 +201,11 @@ attn_status_t launch_prefill_t(const CUtensorMap& mq, const CUtensorMap& mk, con
     cudaGetDevice(&dev);
     const uint64_t bit = 1ull << (dev & 63);
     if (!(attr_mask.load() & bit)) {
-        const attn_status_t s = set_smem(prefill_kernel<D, FP8>, Cfg::SMEM_BYTES);
+        const attn_status_t s = set_smem(prefill_kernel<D, FP8, CAP>, Cfg::SMEM_BYTES);
         if (s != ATTN_OK) return s;
         attr_mask.fetch_or(bit);
     }
-    prefill_kernel<D, FP8><<<static_cast<unsigned>(grid), kPrefillThreads, Cfg::SMEM_BYTES, stream>>>(
+    prefill_kernel<D, FP8, CAP><<<static_cast<unsigned>(grid), kPrefillThreads, Cfg::SMEM_BYTES, stream>>>(
         mq, mk, mv, a);
     return launch_status();
 }
@@ -215,9 +215,16 @@ attn_status_t launch_prefill(int D, int dtype, const CUtensorMap& mq, const CUte
                              cudaStream_t stream) {
     if (grid <= 0) return ATTN_OK;
     if (grid >= (1LL << 31)) return ATTN_ERR_UNSUPPORTED;
-    if (dtype == ATTN_BF16 && D == 128) return launch_prefill_t<128, false>(mq, mk, mv, a, grid, stream);
-    if (dtype == ATTN_BF16 && D == 64) return launch_prefill_t<64, false>(mq, mk, mv, a, grid, stream);
-    if (dtype == ATTN_FP8_E4M3 && D == 128) return launch_prefill_t<128, true>(mq, mk, mv, a, grid, stream);
+    const bool cap = a.softcap > 0.0f;
+    if (dtype == ATTN_BF16 && D == 128)
+        return cap ? launch_prefill_t<128, false, true>(mq, mk, mv, a, grid, stream)
+                   : launch_prefill_t<128, false, false>(mq, mk, mv, a, grid, stream);
+    if (dtype == ATTN_BF16 && D == 64)
+        return cap ? launch_prefill_t<64, false, true>(mq, mk, mv, a, grid, stream)
+                   : launch_prefill_t<64, false, false>(mq, mk, mv, a, grid, stream);
+    if (dtype == ATTN_FP8_E4M3 && D == 128)
+        return cap ? launch_prefill_t<128, true, true>(mq, mk, mv, a, grid, stream)
+                   : launch_prefill_t<128, true, false>(mq, mk, mv, a, grid, stream);
     return ATTN_ERR_UNSUPPORTED;
 }
 
@@ -287,7 +294,7 @@ attn_status_t launch_decode(const CUtensorMap& mk, const CUtensorMap& mv, Decode
     cfg.numAttrs = 1;
     if (cudaLaunchKernelEx(&cfg, decode_combine_kernel<D>, (const float*)a.o_part,
                            (const float*)a.lse_part, (const int*)seqused_k, a.B, a.Hq, a.num_splits,
-                           a.tokens_per_split, max_tokens, a.o, a.lse) != cudaSuccess) {
+                           a.tokens_per_split, max_tokens, a.window, a.o, a.lse) != cudaSuccess) {
         cudaGetLastError();
         return ATTN_ERR_CUDA;
     }
@@ -419,16 +426,36 @@ attn_status_t attn_selftest_exp2(const float* x, float* y, int n, int degree, at
     return launch_status();
 }
 
+// Sliding window and softcap: a window is defined for the causal mask only
+// (any negative window_left means none); softcap must be finite and >= 0.
+static attn_status_t check_score_mods(int mask, int window_left, float softcap) {
+    if (!(softcap >= 0.0f) || !std::isfinite(softcap)) return ATTN_ERR_INVALID_ARG;
+    if (window_left >= 0 && mask != ATTN_MASK_CAUSAL) return ATTN_ERR_UNSUPPORTED;
+    return ATTN_OK;
+}
+
+// Keys a decode query can touch: the whole cache span, or its window plus the
+// part of the first page before it.
+static int decode_span(int max_tokens, int window) {
+    if (window < 0) return max_tokens;
+    return (int)std::min<long long>(max_tokens, (long long)window + 1 + kPageRows);
+}
+
 attn_status_t attn_fwd_dense(const void* q, const void* k, const void* v, void* o, float* lse,
                              int B, int Lq, int Lk, int Hq, int Hkv, int D,
                              const int64_t* sq, const int64_t* sk, const int64_t* sv,
-                             float softmax_scale, int mask, int dtype, const float* dq,
-                             const float* dk, const float* dv, attn_stream_t stream) {
+                             float softmax_scale, int mask, int window_left, float softcap,
+                             int dtype, const float* dq, const float* dk, const float* dv,
+                             attn_stream_t stream) {
     if (!q || !k || !v || !o || !sq || !sk || !sv) return ATTN_ERR_INVALID_ARG;
     if (B < 0 || Lq < 0 || Lk < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
     if (!dtype_ok(dtype)) return ATTN_ERR_INVALID_ARG;
     if (mask != ATTN_MASK_NONE && mask != ATTN_MASK_CAUSAL) {
         return mask == ATTN_MASK_PATCH ? ATTN_ERR_UNSUPPORTED : ATTN_ERR_INVALID_ARG;
+    }
+    {
+        const attn_status_t ms = check_score_mods(mask, window_left, softcap);
+        if (ms != ATTN_OK) return ms;
     }
     if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
     if (dtype == ATTN_FP8_E4M3 && (D != 128)) return ATTN_ERR_UNSUPPORTED;
@@ -466,6 +493,8 @@ attn_status_t attn_fwd_dense(const void* q, const void* k, const void* v, void* 
     a.Hkv = Hkv;
     a.group = Hq / Hkv;
     a.mask = mask;
+    a.window = window_left < 0 ? -1 : window_left;
+    a.softcap = softcap;
     a.varlen = 0;
     a.paged = 0;
     a.Lq = Lq;
@@ -490,8 +519,9 @@ attn_status_t attn_fwd_varlen_paged(
     int max_blocks_per_seq, int num_blocks, int block_size, const int32_t* cu_seqlens_q,
     const int32_t* cu_seqlens_k, const int32_t* seqused_k, int B, int total_q, int total_k,
     int max_seqlen_q, int Hq, int Hkv, int D, float softmax_scale, int mask,
-    const int32_t* patch_kv_range, int dtype, const float* dq, const float* dk, const float* dv,
-    void* o, float* lse, void* workspace, size_t workspace_bytes, attn_stream_t stream) {
+    const int32_t* patch_kv_range, int window_left, float softcap, int dtype, const float* dq,
+    const float* dk, const float* dv, void* o, float* lse, void* workspace,
+    size_t workspace_bytes, attn_stream_t stream) {
     (void)workspace;
     (void)workspace_bytes;
     if (!q || !k_cache || !v_cache || !o || !cu_seqlens_q) return ATTN_ERR_INVALID_ARG;
@@ -500,6 +530,10 @@ attn_status_t attn_fwd_varlen_paged(
     if (!dtype_ok(dtype)) return ATTN_ERR_INVALID_ARG;
     if (mask < ATTN_MASK_NONE || mask > ATTN_MASK_PATCH) return ATTN_ERR_INVALID_ARG;
     if (mask == ATTN_MASK_PATCH && !patch_kv_range) return ATTN_ERR_INVALID_ARG;
+    {
+        const attn_status_t ms = check_score_mods(mask, window_left, softcap);
+        if (ms != ATTN_OK) return ms;
+    }
     if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
     if (dtype == ATTN_FP8_E4M3 && D != 128) return ATTN_ERR_UNSUPPORTED;
     if (dtype == ATTN_FP8_E4M3 && (!dq || !dk || !dv)) return ATTN_ERR_INVALID_ARG;
@@ -543,6 +577,8 @@ attn_status_t attn_fwd_varlen_paged(
     a.Hkv = Hkv;
     a.group = Hq / Hkv;
     a.mask = mask;
+    a.window = window_left < 0 ? -1 : window_left;
+    a.softcap = softcap;
     a.varlen = 1;
     a.paged = paged ? 1 : 0;
     a.cu_q = cu_seqlens_q;
@@ -634,14 +670,20 @@ size_t attn_decode_workspace_size(int B, int Hq, int Hkv, int D, int max_blocks_
 attn_status_t attn_decode_paged(const void* q, const void* k_cache, const void* v_cache,
                                 const int32_t* block_table, int max_blocks_per_seq, int num_blocks,
                                 int block_size, const int32_t* seqused_k, int B, int Hq, int Hkv,
-                                int D, float softmax_scale, int num_splits, int dtype,
-                                const float* dq, const float* dk, const float* dv, void* o,
-                                float* lse, void* workspace, size_t workspace_bytes,
-                                attn_stream_t stream) {
+                                int D, float softmax_scale, int window_left, float softcap,
+                                int num_splits, int dtype, const float* dq, const float* dk,
+                                const float* dv, void* o, float* lse, void* workspace,
+                                size_t workspace_bytes, attn_stream_t stream) {
     (void)dq;
     (void)dk;
     (void)dv;
     if (!q || !k_cache || !v_cache || !block_table || !seqused_k || !o) return ATTN_ERR_INVALID_ARG;
+    {
+        // the query is the newest token: the window is a causal one by construction
+        const attn_status_t ms = check_score_mods(ATTN_MASK_CAUSAL, window_left, softcap);
+        if (ms != ATTN_OK) return ms;
+    }
+    const int window = window_left < 0 ? -1 : window_left;
     if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
     if (num_blocks <= 0 || max_blocks_per_seq <= 0) return ATTN_ERR_INVALID_ARG;
     if (!dtype_ok(dtype)) return ATTN_ERR_INVALID_ARG;
@@ -655,7 +697,7 @@ attn_status_t attn_decode_paged(const void* q, const void* k_cache, const void* 
     if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o))
         return ATTN_ERR_INVALID_ARG;
     int ns, tps;
-    decode_splits(B, Hkv, max_blocks_per_seq * block_size, num_splits, &ns, &tps);
+    decode_splits(B, Hkv, decode_span(max_blocks_per_seq * block_size, window), num_splits, &ns, &tps);
     const size_t need = attn_decode_workspace_size(B, Hq, Hkv, D, max_blocks_per_seq, block_size,
                                                    num_splits);
     if (ns > 1 && !use_page_stream(B, Hq, Hkv, D, num_splits)) {
@@ -695,6 +737,8 @@ attn_status_t attn_decode_paged(const void* q, const void* k_cache, const void* 
         pa.max_blocks = max_blocks_per_seq;
         pa.seqused_k = seqused_k;
         pa.scale = resolve_scale(softmax_scale, D);
+        pa.window = window;
+        pa.softcap = softcap;
         pa.o_part = static_cast<float*>(workspace);
         pa.lse_part = pa.o_part + slots * Hq * D;
         pa.meta = reinterpret_cast<int*>(pa.lse_part + slots * Hq);
@@ -725,6 +769,8 @@ attn_status_t attn_decode_paged(const void* q, const void* k_cache, const void* 
     a.tokens_per_split = tps;
     a.num_splits = ns;
     a.scale = resolve_scale(softmax_scale, D);
+    a.window = window;
+    a.softcap = softcap;
     a.o = static_cast<__nv_bfloat16*>(o);
     a.lse = lse;
     a.direct = ns == 1 ? 1 : 0;
@@ -765,8 +811,9 @@ attn_status_t attn_decode_paged_noalloc(const void* q, const void* k_cache, cons
     void* scratch = noalloc_scratch_address(dev);
     if (!scratch) return ATTN_ERR_CUDA;
     return attn_decode_paged(q, k_cache, v_cache, block_table, max_blocks_per_seq, num_blocks,
-                             block_size, seqused_k, B, Hq, Hkv, D, softmax_scale, 0, dtype, nullptr,
-                             nullptr, nullptr, o, lse, scratch, kNoAllocScratchBytes, stream);
+                             block_size, seqused_k, B, Hq, Hkv, D, softmax_scale, -1, 0.0f, 0, dtype,
+                             nullptr, nullptr, nullptr, o, lse, scratch, kNoAllocScratchBytes,
+                             stream);
 }
 
 }  // extern "C"

@@ -37,6 +37,8 @@ struct DecodeArgs {
     int tokens_per_split;     // multiple of kDecStageTok
     int num_splits;
     float scale;
+    int window;               // sliding window: keys L-1-window .. L-1; < 0: none
+    float softcap;            // > 0: logit s -> softcap * tanh(s / softcap)
     float* o_part;            // [splits][B][Hq][D]
     float* lse_part;          // [splits][B][Hq]
     __nv_bfloat16* o;         // [B][Hq][D]  (direct mode)
@@ -74,9 +76,20 @@ __device__ __forceinline__ uint32_t swz_off(int row, int col, int rows) {
     return c * rows * 128 + row * 128 + ((piece ^ (row & 7)) << 4) + ((col & 7) << 1);
 }
 
+// The decode query is the newest of a sequence's L cached tokens, so a
+// sliding window of W keys lets it see keys L-1-W .. L-1.  First such key,
+// and the first key of the page holding it (where the key range streamed
+// from the cache starts).  W < 0: no window.
+__host__ __device__ __forceinline__ int win_first_key(int L, int W) {
+    return (W >= 0 && L > 0) ? max(0, L - 1 - W) : 0;
+}
+__host__ __device__ __forceinline__ int win_first_page_key(int L, int W) {
+    return win_first_key(L, W) / kPageRows * kPageRows;
+}
+
 // Work item -> (sequence, split, kv head) through the per-sequence split counts.
 struct DecItem {
-    int b, split, g, t_begin, t_end;
+    int b, split, g, t_begin, t_end, k_first;
 };
 
 // Sequence of L keys -> ceil(L / tps) splits of nearly equal size (multiples
@@ -84,7 +97,7 @@ struct DecItem {
 __host__ __device__ __forceinline__ int dec_nsplit(int L, int tps) { return (L + tps - 1) / tps; }
 
 __device__ __forceinline__ DecItem dec_item(int item, const int* prefix, int B, int Hkv, int tps,
-                                            const int* lens) {
+                                            const int* lens, int window) {
     DecItem it;
     it.g = item % Hkv;
     const int r = item / Hkv;
@@ -96,11 +109,13 @@ __device__ __forceinline__ DecItem dec_item(int item, const int* prefix, int B, 
     it.b = lo;
     it.split = r - prefix[lo];
     const int L = lens[lo];
-    const int n = max(dec_nsplit(L, tps), 1);
-    int sz = (L + n - 1) / n;
+    const int kb = win_first_page_key(L, window);   // page-aligned start of the streamed keys
+    const int n = max(dec_nsplit(L - kb, tps), 1);
+    int sz = (L - kb + n - 1) / n;
     sz = (sz + kDecStageTok - 1) / kDecStageTok * kDecStageTok;
-    it.t_begin = it.split * sz;
+    it.t_begin = kb + it.split * sz;
     it.t_end = min(L, it.t_begin + sz);
+    it.k_first = win_first_key(L, window);
     return it;
 }
 
@@ -139,7 +154,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
             int cnt = 0;
             if (b < a.B) {
                 const int L = min(max(a.seqused_k[b], 0), cap);
-                cnt = dec_nsplit(L, tps);
+                cnt = dec_nsplit(L - win_first_page_key(L, a.window), tps);
                 if (a.direct && cnt == 0) cnt = 1;    // a zero-length row is still written
             }
             int incl = cnt;
@@ -175,7 +190,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
         int ctr = 0;       // stages filled so far (ring position and phase)
         bool ok = true;
         for (int item = blockIdx.x; ok && item < total; item += gridDim.x) {
-            const DecItem it = dec_item(item, prefix, a.B, a.Hkv, tps, lenv);
+            const DecItem it = dec_item(item, prefix, a.B, a.Hkv, tps, lenv, a.window);
             const int nstage = (it.t_end > it.t_begin)
                                    ? (it.t_end - it.t_begin + kDecStageTok - 1) / kDecStageTok : 0;
             const int slot0 = it.t_begin / kPageRows;
@@ -230,10 +245,13 @@ __global__ void __launch_bounds__(kDecThreads, 2)
         // ---------------------------------------------------- consumers (a4-a6 for one token)
         const int gid = lane >> 2, t4 = lane & 3;
         const float sl2 = a.scale * kLog2e;
+        const bool capped = a.softcap > 0.0f;
+        const float cap_in = capped ? a.scale / a.softcap : 0.0f;
+        const float cap_out = capped ? a.softcap / a.scale : 0.0f;
         int ctr = 0;
         bool ok = true;
         for (int item = blockIdx.x; item < total; item += gridDim.x) {
-            const DecItem it = dec_item(item, prefix, a.B, a.Hkv, tps, lenv);
+            const DecItem it = dec_item(item, prefix, a.B, a.Hkv, tps, lenv, a.window);
             const int nstage = (it.t_end > it.t_begin)
                                    ? (it.t_end - it.t_begin + kDecStageTok - 1) / kDecStageTok : 0;
             // Q fragments (rows = the G query heads of KV head g; rows >= G are zero).
@@ -291,13 +309,22 @@ __global__ void __launch_bounds__(kDecThreads, 2)
                         mma_bf16_16816(sc[0], qa[kk], b0, b1);
                         mma_bf16_16816(sc[1], qa[kk], b2, b3);
                     }
+                    if (capped) {
+#pragma unroll
+                        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) sc[nt][e] = softcap_raw(sc[nt][e], cap_in, cap_out);
+                    }
                     float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
                     for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
                         for (int e = 0; e < 2; ++e) {
                             const int kv = tok0 + nt * 8 + 2 * t4 + e;
-                            if (kv >= it.t_end) { sc[nt][e] = -INFINITY; sc[nt][2 + e] = -INFINITY; }
+                            if (kv >= it.t_end || kv < it.k_first) {
+                                sc[nt][e] = -INFINITY;
+                                sc[nt][2 + e] = -INFINITY;
+                            }
                             mx0 = fmaxf(mx0, sc[nt][e]);
                             mx1 = fmaxf(mx1, sc[nt][2 + e]);
                         }
@@ -429,6 +456,8 @@ struct DecodePagesArgs {
     int max_blocks;
     const int* seqused_k;
     float scale;
+    int window;               // sliding window: keys L-1-window .. L-1; < 0: none
+    float softcap;            // > 0: logit s -> softcap * tanh(s / softcap)
     float* o_part;            // [grid + B][Hq][D]
     float* lse_part;          // [grid + B][Hq]
     int* meta;                // [B + 1] page prefix, then pages per CTA (written by CTA 0)
@@ -474,7 +503,7 @@ __global__ void __launch_bounds__(32 * (kPgMaxWarps + 1), 1)
             if (b < a.B) {
                 const int L = min(max(a.seqused_k[b], 0), cap);
                 lenv[b] = L;
-                cnt = (L + kPageRows - 1) / kPageRows;
+                cnt = (L + kPageRows - 1) / kPageRows - win_first_page_key(L, a.window) / kPageRows;
             }
             int incl = cnt;
 #pragma unroll
@@ -527,7 +556,7 @@ __global__ void __launch_bounds__(32 * (kPgMaxWarps + 1), 1)
             int phys = 0;
             if (base + lane < npages) {
                 const int b = seq_of(g);
-                const int slot = g - prefix[b];
+                const int slot = g - prefix[b] + win_first_page_key(lenv[b], a.window) / kPageRows;
                 phys = a.block_table[(long long)b * a.max_blocks + slot];
             }
             const int cnt = min(32, npages - base);
@@ -562,10 +591,13 @@ __global__ void __launch_bounds__(32 * (kPgMaxWarps + 1), 1)
         const int h = warp;
         const int gid = lane >> 2, t4 = lane & 3;
         const float sl2 = a.scale * kLog2e;
+        const bool capped = a.softcap > 0.0f;
+        const float cap_in = capped ? a.scale / a.softcap : 0.0f;
+        const float cap_out = capped ? a.softcap / a.scale : 0.0f;
         uint32_t qa[D / 16][4];
         float o[D / 8][4];
         float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.0f, l1 = 0.0f;
-        int b = -1, b_end = 0, L = 0;
+        int b = -1, b_end = 0, L = 0, kb = 0, kf = 0;
         auto load_q = [&](int bb) {
             const __nv_bfloat16* qb = a.q + ((long long)bb * a.Hq + (long long)h * G) * D;
 #pragma unroll
@@ -620,6 +652,8 @@ __global__ void __launch_bounds__(32 * (kPgMaxWarps + 1), 1)
                 b = seq_of(g);
                 b_end = prefix[b + 1];
                 L = lenv[b];
+                kb = win_first_page_key(L, a.window);
+                kf = win_first_key(L, a.window);
                 load_q(b);
                 reset();
             }
@@ -628,7 +662,7 @@ __global__ void __launch_bounds__(32 * (kPgMaxWarps + 1), 1)
                 ok = mbar_wait(&full[st], (i / NS) & 1, kErrDecFull);
                 ok = __all_sync(0xffffffffu, ok);
             }
-            const int tok0 = (g - prefix[b]) * kPageRows;     // first key of this page
+            const int tok0 = kb + (g - prefix[b]) * kPageRows;     // first key of this page
             uint8_t* sk = smem + st * SB;
             uint8_t* sv = sk + SB / 2;
             const int r0 = h * kPageRows;                      // this head's first row in the stage
@@ -654,13 +688,19 @@ __global__ void __launch_bounds__(32 * (kPgMaxWarps + 1), 1)
                     mma_bf16_16816(sc[0], qa[kk], b0, b1);
                     mma_bf16_16816(sc[1], qa[kk], b2, b3);
                 }
+                if (capped) {
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) sc[nt][e] = softcap_raw(sc[nt][e], cap_in, cap_out);
+                }
                 float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
                 for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
                     for (int e = 0; e < 2; ++e) {
                         const int kv = tok0 + nt * 8 + 2 * t4 + e;
-                        if (kv >= L) { sc[nt][e] = -INFINITY; sc[nt][2 + e] = -INFINITY; }
+                        if (kv >= L || kv < kf) { sc[nt][e] = -INFINITY; sc[nt][2 + e] = -INFINITY; }
                         mx0 = fmaxf(mx0, sc[nt][e]);
                         mx1 = fmaxf(mx1, sc[nt][2 + e]);
                     }
@@ -769,8 +809,8 @@ template <int D>
 __global__ void __launch_bounds__(D)
     decode_combine_kernel(const float* __restrict__ o_part, const float* __restrict__ lse_part,
                           const int* __restrict__ seqused_k, int B, int Hq, int num_splits,
-                          int tokens_per_split, int max_tokens, __nv_bfloat16* __restrict__ o,
-                          float* __restrict__ lse) {
+                          int tokens_per_split, int max_tokens, int window,
+                          __nv_bfloat16* __restrict__ o, float* __restrict__ lse) {
     __shared__ float w_s[kMaxSplits];
     __shared__ float lse_s;
     // Launched early (programmatic dependent launch): wait here for the split grid.
@@ -779,7 +819,7 @@ __global__ void __launch_bounds__(D)
     const int b = bh / Hq;
     const int d = threadIdx.x;
     const int L = min(max(seqused_k[b], 0), max_tokens);
-    const int ns = min(num_splits, (L + tokens_per_split - 1) / tokens_per_split);
+    const int ns = min(num_splits, dec_nsplit(L - win_first_page_key(L, window), tokens_per_split));
     const long long stride = (long long)B * Hq;
     if (threadIdx.x < 32) {
         const int lane = threadIdx.x;

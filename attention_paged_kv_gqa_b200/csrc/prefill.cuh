@@ -67,6 +67,8 @@ enum : int {
 struct PrefillArgs {
     int B, Hq, Hkv, group;
     int mask;
+    int window;          // causal only: keys i' - window .. i' (i' = i + Lk - Lq); < 0: none
+    float softcap;       // > 0: logit s -> softcap * tanh(s / softcap); 0: none
     int varlen;          // 1: rows addressed through cu_seqlens (batch coordinate 0)
     int paged;           // 1: K/V through block_table, 16-token pages
     int Lq, Lk;          // dense sizes (varlen == 0)
@@ -116,7 +118,9 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
     return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
-template <int D, bool FP8>
+// CAP: the score softcap is compiled in (a separate instance, so that the
+// uncapped kernel carries none of its code).
+template <int D, bool FP8, bool CAP>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const PrefillArgs a) {
@@ -247,6 +251,11 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         } else if (a.mask == kMaskCausal) {
             const int maxkey = rows_end - 1 + (Lk - Lq);
             if (maxkey >= 0) hi_t[t] = min(nkt, maxkey / kBN + 1);
+            if (a.window >= 0 && hi_t[t] > 0) {
+                // sliding window: the sub-tile's first row sees the earliest key
+                lo_t[t] = max(q0[t] + (Lk - Lq) - a.window, 0) / kBN;
+                if (lo_t[t] >= hi_t[t]) lo_t[t] = hi_t[t] = 0;
+            }
         } else {
             const int s = sched[2 * t], e = sched[2 * t + 1];
             if (s < e) {
@@ -460,14 +469,21 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         const bool row_ok = (t == 0 ? valid0 : valid1) && qi < Lq;
         const int head_t = head[t];
         float sl2 = a.scale * kLog2e;
+        float eff = a.scale;                 // logit = eff * (raw dot product)
         float out_scale = 1.0f;
         if constexpr (FP8) {
             sl2 *= __ldg(a.descale_q) * __ldg(a.descale_k);
+            eff *= __ldg(a.descale_q) * __ldg(a.descale_k);
             out_scale = __ldg(a.descale_v);
         }
+        const float cap_in = CAP ? eff / a.softcap : 0.0f;
+        const float cap_out = CAP ? a.softcap / eff : 0.0f;
         // Allowed keys of this row: [klo, khi).
         int klo = 0, khi = Lk;
-        if (a.mask == kMaskCausal) khi = min(Lk, qi + (Lk - Lq) + 1);
+        if (a.mask == kMaskCausal) {
+            khi = min(Lk, qi + (Lk - Lq) + 1);
+            if (a.window >= 0) klo = max(qi + (Lk - Lq) - a.window, 0);
+        }
         if (a.mask == kMaskPatch && row_ok) {
             klo = max(a.patch[2LL * (q_off + qi)], 0);
             khi = min(a.patch[2LL * (q_off + qi) + 1], Lk);
@@ -496,6 +512,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                 tmem_wait_ld();
 #pragma unroll
                 for (int c = 0; c < kBN; ++c) s[c] = __uint_as_float(u[c]);
+            }
+            if constexpr (CAP) {
+#pragma unroll
+                for (int c = 0; c < kBN; ++c) s[c] = softcap_raw(s[c], cap_in, cap_out);
             }
             const int kbase = j * kBN;
             if (kbase < klo || kbase + kBN > khi) {

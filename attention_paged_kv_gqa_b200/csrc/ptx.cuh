@@ -290,6 +290,23 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
+// tanh(x) = 1 - 2 / (e^(2x) + 1), from the MUFU exp2 and a fast reciprocal:
+// absolute error about 1e-7 over the whole range (e^(2x) overflowing to inf
+// gives 1, underflowing to 0 gives -1).  tanh.approx.f32 would be off by up to
+// ~5e-4 relative, i.e. 2.5e-2 in a logit capped at 50 -- too coarse for the
+// LSE bound of 1e-3.
+__device__ __forceinline__ float tanh_ex2(float x) {
+    const float e = ex2(x * 2.88539008177792681f);   // 2 log2(e)
+    return 1.0f - __fdividef(2.0f, e + 1.0f);
+}
+
+// Score softcap applied to a raw dot product q.k whose softmax logit is
+// eff * q.k: returns (c / eff) * tanh(eff * q.k / c), the raw value whose
+// logit is c * tanh(logit / c).  k_in = eff / c, k_out = c / eff.
+__device__ __forceinline__ float softcap_raw(float qk, float k_in, float k_out) {
+    return k_out * tanh_ex2(qk * k_in);
+}
+
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
     float r;
     asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));

@@ -46,6 +46,19 @@
  *    ATTN_MASK_PATCH allows key j for query i iff start_i <= j < end_i, with the
  *    sequence-local interval [start_i, end_i) given per query.  A query with no
  *    allowed key gets O = 0 and LSE = -inf.
+ *  - Sliding window and softcap (the "local window on/off" and "softcap 0/50"
+ *    options of the parity matrix in "[CUDA] PagedAttention: add SM<80 fp16
+ *    fallback via memory-efficient attention", Testing; nanochat's SSSL
+ *    window pattern in "FA3 loader reports success on Blackwell (sm_120) then
+ *    dies at first kernel launch"):
+ *      window_left >= 0 keeps, for the causal mask only, the keys
+ *        i' - window_left <= j <= i'   (i' = i + Lk - Lq, the row's diagonal);
+ *        a negative window_left means no window; with another mask it
+ *        returns ATTN_ERR_UNSUPPORTED.
+ *      softcap > 0 replaces each scaled logit s = scale * q.k (for fp8 the
+ *        dequantised one) by softcap * tanh(s / softcap) before the softmax
+ *        and the LSE; 0 means none; negative or non-finite values return
+ *        ATTN_ERR_INVALID_ARG.
  *  - Stream: `stream` is a cudaStream_t (NULL = legacy default stream).
  */
 #ifndef ATTN_B200_H
@@ -117,7 +130,7 @@ attn_status_t attn_fwd_dense(
     const void *q, const void *k, const void *v, void *o, float *lse,
     int B, int Lq, int Lk, int num_heads_q, int num_heads_kv, int head_dim,
     const int64_t *strides_q, const int64_t *strides_k, const int64_t *strides_v,
-    float softmax_scale, int mask, int dtype,
+    float softmax_scale, int mask, int window_left, float softcap, int dtype,
     const float *descale_q, const float *descale_k, const float *descale_v,
     attn_stream_t stream);
 
@@ -147,6 +160,7 @@ attn_status_t attn_fwd_varlen_paged(
     int B, int total_q, int total_k, int max_seqlen_q,
     int num_heads_q, int num_heads_kv, int head_dim,
     float softmax_scale, int mask, const int32_t *patch_kv_range,
+    int window_left, float softcap,
     int dtype, const float *descale_q, const float *descale_k, const float *descale_v,
     void *o, float *lse, void *workspace, size_t workspace_bytes, attn_stream_t stream);
 
@@ -160,7 +174,9 @@ size_t attn_decode_workspace_size(int B, int num_heads_q, int num_heads_kv, int 
 
 /*
  * Paged decode: one query token per sequence, split-KV with an LSE-weighted
- * combine.  Non-causal over the sequence's cached keys.
+ * combine.  The query is the newest of the sequence's cached keys and sees
+ * all of them, or with window_left >= 0 only keys L-1-window_left .. L-1
+ * (L = seqused_k[b]); softcap as above.
  *   q            [B, Hq, D] bf16, contiguous.
  *   k_cache/v_cache, block_table, block_size: as in attn_fwd_varlen_paged.
  *   seqused_k    int32 [B], keys cached per sequence (0 gives O = 0, LSE = -inf).
@@ -174,7 +190,7 @@ attn_status_t attn_decode_paged(
     const void *q, const void *k_cache, const void *v_cache, const int32_t *block_table,
     int max_blocks_per_seq, int num_blocks, int block_size, const int32_t *seqused_k,
     int B, int num_heads_q, int num_heads_kv, int head_dim, float softmax_scale,
-    int num_splits, int dtype,
+    int window_left, float softcap, int num_splits, int dtype,
     const float *descale_q, const float *descale_k, const float *descale_v,
     void *o, float *lse, void *workspace, size_t workspace_bytes, attn_stream_t stream);
 
@@ -187,7 +203,8 @@ attn_status_t attn_decode_paged(
  * allocation and exposes no allocator, or a latency-critical serving loop
  * whose memory is sized once at start-up and which must not reach
  * cudaMalloc (an implicit synchronisation) while it runs.
- *   Arguments: as attn_decode_paged, without num_splits and workspace.
+ *   Arguments: as attn_decode_paged, without window_left, softcap, num_splits
+ *   and workspace (no sliding window, no softcap).
  *   Limits: requests whose split-KV partials need more than 8 MiB (about
  *   (SMs + B) * Hq * (head_dim + 1) * 4 bytes) return ATTN_ERR_SCRATCH_LIMIT;
  *   shapes outside the page-stream decode (more than 8 KV heads, more than 16

@@ -58,17 +58,17 @@ def _strides():
 
 def test_null_pointers_rejected_before_launch(L):
     st = L.attn_fwd_dense(None, None, None, None, None, 1, 128, 128, 2, 2, 64, _strides(),
-                          _strides(), _strides(), 0.0, 1, 0, None, None, None, None)
+                          _strides(), _strides(), 0.0, 1, -1, 0.0, 0, None, None, None, None)
     assert st == 1
 
 
 def test_bad_group_and_head_dim(L):
     p = ctypes.c_void_p(1 << 20)
     st = L.attn_fwd_dense(p, p, p, p, None, 1, 128, 128, 3, 2, 64, _strides(), _strides(),
-                          _strides(), 0.0, 1, 0, None, None, None, None)
+                          _strides(), 0.0, 1, -1, 0.0, 0, None, None, None, None)
     assert st == 1                     # Hq % Hkv != 0
     st = L.attn_fwd_dense(p, p, p, p, None, 1, 128, 128, 2, 2, 96, _strides(), _strides(),
-                          _strides(), 0.0, 1, 0, None, None, None, None)
+                          _strides(), 0.0, 1, -1, 0.0, 0, None, None, None, None)
     assert st == 2                     # head_dim 96 unsupported
 
 
@@ -76,11 +76,11 @@ def test_misaligned_pointer_and_fp8_without_descale(L):
     p = ctypes.c_void_p(1 << 20)
     bad = ctypes.c_void_p((1 << 20) + 8)
     st = L.attn_fwd_dense(bad, p, p, p, None, 1, 128, 128, 2, 2, 64, _strides(), _strides(),
-                          _strides(), 0.0, 1, 0, None, None, None, None)
+                          _strides(), 0.0, 1, -1, 0.0, 0, None, None, None, None)
     assert st == 1
     s128 = (ctypes.c_int64 * 3)(128 * 2 * 128, 2 * 128, 128)
-    st = L.attn_fwd_dense(p, p, p, p, None, 1, 128, 128, 2, 2, 128, s128, s128, s128, 0.0, 1, 1,
-                          None, None, None, None)
+    st = L.attn_fwd_dense(p, p, p, p, None, 1, 128, 128, 2, 2, 128, s128, s128, s128, 0.0, 1, -1, 0.0,
+                          1, None, None, None, None)
     assert st == 1
 
 
@@ -89,11 +89,13 @@ def test_paged_block_size_and_patch_requirements(L):
     cu = ctypes.c_void_p(1 << 21)
     # block_size 32 -> unsupported
     st = L.attn_fwd_varlen_paged(p, p, p, p, 4, 100, 32, cu, None, cu, 1, 16, 0, 16, 2, 2, 64,
-                                 0.0, 1, None, 0, None, None, None, p, None, None, 0, None)
+                                 0.0, 1, None, -1, 0.0, 0, None, None, None, p, None, None, 0,
+                                 None)
     assert st == 2
     # patch mask without ranges -> invalid
     st = L.attn_fwd_varlen_paged(p, p, p, p, 4, 100, 16, cu, None, cu, 1, 16, 0, 16, 2, 2, 64,
-                                 0.0, 2, None, 0, None, None, None, p, None, None, 0, None)
+                                 0.0, 2, None, -1, 0.0, 0, None, None, None, p, None, None, 0,
+                                 None)
     assert st == 1
 
 
@@ -103,6 +105,25 @@ def test_decode_workspace_size_and_limits(L):
     assert L.attn_decode_workspace_size(0, 32, 8, 128, 512, 16, 0) == 0
     p = ctypes.c_void_p(1 << 20)
     # group of 32 query heads per KV head is beyond the decode kernel's 16 rows
-    st = L.attn_decode_paged(p, p, p, p, 4, 100, 16, p, 1, 32, 1, 128, 0.0, 1, 0, None, None,
-                             None, p, None, p, 1 << 20, None)
+    st = L.attn_decode_paged(p, p, p, p, 4, 100, 16, p, 1, 32, 1, 128, 0.0, -1, 0.0, 1, 0, None,
+                             None, None, p, None, p, 1 << 20, None)
     assert st == 2
+
+
+def test_window_and_softcap_rules(L):
+    """A window needs the causal mask; a softcap must be finite and >= 0 (before any launch)."""
+    p = ctypes.c_void_p(1 << 20)
+    dense = lambda mask, w, c: L.attn_fwd_dense(p, p, p, p, None, 1, 128, 128, 2, 2, 64, _strides(),
+                                                _strides(), _strides(), 0.0, mask, w, c, 0, None,
+                                                None, None, None)
+    assert dense(0, 16, 0.0) == 2                  # window without the causal mask
+    assert dense(1, 16, -1.0) == 1                 # negative softcap
+    assert dense(1, -1, float("nan")) == 1
+    assert dense(1, -1, float("inf")) == 1
+    cu = ctypes.c_void_p(1 << 21)
+    st = L.attn_fwd_varlen_paged(p, p, p, p, 4, 100, 16, cu, None, cu, 1, 16, 0, 16, 2, 2, 64,
+                                 0.0, 2, p, 8, 0.0, 0, None, None, None, p, None, None, 0, None)
+    assert st == 2                                 # window with the patch mask
+    st = L.attn_decode_paged(p, p, p, p, 4, 100, 16, p, 1, 8, 2, 128, 0.0, 5, -2.0, 0, 0, None,
+                             None, None, p, None, p, 1 << 20, None)
+    assert st == 1                                 # negative softcap in decode
