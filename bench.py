@@ -12,6 +12,9 @@ Carried in the same line:
                  Hq=32, Hkv=8, D=128 -> TFLOP/s (4*D*allowed pairs per head)
   "prefill_fp8": fp8 e4m3 dense causal B=4, H=16, L=4096, D=128 -> TFLOP/s,
                  with the bf16 kernel on the same data beside it.
+  "window_softcap": the decode and varlen prefill workloads again with a
+                 sliding window of 1024 keys and a softcap of 50 (GB/s and
+                 TFLOP/s over the keys inside each window only).
 
 Timing: W warm-up steps, then K steps each bracketed by CUDA events on the
 launching stream, a 256 MiB L2 flush between steps outside the events, and a
@@ -76,7 +79,8 @@ def parse_args():
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-prefill", action="store_true")
-    p.add_argument("--workload", choices=["all", "decode", "prefill", "fp8"], default="all",
+    p.add_argument("--workload", choices=["all", "decode", "prefill", "fp8", "window"],
+                   default="all",
                    help="run only one workload (profiling runs); the JSON line then carries "
                         "only what ran")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -235,6 +239,24 @@ def causal_flops(lens, Hq, D):
     return float(4 * D * Hq * (lens * (lens + 1) // 2).sum())
 
 
+def window_causal_flops(lens, Hq, D, window):
+    """Allowed pairs of a causal sliding window: row i sees min(i + 1, window + 1) keys."""
+    pairs = 0
+    for L in np.asarray(lens, np.int64):
+        full = min(int(L), window + 1)          # rows 0 .. full-1 see i + 1 keys
+        pairs += full * (full + 1) // 2 + (int(L) - full) * (window + 1)
+    return float(4 * D * Hq * pairs)
+
+
+def window_decode_bytes(t, Hq, Hkv, D, window):
+    """decode_bytes over the keys inside each sequence's window (newest query token)."""
+    lens = np.minimum(t["seqused_k"].numpy().astype(np.int64), window + 1)
+    B = len(lens)
+    kv = int(lens.sum()) * Hkv * D * 2 * 2
+    pages = int(((lens + 15) // 16).sum()) * 4
+    return kv + B * Hq * D * 2 * 2 + B * Hq * 4 + pages + B * 4
+
+
 # --------------------------------------------------------------------------- CPU oracle legs
 def oracle_decode_sample(w, target_tokens=8192, offset=0):
     """Runs the fp64 oracle on a bounded sample of the decode batch; returns (seconds, bytes)."""
@@ -338,6 +360,8 @@ def run_ours(args, rank, world, local):
         run_prefill(args, A, W, dev, world, flush, peaks, peak_kind, line)
     if args.workload in ("all", "fp8") and not args.no_prefill:
         run_fp8(args, A, W, dev, world, flush, peaks, peak_kind, line)
+    if args.workload in ("all", "window") and not args.no_prefill:
+        run_window(args, A, W, dev, world, flush, peaks, peak_kind, line)
     if args.workload in ("all", "decode") and rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
     if rank == 0:
@@ -488,6 +512,73 @@ def run_fp8(args, A, W, dev, world, flush, peaks, peak_kind, line):
                      "peak_kind": peak_kind + " bf16 x 2 (nominal fp8/bf16 ratio)"},
     }
     del d8
+
+
+WINDOW, SOFTCAP = 1024, 50.0
+
+
+def run_window(args, A, W, dev, world, flush, peaks, peak_kind, line):
+    """Decode and varlen prefill with a sliding window, a softcap, and both."""
+    w = W.paged_decode(seed=args.seed)
+    t, P = w.tensors, w.params
+    d = {k: v.to(dev) for k, v in t.items()}
+    ws = torch.empty(max(A.attn_decode_workspace_size(P["B"], P["Hq"], P["Hkv"], P["D"],
+                                                      P["max_blocks_per_seq"]), 16),
+                     dtype=torch.uint8, device=dev)
+    o = torch.empty(P["B"], P["Hq"], P["D"], dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(P["B"], P["Hq"], dtype=torch.float32, device=dev)
+    out = {"window_left": WINDOW, "softcap": SOFTCAP}
+    for name, wl, cap in (("decode_window", WINDOW, 0.0), ("decode_softcap", -1, SOFTCAP),
+                          ("decode_window_softcap", WINDOW, SOFTCAP)):
+        def dec_step():
+            A.attn_decode_paged(d["q"], d["k_cache"], d["v_cache"], d["block_table"],
+                                d["seqused_k"], scale=P["scale"], window_left=wl, softcap=cap,
+                                out=o, lse=lse, workspace=ws)
+
+        dms = statistics.mean(time_steps(dec_step, args.steps, args.warmup, world, flush))
+        nb = (window_decode_bytes(t, P["Hq"], P["Hkv"], P["D"], wl) if wl >= 0
+              else decode_bytes(t, P["Hq"], P["Hkv"], P["D"]))
+        gbs = nb / (dms * 1e-3) / 1e9
+        out[name] = {"value": round(gbs, 2), "unit": "GB/s", "ms_per_step": round(dms, 5),
+                     "bytes_per_step": nb,
+                     "roofline": {"bound": "hbm", "achieved": round(gbs, 1),
+                                  "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                  "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": None,
+                                  "peak_kind": peak_kind}}
+    del d
+
+    wp = W.varlen_paged_prefill(seed=args.seed)
+    tp, Pp = wp.tensors, wp.params
+    dp = {k: v.to(dev) for k, v in tp.items()}
+    op = torch.empty(Pp["total_q"], Pp["Hq"], Pp["D"], dtype=torch.bfloat16, device=dev)
+    lp = torch.empty(Pp["Hq"], Pp["total_q"], dtype=torch.float32, device=dev)
+    lens = tp["seqused_k"].numpy()
+    for name, wl, cap in (("prefill_window", WINDOW, 0.0), ("prefill_softcap", -1, SOFTCAP),
+                          ("prefill_window_softcap", WINDOW, SOFTCAP)):
+        def pf_step():
+            A.attn_fwd_varlen_paged(dp["q"], dp["k_cache"], dp["v_cache"],
+                                    cu_seqlens_q=dp["cu_seqlens_q"],
+                                    max_seqlen_q=Pp["max_seqlen_q"],
+                                    block_table=dp["block_table"], seqused_k=dp["seqused_k"],
+                                    mask=A.MASK_CAUSAL, scale=Pp["scale"], window_left=wl,
+                                    softcap=cap, out=op, lse=lp)
+
+        pms = statistics.mean(time_steps(pf_step, args.steps, args.warmup, world, flush))
+        fl = (window_causal_flops(lens, Pp["Hq"], Pp["D"], wl) if wl >= 0
+              else causal_flops(lens, Pp["Hq"], Pp["D"]))
+        tf = fl / (pms * 1e-3) / 1e12
+        out[name] = {"value": round(tf, 2), "unit": "TFLOP/s", "ms_per_step": round(pms, 5),
+                     "flops_per_step": fl,
+                     "roofline": {"bound": "tensor", "achieved": round(tf, 1),
+                                  "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                                  "frac": round(tf / peaks["bf16_tflops"], 4), "traffic": None,
+                                  "peak_kind": peak_kind}}
+    del dp
+    out["workloads"] = ("the paged GQA decode and varlen paged GQA prefill workloads above, "
+                        "with window_left %d (decode: keys L-1-%d .. L-1) and/or softcap %g; "
+                        "work counted over the keys inside each window only" % (WINDOW, WINDOW,
+                                                                                 SOFTCAP))
+    line["window_softcap"] = out
 
 
 def cpu_baseline(w):
