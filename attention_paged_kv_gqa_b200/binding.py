@@ -62,6 +62,11 @@ def lib():
         L.attn_decode_paged.restype = I
         L.attn_decode_paged_noalloc.argtypes = [P, P, P, P, I, I, I, P, I, I, I, I, F, I, P, P, P]
         L.attn_decode_paged_noalloc.restype = I
+        L.attn_kv_append_paged.argtypes = [P, P, P, P, P, I, I, I, P, P, P, I, I, I, I, I, P]
+        L.attn_kv_append_paged.restype = I
+        L.attn_decode_paged_append.argtypes = [P, P, P, P, P, P, I, I, I, P, P, I, I, I, I, F, I, F,
+                                               I, I, P, P, P, Z, P]
+        L.attn_decode_paged_append.restype = I
         _lib = L
     return _lib
 
@@ -236,3 +241,52 @@ def attn_decode_paged_noalloc(q, k_cache, v_cache, block_table, seqused_k, *, sc
                                          _dtype_code(q), _ptr(out), _ptr(lse), _stream(stream))
     _check(st, "attn_decode_paged_noalloc")
     return out, lse
+
+
+def attn_kv_append_paged(k_new, v_new, k_cache, v_cache, block_table, seqused_k, *,
+                         cu_seqlens_new=None, seqused_k_out=None, stream=None):
+    """Writes new tokens' K/V ([total_new, Hkv, D]) into the paged cache in place.
+
+    Sequence b's i-th new token goes to position seqused_k[b] + i.  Returns
+    seqused_k_out (lengths after), allocated here when not given.
+    cu_seqlens_new None means one new token per sequence.
+    """
+    total_new, Hkv, D = k_new.shape
+    B = seqused_k.numel()
+    num_blocks, block_size = k_cache.shape[0], k_cache.shape[1]
+    if seqused_k_out is None:
+        seqused_k_out = torch.empty_like(seqused_k)
+    st = lib().attn_kv_append_paged(_ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache),
+                                    _ptr(block_table), block_table.shape[1], num_blocks,
+                                    block_size, _ptr(cu_seqlens_new), _ptr(seqused_k),
+                                    _ptr(seqused_k_out), B, total_new, Hkv, D, _dtype_code(k_new),
+                                    _stream(stream))
+    _check(st, "attn_kv_append_paged")
+    return seqused_k_out
+
+
+def attn_decode_paged_append(q, k_new, v_new, k_cache, v_cache, block_table, seqused_k, *,
+                             seqused_k_out=None, scale=None, num_splits=0, window_left=-1,
+                             softcap=0.0, out=None, lse=None, workspace=None, return_lse=True,
+                             stream=None):
+    """Appends one token per sequence (k_new/v_new [B, Hkv, D]) to the paged cache, then
+    decodes q [B, Hq, D] over the updated cache.  Returns (o, lse, seqused_k_out)."""
+    B, Hq, D = q.shape
+    num_blocks, block_size, Hkv = k_cache.shape[0], k_cache.shape[1], k_cache.shape[2]
+    mbps = block_table.shape[1]
+    if seqused_k_out is None:
+        seqused_k_out = torch.empty_like(seqused_k)
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=torch.bfloat16, device=q.device)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    ws_bytes = attn_decode_workspace_size(B, Hq, Hkv, D, mbps, block_size, num_splits)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=q.device)
+    st = lib().attn_decode_paged_append(
+        _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), mbps,
+        num_blocks, block_size, _ptr(seqused_k), _ptr(seqused_k_out), B, Hq, Hkv, D, _scale(scale),
+        int(window_left), float(softcap), int(num_splits), _dtype_code(q), _ptr(out), _ptr(lse),
+        _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(st, "attn_decode_paged_append")
+    return out, lse, seqused_k_out

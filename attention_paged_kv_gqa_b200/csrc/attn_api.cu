@@ -21,6 +21,7 @@
 #include "attn_b200.h"
 #include "decode.cuh"
 #include "prefill.cuh"
+#include "append.cuh"
 
 using namespace attn;
 
@@ -191,6 +192,33 @@ attn_status_t launch_status() {
     return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
+// Launches `kernel` on `st`; with `pdl` as a programmatic dependent of the
+// kernel launched before it on the stream (the kernel must griddepcontrol.wait).
+template <typename... KArgs, typename... Args>
+attn_status_t launch_maybe_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                               cudaStream_t st, bool pdl, Args... args) {
+    if (!pdl) {
+        kernel<<<grid, block, smem, st>>>(args...);
+        return launch_status();
+    }
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kernel, args...) != cudaSuccess) {
+        cudaGetLastError();
+        return ATTN_ERR_CUDA;
+    }
+    return ATTN_OK;
+}
+
 // ------------------------------------------------------------------ prefill dispatch
 template <int D, bool FP8, bool CAP>
 attn_status_t launch_prefill_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
@@ -261,7 +289,7 @@ bool decode_geometry(int G, int B, int* ns_out, int* ctas_per_sm, int* smem_out)
 template <int D>
 attn_status_t launch_decode(const CUtensorMap& mk, const CUtensorMap& mv, DecodeArgs a,
                             int sms, long long items_max, cudaStream_t st, const int32_t* seqused_k,
-                            int max_tokens) {
+                            int max_tokens, bool pdl = false) {
     static std::atomic<uint64_t> attr_mask{0};   // one bit per device
     int dev = 0;
     cudaGetDevice(&dev);
@@ -275,8 +303,8 @@ attn_status_t launch_decode(const CUtensorMap& mk, const CUtensorMap& mv, Decode
     if (!decode_geometry<D>(a.group, a.B, &ns, &per_sm, &smem)) return ATTN_ERR_UNSUPPORTED;
     a.nstages = ns;
     const int grid = (int)std::min<long long>((long long)sms * per_sm, std::max<long long>(items_max, 1));
-    decode_split_kernel<D><<<grid, kDecThreads, smem, st>>>(mk, mv, a);
-    attn_status_t s = launch_status();
+    attn_status_t s = launch_maybe_pdl(decode_split_kernel<D>, dim3(grid), dim3(kDecThreads), smem, st,
+                                       pdl, mk, mv, a);
     if (s != ATTN_OK || a.direct) return s;
     // The combine kernel is launched as a programmatic dependent of the split
     // kernel: it is scheduled while the split grid runs and waits on the grid
@@ -336,7 +364,8 @@ void* noalloc_scratch_address(int dev) {
 
 template <int D>
 attn_status_t launch_decode_pages(const CUtensorMap& mk, const CUtensorMap& mv, const DecodePagesArgs& a,
-                                  int grid, cudaStream_t st, __nv_bfloat16* o, float* lse) {
+                                  int grid, cudaStream_t st, __nv_bfloat16* o, float* lse,
+                                  bool pdl = false) {
     static std::atomic<uint64_t> attr_mask{0};   // one bit per device
     int dev = 0;
     cudaGetDevice(&dev);
@@ -347,8 +376,8 @@ attn_status_t launch_decode_pages(const CUtensorMap& mk, const CUtensorMap& mv, 
         attr_mask.fetch_or(bit);
     }
     const int smem = DecodePagesCfg<D>::smem_bytes(a.Hkv, a.B, a.nstages);
-    decode_pages_kernel<D><<<grid, 32 * (a.Hkv + 1), smem, st>>>(mk, mv, a);
-    attn_status_t s = launch_status();
+    attn_status_t s = launch_maybe_pdl(decode_pages_kernel<D>, dim3(grid), dim3(32 * (a.Hkv + 1)),
+                                       smem, st, pdl, mk, mv, a);
     if (s != ATTN_OK) return s;
     cudaLaunchConfig_t cfg;
     std::memset(&cfg, 0, sizeof(cfg));
@@ -667,13 +696,16 @@ size_t attn_decode_workspace_size(int B, int Hq, int Hkv, int D, int max_blocks_
     return (size_t)ns * B * Hq * (D + 1) * sizeof(float) + 16;
 }
 
-attn_status_t attn_decode_paged(const void* q, const void* k_cache, const void* v_cache,
-                                const int32_t* block_table, int max_blocks_per_seq, int num_blocks,
-                                int block_size, const int32_t* seqused_k, int B, int Hq, int Hkv,
-                                int D, float softmax_scale, int window_left, float softcap,
-                                int num_splits, int dtype, const float* dq, const float* dk,
-                                const float* dv, void* o, float* lse, void* workspace,
-                                size_t workspace_bytes, attn_stream_t stream) {
+// The paged decode; with `pdl` its first kernel is launched as a programmatic
+// dependent of the kernel launched before it on the stream (a KV append).
+static attn_status_t decode_paged_impl(const void* q, const void* k_cache, const void* v_cache,
+                                       const int32_t* block_table, int max_blocks_per_seq,
+                                       int num_blocks, int block_size, const int32_t* seqused_k,
+                                       int B, int Hq, int Hkv, int D, float softmax_scale,
+                                       int window_left, float softcap, int num_splits, int dtype,
+                                       const float* dq, const float* dk, const float* dv, void* o,
+                                       float* lse, void* workspace, size_t workspace_bytes,
+                                       attn_stream_t stream, bool pdl) {
     (void)dq;
     (void)dk;
     (void)dv;
@@ -743,8 +775,9 @@ attn_status_t attn_decode_paged(const void* q, const void* k_cache, const void* 
         pa.lse_part = pa.o_part + slots * Hq * D;
         pa.meta = reinterpret_cast<int*>(pa.lse_part + slots * Hq);
         pa.nstages = decode_pages_stages(D, Hkv, B);
-        if (D == 128) return launch_decode_pages<128>(pk, pv, pa, grid, stp, static_cast<__nv_bfloat16*>(o), lse);
-        return launch_decode_pages<64>(pk, pv, pa, grid, stp, static_cast<__nv_bfloat16*>(o), lse);
+        if (D == 128)
+            return launch_decode_pages<128>(pk, pv, pa, grid, stp, static_cast<__nv_bfloat16*>(o), lse, pdl);
+        return launch_decode_pages<64>(pk, pv, pa, grid, stp, static_cast<__nv_bfloat16*>(o), lse, pdl);
     }
 
     const uint64_t rowk = (uint64_t)Hkv * D * 2;
@@ -782,12 +815,127 @@ attn_status_t attn_decode_paged(const void* q, const void* k_cache, const void* 
     const long long items_max = (long long)B * Hkv * ns;
     if (D == 128)
         s = launch_decode<128>(mk, mv, a, sm_count(dev), items_max, st, seqused_k,
-                               max_blocks_per_seq * block_size);
+                               max_blocks_per_seq * block_size, pdl);
     else
         s = launch_decode<64>(mk, mv, a, sm_count(dev), items_max, st, seqused_k,
-                              max_blocks_per_seq * block_size);
+                              max_blocks_per_seq * block_size, pdl);
     if (s != ATTN_OK) return s;
     return launch_status();
+}
+
+attn_status_t attn_decode_paged(const void* q, const void* k_cache, const void* v_cache,
+                                const int32_t* block_table, int max_blocks_per_seq, int num_blocks,
+                                int block_size, const int32_t* seqused_k, int B, int Hq, int Hkv,
+                                int D, float softmax_scale, int window_left, float softcap,
+                                int num_splits, int dtype, const float* dq, const float* dk,
+                                const float* dv, void* o, float* lse, void* workspace,
+                                size_t workspace_bytes, attn_stream_t stream) {
+    return decode_paged_impl(q, k_cache, v_cache, block_table, max_blocks_per_seq, num_blocks,
+                             block_size, seqused_k, B, Hq, Hkv, D, softmax_scale, window_left,
+                             softcap, num_splits, dtype, dq, dk, dv, o, lse, workspace,
+                             workspace_bytes, stream, false);
+}
+
+// Shared checks and launch of the KV append; `one_per_seq` means
+// cu_seqlens_new is absent and each sequence gets exactly one new token.
+static attn_status_t kv_append_launch(const void* k_new, const void* v_new, void* k_cache,
+                                      void* v_cache, const int32_t* block_table,
+                                      int max_blocks_per_seq, int num_blocks, int block_size,
+                                      const int32_t* cu_seqlens_new, const int32_t* seqused_k,
+                                      int32_t* seqused_k_out, int B, int total_new, int Hkv, int D,
+                                      int dtype, attn_stream_t stream) {
+    if (!k_new || !v_new || !k_cache || !v_cache || !block_table || !seqused_k)
+        return ATTN_ERR_INVALID_ARG;
+    if (B < 0 || total_new < 0 || Hkv <= 0 || D <= 0 || max_blocks_per_seq <= 0 || num_blocks <= 0)
+        return ATTN_ERR_INVALID_ARG;
+    if (!dtype_ok(dtype)) return ATTN_ERR_INVALID_ARG;
+    if (!cu_seqlens_new && total_new != B) return ATTN_ERR_INVALID_ARG;
+    if (seqused_k_out && (const void*)seqused_k_out == (const void*)seqused_k) return ATTN_ERR_INVALID_ARG;
+    if (block_size != kPageRows) return ATTN_ERR_UNSUPPORTED;
+    const long long row_bytes = (long long)D * elem_bytes(dtype);
+    if (row_bytes % 16) return ATTN_ERR_INVALID_ARG;
+    if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) || !aligned16(v_cache))
+        return ATTN_ERR_INVALID_ARG;
+    if ((long long)num_blocks * block_size * Hkv * row_bytes / 16 >= (1LL << 62)) return ATTN_ERR_UNSUPPORTED;
+    int dev = 0;
+    const attn_status_t dvs = current_device_ok(&dev);
+    if (dvs != ATTN_OK) return dvs;
+    if (B == 0) return ATTN_OK;
+    AppendArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.k_new = static_cast<const uint4*>(k_new);
+    a.v_new = static_cast<const uint4*>(v_new);
+    a.k_cache = static_cast<uint4*>(k_cache);
+    a.v_cache = static_cast<uint4*>(v_cache);
+    a.block_table = block_table;
+    a.max_blocks = max_blocks_per_seq;
+    a.num_blocks = num_blocks;
+    a.cu_new = cu_seqlens_new;
+    a.seqused_k = seqused_k;
+    a.seqused_k_out = seqused_k_out;
+    a.B = B;
+    a.total_new = total_new;
+    a.pieces_per_token = (int)((long long)Hkv * row_bytes / 16);
+    const int warps_per_block = kAppendThreads / 32;
+    const long long want = std::max<long long>((long long)std::max(total_new, B) + warps_per_block - 1,
+                                               warps_per_block) / warps_per_block;
+    const int grid = (int)std::min<long long>(want, (long long)sm_count(dev) * 8);
+    kv_append_kernel<<<grid, kAppendThreads, 0, static_cast<cudaStream_t>(stream)>>>(a);
+    return launch_status();
+}
+
+attn_status_t attn_kv_append_paged(const void* k_new, const void* v_new, void* k_cache,
+                                   void* v_cache, const int32_t* block_table,
+                                   int max_blocks_per_seq, int num_blocks, int block_size,
+                                   const int32_t* cu_seqlens_new, const int32_t* seqused_k,
+                                   int32_t* seqused_k_out, int B, int total_new, int num_heads_kv,
+                                   int head_dim, int dtype, attn_stream_t stream) {
+    return kv_append_launch(k_new, v_new, k_cache, v_cache, block_table, max_blocks_per_seq,
+                            num_blocks, block_size, cu_seqlens_new, seqused_k, seqused_k_out, B,
+                            total_new, num_heads_kv, head_dim, dtype, stream);
+}
+
+attn_status_t attn_decode_paged_append(const void* q, const void* k_new, const void* v_new,
+                                       void* k_cache, void* v_cache, const int32_t* block_table,
+                                       int max_blocks_per_seq, int num_blocks, int block_size,
+                                       const int32_t* seqused_k, int32_t* seqused_k_out, int B,
+                                       int Hq, int Hkv, int D, float softmax_scale,
+                                       int window_left, float softcap, int num_splits, int dtype,
+                                       void* o, float* lse, void* workspace,
+                                       size_t workspace_bytes, attn_stream_t stream) {
+    if (!seqused_k_out) return ATTN_ERR_INVALID_ARG;
+    // Validate the decode half before anything is launched (no partial work on a bad call).
+    if (!q || !o) return ATTN_ERR_INVALID_ARG;
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
+    if (!dtype_ok(dtype)) return ATTN_ERR_INVALID_ARG;
+    if (dtype != ATTN_BF16) return ATTN_ERR_UNSUPPORTED;
+    if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+    if (Hq / Hkv > kDecRows || B > kDecMaxSeqs) return ATTN_ERR_UNSUPPORTED;
+    {
+        const attn_status_t ms = check_score_mods(ATTN_MASK_CAUSAL, window_left, softcap);
+        if (ms != ATTN_OK) return ms;
+    }
+    if (!aligned16(q) || !aligned16(o)) return ATTN_ERR_INVALID_ARG;
+    if (B > 0) {
+        int ns, tps;
+        const int span = decode_span(max_blocks_per_seq * block_size, window_left < 0 ? -1 : window_left);
+        decode_splits(B, Hkv, span, num_splits, &ns, &tps);
+        const bool stream_pages = use_page_stream(B, Hq, Hkv, D, num_splits);
+        if (stream_pages || ns > 1) {
+            const size_t need = attn_decode_workspace_size(B, Hq, Hkv, D, max_blocks_per_seq,
+                                                           block_size, num_splits);
+            if (!workspace || !aligned16(workspace)) return ATTN_ERR_INVALID_ARG;
+            if (workspace_bytes < need) return ATTN_ERR_WORKSPACE_TOO_SMALL;
+        }
+    }
+    attn_status_t s = kv_append_launch(k_new, v_new, k_cache, v_cache, block_table,
+                                       max_blocks_per_seq, num_blocks, block_size, nullptr,
+                                       seqused_k, seqused_k_out, B, B, Hkv, D, dtype, stream);
+    if (s != ATTN_OK || B == 0) return s;
+    return decode_paged_impl(q, k_cache, v_cache, block_table, max_blocks_per_seq, num_blocks,
+                             block_size, seqused_k_out, B, Hq, Hkv, D, softmax_scale, window_left,
+                             softcap, num_splits, dtype, nullptr, nullptr, nullptr, o, lse,
+                             workspace, workspace_bytes, stream, true);
 }
 
 attn_status_t attn_decode_paged_noalloc(const void* q, const void* k_cache, const void* v_cache,

@@ -142,6 +142,9 @@ __global__ void __launch_bounds__(kDecThreads, 2)
 
     // Let the combine kernel launch now; it waits for this grid's results itself.
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    // Launched as a programmatic dependent of a KV append, wait for it before
+    // reading the lengths or the cache (a no-op for an ordinary launch).
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int tps = a.tokens_per_split;
@@ -493,6 +496,7 @@ __global__ void __launch_bounds__(32 * (kPgMaxWarps + 1), 1)
     uint64_t* empty = full + NS;
 
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");   // after a KV append (see above)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int cap = a.max_blocks * kPageRows;
     if (warp == 0) {

@@ -195,6 +195,55 @@ attn_status_t attn_decode_paged(
     void *o, float *lse, void *workspace, size_t workspace_bytes, attn_stream_t stream);
 
 /*
+ * Paged KV append: writes new tokens' keys and values into the paged cache
+ * (the ReshapeAndCache step of "[CUDA] PagedAttention: add SM<80 fp16
+ * fallback via memory-efficient attention", Implementation step 1; the K_new
+ * / AppendKV path of "Rope dim").  Sequence b holds seqused_k[b] cached tokens
+ * before the call; its i-th new token (row cu_seqlens_new[b] + i of k_new /
+ * v_new) is stored at cache position p = seqused_k[b] + i, i.e. row p % 16 of
+ * page block_table[b * max_blocks_per_seq + p / 16].  Nothing else in the
+ * cache is written.
+ *   k_new/v_new    [total_new, Hkv, D], contiguous, of `dtype` (bf16 or e4m3
+ *                  codes; the bytes are copied as they are).
+ *   k_cache/v_cache [num_blocks, block_size, Hkv, D], contiguous, same dtype.
+ *   cu_seqlens_new int32 [B+1] (NULL: exactly one new token per sequence,
+ *                  total_new == B).
+ *   seqused_k      int32 [B], lengths before the call (read only).
+ *   seqused_k_out  int32 [B] or NULL: receives seqused_k[b] + n_b.  It must
+ *                  not be the same buffer as seqused_k (ATTN_ERR_INVALID_ARG).
+ * Requirements: block_size == 16; head_dim * element bytes a multiple of 16;
+ * 16-byte aligned k_new, v_new and caches.  The appended positions of
+ * different sequences must map to different cache rows.  A position past a
+ * sequence's block table, or a page index outside [0, num_blocks), is not
+ * written: the kernel records code 501 (position) or 502 (page) in the device
+ * error word (attn_device_error) and copies the remaining tokens.
+ */
+attn_status_t attn_kv_append_paged(
+    const void *k_new, const void *v_new, void *k_cache, void *v_cache,
+    const int32_t *block_table, int max_blocks_per_seq, int num_blocks, int block_size,
+    const int32_t *cu_seqlens_new, const int32_t *seqused_k, int32_t *seqused_k_out,
+    int B, int total_new, int num_heads_kv, int head_dim, int dtype, attn_stream_t stream);
+
+/*
+ * One decode step with its KV append in one call: appends one new token per
+ * sequence (k_new/v_new [B, Hkv, D]) as attn_kv_append_paged does, then runs
+ * attn_decode_paged for q [B, Hq, D] over the updated cache, whose lengths
+ * the append writes to seqused_k_out (required; lengths before the call in
+ * seqused_k).  The decode is launched as a programmatic dependent of the
+ * append, so its launch overlaps the append and it waits for the append's
+ * writes on the device.  Arguments otherwise as attn_decode_paged (bf16).
+ * The decode's arguments are checked before the append is launched; should
+ * the decode still fail to launch, the append has already taken effect.
+ */
+attn_status_t attn_decode_paged_append(
+    const void *q, const void *k_new, const void *v_new, void *k_cache, void *v_cache,
+    const int32_t *block_table, int max_blocks_per_seq, int num_blocks, int block_size,
+    const int32_t *seqused_k, int32_t *seqused_k_out,
+    int B, int num_heads_q, int num_heads_kv, int head_dim, float softmax_scale,
+    int window_left, float softcap, int num_splits, int dtype,
+    void *o, float *lse, void *workspace, size_t workspace_bytes, attn_stream_t stream);
+
+/*
  * attn_decode_paged without any device allocation by the caller: the same
  * paged decode (automatic split choice), with its scratch taken from a fixed
  * 8 MiB array that this library keeps in device memory.  No counterpart on
