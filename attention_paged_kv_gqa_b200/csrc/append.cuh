@@ -66,13 +66,30 @@ __global__ void __launch_bounds__(kAppendThreads) kv_append_kernel(const AppendA
             if (lane == 0) record_error(kErrAppendPage);
             continue;
         }
-        const long long src = (long long)t * P;
-        const long long dst = ((long long)page * kPageRows + p % kPageRows) * P;
-        for (int i = lane; i < P; i += 32) {
-            const uint4 kv = __ldg(&a.k_new[src + i]);
-            const uint4 vv = __ldg(&a.v_new[src + i]);
-            a.k_cache[dst + i] = kv;
-            a.v_cache[dst + i] = vv;
+        const uint4* __restrict__ ks = a.k_new + (long long)t * P;
+        const uint4* __restrict__ vs = a.v_new + (long long)t * P;
+        uint4* __restrict__ kd = a.k_cache + ((long long)page * kPageRows + p % kPageRows) * P;
+        uint4* __restrict__ vd = a.v_cache + ((long long)page * kPageRows + p % kPageRows) * P;
+        // all of a lane's loads of a group are in flight before its stores
+        constexpr int U = 4;
+        for (int i0 = lane; i0 < P; i0 += 32 * U) {
+            uint4 kr[U], vr[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int i = i0 + 32 * u;
+                if (i < P) {
+                    kr[u] = __ldg(ks + i);
+                    vr[u] = __ldg(vs + i);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int i = i0 + 32 * u;
+                if (i < P) {
+                    kd[i] = kr[u];
+                    vd[i] = vr[u];
+                }
+            }
         }
     }
     if (a.seqused_k_out) {

@@ -15,6 +15,9 @@ Carried in the same line:
   "window_softcap": the decode and varlen prefill workloads again with a
                  sliding window of 1024 keys and a softcap of 50 (GB/s and
                  TFLOP/s over the keys inside each window only).
+  "kv_append":   paged KV append of every token of the varlen prefill
+                 workload (GB/s of new K/V read + cache rows written), and
+                 one decode step with its one-token append (GB/s as decode).
 
 Timing: W warm-up steps, then K steps each bracketed by CUDA events on the
 launching stream, a 256 MiB L2 flush between steps outside the events, and a
@@ -79,7 +82,7 @@ def parse_args():
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-prefill", action="store_true")
-    p.add_argument("--workload", choices=["all", "decode", "prefill", "fp8", "window"],
+    p.add_argument("--workload", choices=["all", "decode", "prefill", "fp8", "window", "append"],
                    default="all",
                    help="run only one workload (profiling runs); the JSON line then carries "
                         "only what ran")
@@ -362,6 +365,8 @@ def run_ours(args, rank, world, local):
         run_fp8(args, A, W, dev, world, flush, peaks, peak_kind, line)
     if args.workload in ("all", "window") and not args.no_prefill:
         run_window(args, A, W, dev, world, flush, peaks, peak_kind, line)
+    if args.workload in ("all", "append"):
+        run_append(args, A, W, dev, world, flush, peaks, peak_kind, line)
     if args.workload in ("all", "decode") and rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
     if rank == 0:
@@ -579,6 +584,76 @@ def run_window(args, A, W, dev, world, flush, peaks, peak_kind, line):
                         "work counted over the keys inside each window only" % (WINDOW, WINDOW,
                                                                                  SOFTCAP))
     line["window_softcap"] = out
+
+
+def run_append(args, A, W, dev, world, flush, peaks, peak_kind, line):
+    """Paged KV append at prefill size, and a decode step with its append."""
+    wp = W.varlen_paged_prefill(seed=args.seed)
+    tp, Pp = wp.tensors, wp.params
+    lens = tp["seqused_k"]
+    total, Hkv, D = Pp["total_q"], Pp["Hkv"], Pp["D"]
+    k_new = W.randn_bf16((total, Hkv, D), args.seed, 31).to(dev)   # every token's new K/V
+    v_new = W.randn_bf16((total, Hkv, D), args.seed, 32).to(dev)
+    kc, vc = tp["k_cache"].to(dev), tp["v_cache"].to(dev)
+    bt = tp["block_table"].to(dev)
+    zeros = torch.zeros_like(lens).to(dev)                   # sequences start empty
+    cu = tp["cu_seqlens_k"].to(dev)
+    after = torch.empty_like(zeros)
+
+    def app_step():
+        A.attn_kv_append_paged(k_new, v_new, kc, vc, bt, zeros, cu_seqlens_new=cu,
+                               seqused_k_out=after)
+
+    ams = statistics.mean(time_steps(app_step, args.steps, args.warmup, world, flush))
+    nbytes = 2 * 2 * total * Hkv * D * 2 + int(lens.numel()) * 4 * 3 + 4 * (lens.numel() + 1)
+    gbs = nbytes / (ams * 1e-3) / 1e9
+    del k_new, v_new, kc, vc
+
+    w = W.paged_decode(seed=args.seed)
+    t, P = w.tensors, w.params
+    # one more page-table slot of room per sequence is already there (L <= 8192 < 512 pages)
+    d = {k: v.to(dev) for k, v in t.items()}
+    g = torch.Generator().manual_seed(args.seed + 99)
+    kn = torch.randn(P["B"], P["Hkv"], P["D"], generator=g).to(torch.bfloat16).to(dev)
+    vn = torch.randn(P["B"], P["Hkv"], P["D"], generator=g).to(torch.bfloat16).to(dev)
+    # lengths one short of the workload's, so the appended token is the last cached one
+    before = (t["seqused_k"] - 1).clamp(min=0).to(dev)
+    after = torch.empty_like(before)
+    ws = torch.empty(max(A.attn_decode_workspace_size(P["B"], P["Hq"], P["Hkv"], P["D"],
+                                                      P["max_blocks_per_seq"]), 16),
+                     dtype=torch.uint8, device=dev)
+    o = torch.empty(P["B"], P["Hq"], P["D"], dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(P["B"], P["Hq"], dtype=torch.float32, device=dev)
+
+    def dec_step():
+        A.attn_decode_paged_append(d["q"], kn, vn, d["k_cache"], d["v_cache"], d["block_table"],
+                                   before, seqused_k_out=after, scale=P["scale"], out=o, lse=lse,
+                                   workspace=ws)
+
+    dms = statistics.mean(time_steps(dec_step, args.steps, args.warmup, world, flush))
+    lens_after = (t["seqused_k"] - 1).clamp(min=0) + 1
+    nb_dec = decode_bytes({"seqused_k": lens_after}, P["Hq"], P["Hkv"], P["D"]) + \
+        2 * 2 * P["B"] * P["Hkv"] * P["D"] * 2
+    dgbs = nb_dec / (dms * 1e-3) / 1e9
+    del d
+    line["kv_append"] = {
+        "prefill_size": {
+            "workload": "every token of the varlen paged prefill workload (%d tokens, Hkv=8, "
+                        "D=128, bf16) appended to empty sequences" % total,
+            "value": round(gbs, 2), "unit": "GB/s", "ms_per_step": round(ams, 5),
+            "bytes_per_step": nbytes,
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4),
+                         "traffic": None, "kernel": "kv_append_kernel", "peak_kind": peak_kind}},
+        "decode_step": {
+            "workload": "the paged GQA decode workload, each sequence appending its newest "
+                        "token in the same call (append + decode)",
+            "value": round(dgbs, 2), "unit": "GB/s", "ms_per_step": round(dms, 5),
+            "bytes_per_step": nb_dec,
+            "roofline": {"bound": "hbm", "achieved": round(dgbs, 1), "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": round(dgbs / peaks["hbm_gbs"], 4),
+                         "traffic": None, "peak_kind": peak_kind}},
+    }
 
 
 def cpu_baseline(w):
