@@ -59,6 +59,8 @@ def bind(lib):
                                     D, I, P, I, D, P, P, I, I]
     lib.attn_oracle_combine.restype = None
     lib.attn_oracle_combine.argtypes = [P, P, I, I, I, P, P]
+    lib.attn_oracle_bwd.restype = I
+    lib.attn_oracle_bwd.argtypes = [P, P, P, P, P, P, I, I, I, I, D, I, I, P, P, P, I]
     return lib
 
 
@@ -175,3 +177,43 @@ def combine(o_parts, lse_parts):
     lse = np.zeros(N, np.float64)
     lib.attn_oracle_combine(_ptr(op), _ptr(lp), S, N, D, _ptr(o), _ptr(lse))
     return o, lse
+
+
+def attn_bwd_varlen(q, k, v, do, *, cu_seqlens_q, cu_seqlens_k, num_heads_kv, scale,
+                    mask=MASK_NONE, window_left=-1, nthreads=None):
+    """Gradients of the varlen forward in fp64: (dQ [total_q, Hq, D], dK, dV [total_k, Hkv, D]).
+
+    q, do [total_q, Hq, D]; k, v [total_k, Hkv, D] (packed, no paging).  The
+    forward's O and LSE are recomputed exactly from q, k, v.
+    """
+    lib = _load()
+    qa, ka, va, da = _f64(q), _f64(k), _f64(v), _f64(do)
+    total_q, Hq, D = qa.shape
+    cq, ck = _i32(cu_seqlens_q), _i32(cu_seqlens_k)
+    B = len(cq) - 1
+    dq = np.zeros_like(qa)
+    dk = np.zeros_like(ka)
+    dv = np.zeros_like(va)
+    if scale is None or scale <= 0:
+        scale = default_scale(D)
+    rc = lib.attn_oracle_bwd(_ptr(qa), _ptr(ka), _ptr(va), _ptr(da), _ptr(cq), _ptr(ck), B, Hq,
+                             int(num_heads_kv), D, float(scale), int(mask), int(window_left),
+                             _ptr(dq), _ptr(dk), _ptr(dv), int(nthreads or os.cpu_count() or 1))
+    if rc != 0:
+        raise ValueError("oracle rejected its arguments (rc=%d)" % rc)
+    return dq, dk, dv
+
+
+def attn_bwd_dense(q, k, v, do, *, scale, causal, window_left=-1, nthreads=None):
+    """Dense [B, L, H, D] gradients in fp64: (dQ [B, Lq, Hq, D], dK, dV [B, Lk, Hkv, D])."""
+    qa, ka, va, da = _f64(q), _f64(k), _f64(v), _f64(do)
+    B, Lq, Hq, D = qa.shape
+    Lk, Hkv = ka.shape[1], ka.shape[2]
+    cq = np.arange(B + 1, dtype=np.int32) * Lq
+    ck = np.arange(B + 1, dtype=np.int32) * Lk
+    dq, dk, dv = attn_bwd_varlen(qa.reshape(B * Lq, Hq, D), ka.reshape(B * Lk, Hkv, D),
+                                 va.reshape(B * Lk, Hkv, D), da.reshape(B * Lq, Hq, D),
+                                 cu_seqlens_q=cq, cu_seqlens_k=ck, num_heads_kv=Hkv, scale=scale,
+                                 mask=MASK_CAUSAL if causal else MASK_NONE,
+                                 window_left=window_left, nthreads=nthreads)
+    return dq.reshape(B, Lq, Hq, D), dk.reshape(B, Lk, Hkv, D), dv.reshape(B, Lk, Hkv, D)

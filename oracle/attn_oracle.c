@@ -190,3 +190,108 @@ void attn_oracle_combine(const double *o_parts, const double *lse_parts, int S, 
         }
     }
 }
+
+/*
+ * Backward of the same forward (the gradients of the attention output, for
+ * the training path the BLT page runs through the FlexAttention autograd and
+ * the FlashAttnVarlenFunc backward of "Rope dim"), written out as the plain
+ * derivative of the definition above.  Packed varlen [total, heads, D]
+ * (no paging), masks none / causal (optionally windowed); no softcap.
+ *
+ * For sequence b, query head h (kv head g), query i and allowed key j:
+ *   P_ij     = exp(s_ij - LSE_i)                    the forward's probabilities
+ *   dV_j    += P_ij dO_i                            summed over the group's heads
+ *   dP_ij    = dO_i . v_j
+ *   Delta_i  = sum_j P_ij dP_ij                      (= dO_i . O_i)
+ *   dS_ij    = P_ij (dP_ij - Delta_i)
+ *   dQ_i     = scale * sum_j dS_ij k_j
+ *   dK_j    += scale * dS_ij q_i                    summed over the group's heads
+ * O, LSE are recomputed here from q, k, v (exactly, in fp64).  A row with no
+ * allowed key contributes nothing and gets dQ = 0.
+ *   q, do_ [total_q][Hq][D];  k, v [total_k][Hkv][D];  dq like q; dk, dv like k.
+ * Returns 0, or -1 for arguments it cannot interpret.
+ */
+int attn_oracle_bwd(const double *q, const double *k, const double *v, const double *do_,
+                    const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k, int B, int Hq,
+                    int Hkv, int D, double scale, int mask, int window_left, double *dq,
+                    double *dk, double *dv, int nthreads) {
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || Hq % Hkv != 0) return -1;
+    if (!cu_seqlens_q || !cu_seqlens_k) return -1;
+    if (mask != ORACLE_MASK_NONE && mask != ORACLE_MASK_CAUSAL) return -1;
+    if (window_left >= 0 && mask != ORACLE_MASK_CAUSAL) return -1;
+    const int group = Hq / Hkv;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+    (void)nthreads;
+#endif
+    int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(|| : bad)
+    for (long long task = 0; task < (long long)B * Hkv; ++task) {
+        const int b = (int)(task / Hkv), g = (int)(task % Hkv);
+        const int q0 = cu_seqlens_q[b], k0 = cu_seqlens_k[b];
+        const int Lq = cu_seqlens_q[b + 1] - q0, Lk = cu_seqlens_k[b + 1] - k0;
+        for (int j = 0; j < Lk; ++j)
+            for (int d = 0; d < D; ++d) {
+                dk[((long long)(k0 + j) * Hkv + g) * D + d] = 0.0;
+                dv[((long long)(k0 + j) * Hkv + g) * D + d] = 0.0;
+            }
+        double *s = (double *)malloc(sizeof(double) * (size_t)(Lk > 0 ? Lk : 1));
+        double *p = (double *)malloc(sizeof(double) * (size_t)(Lk > 0 ? Lk : 1));
+        double *dp = (double *)malloc(sizeof(double) * (size_t)(Lk > 0 ? Lk : 1));
+        if (!s || !p || !dp) { bad = 1; free(s); free(p); free(dp); continue; }
+        for (int h = g * group; h < (g + 1) * group; ++h) {
+            for (int i = 0; i < Lq; ++i) {
+                const double *qi = q + ((long long)(q0 + i) * Hq + h) * D;
+                const double *doi = do_ + ((long long)(q0 + i) * Hq + h) * D;
+                double *dqi = dq + ((long long)(q0 + i) * Hq + h) * D;
+                for (int d = 0; d < D; ++d) dqi[d] = 0.0;
+                /* scores, max and log-sum-exp of the row (the forward) */
+                double M = -INFINITY;
+                int any = 0;
+                for (int j = 0; j < Lk; ++j) {
+                    const double *kj = k + ((long long)(k0 + j) * Hkv + g) * D;
+                    double acc = 0.0;
+                    for (int d = 0; d < D; ++d) acc += qi[d] * kj[d];
+                    s[j] = acc * scale;
+                    if (!allowed(mask, i, j, Lq, Lk, NULL, window_left)) continue;
+                    if (!any || s[j] > M) M = s[j];
+                    any = 1;
+                }
+                if (!any) continue;
+                double Z = 0.0;
+                for (int j = 0; j < Lk; ++j)
+                    if (allowed(mask, i, j, Lq, Lk, NULL, window_left)) Z += exp(s[j] - M);
+                const double lse = M + log(Z);
+                /* P, dP and Delta */
+                double delta = 0.0;
+                for (int j = 0; j < Lk; ++j) {
+                    if (!allowed(mask, i, j, Lq, Lk, NULL, window_left)) { p[j] = 0.0; dp[j] = 0.0; continue; }
+                    p[j] = exp(s[j] - lse);
+                    const double *vj = v + ((long long)(k0 + j) * Hkv + g) * D;
+                    double acc = 0.0;
+                    for (int d = 0; d < D; ++d) acc += doi[d] * vj[d];
+                    dp[j] = acc;
+                    delta += p[j] * dp[j];
+                }
+                /* gradients */
+                for (int j = 0; j < Lk; ++j) {
+                    if (p[j] == 0.0) continue;
+                    const double ds = p[j] * (dp[j] - delta);
+                    const double *kj = k + ((long long)(k0 + j) * Hkv + g) * D;
+                    double *dkj = dk + ((long long)(k0 + j) * Hkv + g) * D;
+                    double *dvj = dv + ((long long)(k0 + j) * Hkv + g) * D;
+                    for (int d = 0; d < D; ++d) {
+                        dqi[d] += scale * ds * kj[d];
+                        dkj[d] += scale * ds * qi[d];
+                        dvj[d] += p[j] * doi[d];
+                    }
+                }
+            }
+        }
+        free(s);
+        free(p);
+        free(dp);
+    }
+    return bad ? -2 : 0;
+}
