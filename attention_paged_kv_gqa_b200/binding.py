@@ -67,6 +67,11 @@ def lib():
         L.attn_decode_paged_append.argtypes = [P, P, P, P, P, P, I, I, I, P, P, I, I, I, I, F, I, F,
                                                I, I, P, P, P, Z, P]
         L.attn_decode_paged_append.restype = I
+        L.attn_bwd_workspace_size.argtypes = [I, I]
+        L.attn_bwd_workspace_size.restype = Z
+        L.attn_bwd_varlen.argtypes = [P, P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, F,
+                                      I, I, P, Z, P]
+        L.attn_bwd_varlen.restype = I
         _lib = L
     return _lib
 
@@ -290,3 +295,48 @@ def attn_decode_paged_append(q, k_new, v_new, k_cache, v_cache, block_table, seq
         _ptr(workspace), workspace.numel(), _stream(stream))
     _check(st, "attn_decode_paged_append")
     return out, lse, seqused_k_out
+
+
+def attn_bwd_varlen(q, k, v, o, dout, lse, *, cu_seqlens_q, cu_seqlens_k, max_seqlen_q,
+                    max_seqlen_k, mask=MASK_NONE, scale=None, window_left=-1, dq=None, dk=None,
+                    dv=None, workspace=None, stream=None):
+    """Gradients of the varlen forward: (dq [total_q, Hq, D], dk, dv [total_k, Hkv, D]).
+
+    q, o, dout [total_q, Hq, D] bf16; k, v [total_k, Hkv, D] bf16; lse [Hq, total_q]
+    fp32 from the forward.
+    """
+    total_q, Hq, D = q.shape
+    total_k, Hkv = k.shape[0], k.shape[1]
+    B = cu_seqlens_q.numel() - 1
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    ws_bytes = int(lib().attn_bwd_workspace_size(Hq, total_q))
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=q.device)
+    st = lib().attn_bwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq),
+                               _ptr(dk), _ptr(dv), _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), B,
+                               total_q, total_k, int(max_seqlen_q), int(max_seqlen_k), Hq, Hkv, D,
+                               _scale(scale), int(mask), int(window_left), _ptr(workspace),
+                               workspace.numel(), _stream(stream))
+    _check(st, "attn_bwd_varlen")
+    return dq, dk, dv
+
+
+def attn_bwd_dense(q, k, v, o, dout, lse, *, causal=False, scale=None, window_left=-1,
+                   stream=None):
+    """Dense [B, L, H, D] convenience over attn_bwd_varlen (lse [B, Hq, Lq] from
+    attn_fwd_dense).  Returns (dq, dk, dv) in the dense layouts."""
+    B, Lq, Hq, D = q.shape
+    Lk, Hkv = k.shape[1], k.shape[2]
+    dev = q.device
+    cq = torch.arange(B + 1, dtype=torch.int32, device=dev) * Lq
+    ck = torch.arange(B + 1, dtype=torch.int32, device=dev) * Lk
+    lse_v = lse.permute(1, 0, 2).reshape(Hq, B * Lq).contiguous()
+    dq, dk, dv = attn_bwd_varlen(q.reshape(B * Lq, Hq, D), k.reshape(B * Lk, Hkv, D),
+                                 v.reshape(B * Lk, Hkv, D), o.reshape(B * Lq, Hq, D),
+                                 dout.reshape(B * Lq, Hq, D), lse_v, cu_seqlens_q=cq,
+                                 cu_seqlens_k=ck, max_seqlen_q=Lq, max_seqlen_k=Lk,
+                                 mask=MASK_CAUSAL if causal else MASK_NONE, scale=scale,
+                                 window_left=window_left, stream=stream)
+    return dq.reshape(B, Lq, Hq, D), dk.reshape(B, Lk, Hkv, D), dv.reshape(B, Lk, Hkv, D)

@@ -22,6 +22,7 @@
 #include "decode.cuh"
 #include "prefill.cuh"
 #include "append.cuh"
+#include "backward.cuh"
 
 using namespace attn;
 
@@ -393,6 +394,43 @@ attn_status_t launch_decode_pages(const CUtensorMap& mk, const CUtensorMap& mv, 
                            (const float*)a.lse_part, (const int*)a.meta, a.B, a.Hq, o, lse) != cudaSuccess) {
         cudaGetLastError();
         return ATTN_ERR_CUDA;
+    }
+    return ATTN_OK;
+}
+
+// Backward: Delta, then the dK/dV and the dQ kernels, on one stream.
+template <int D>
+attn_status_t launch_backward(const CUtensorMap& mq, const CUtensorMap& mdo, const CUtensorMap& mk,
+                              const CUtensorMap& mv, const BwdArgs& a, const void* o,
+                              const void* dout, float* delta, int sms, cudaStream_t st) {
+    using Cfg = BwdCfg<D>;
+    static std::atomic<uint64_t> attr_mask{0};   // one bit per device
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const uint64_t bit = 1ull << (dev & 63);
+    if (!(attr_mask.load() & bit)) {
+        attn_status_t s = set_smem(bwd_dkdv_kernel<D>, Cfg::SMEM_A);
+        if (s == ATTN_OK) s = set_smem(bwd_dq_kernel<D>, Cfg::SMEM_B);
+        if (s != ATTN_OK) return s;
+        attr_mask.fetch_or(bit);
+    }
+    const long long rows = (long long)a.total_q * a.Hq;
+    const int dgrid = (int)std::max<long long>(1, std::min<long long>((rows + 7) / 8, (long long)sms * 32));
+    bwd_delta_kernel<D><<<dgrid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(o),
+                                                static_cast<const __nv_bfloat16*>(dout), delta,
+                                                a.total_q, a.Hq);
+    attn_status_t s = launch_status();
+    if (s != ATTN_OK) return s;
+    const long long g1 = (long long)a.nkt * a.B * a.Hkv;
+    const long long g2 = (long long)a.nqt * a.B * a.Hq;
+    if (g1 >= (1LL << 31) || g2 >= (1LL << 31)) return ATTN_ERR_UNSUPPORTED;
+    if (g1 > 0) {
+        bwd_dkdv_kernel<D><<<(unsigned)g1, kBwdThreads, Cfg::SMEM_A, st>>>(mq, mdo, mk, mv, a);
+        if ((s = launch_status()) != ATTN_OK) return s;
+    }
+    if (g2 > 0) {
+        bwd_dq_kernel<D><<<(unsigned)g2, kBwdThreads, Cfg::SMEM_B, st>>>(mq, mdo, mk, mv, a);
+        if ((s = launch_status()) != ATTN_OK) return s;
     }
     return ATTN_OK;
 }
@@ -936,6 +974,79 @@ attn_status_t attn_decode_paged_append(const void* q, const void* k_new, const v
                              block_size, seqused_k_out, B, Hq, Hkv, D, softmax_scale, window_left,
                              softcap, num_splits, dtype, nullptr, nullptr, nullptr, o, lse,
                              workspace, workspace_bytes, stream, true);
+}
+
+size_t attn_bwd_workspace_size(int num_heads_q, int total_q) {
+    if (num_heads_q <= 0 || total_q < 0) return 0;
+    return (size_t)num_heads_q * (size_t)total_q * sizeof(float) + 16;
+}
+
+attn_status_t attn_bwd_varlen(const void* q, const void* k, const void* v, const void* o,
+                              const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                              const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int B,
+                              int total_q, int total_k, int max_seqlen_q, int max_seqlen_k, int Hq,
+                              int Hkv, int D, float softmax_scale, int mask, int window_left,
+                              void* workspace, size_t workspace_bytes, attn_stream_t stream) {
+    if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv || !cu_seqlens_q || !cu_seqlens_k)
+        return ATTN_ERR_INVALID_ARG;
+    if (B < 0 || total_q < 0 || total_k < 0 || max_seqlen_q < 0 || max_seqlen_k < 0 || Hq <= 0 ||
+        Hkv <= 0 || Hq % Hkv != 0)
+        return ATTN_ERR_INVALID_ARG;
+    if (mask != ATTN_MASK_NONE && mask != ATTN_MASK_CAUSAL)
+        return mask == ATTN_MASK_PATCH ? ATTN_ERR_UNSUPPORTED : ATTN_ERR_INVALID_ARG;
+    if (window_left >= 0 && mask != ATTN_MASK_CAUSAL) return ATTN_ERR_UNSUPPORTED;
+    if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
+        !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+        return ATTN_ERR_INVALID_ARG;
+    const size_t need = attn_bwd_workspace_size(Hq, total_q);
+    if (!workspace || !aligned16(workspace)) return ATTN_ERR_INVALID_ARG;
+    if (workspace_bytes < need) return ATTN_ERR_WORKSPACE_TOO_SMALL;
+    if ((long long)total_q * Hq >= (1LL << 31) || (long long)total_k >= (1LL << 31))
+        return ATTN_ERR_UNSUPPORTED;
+    int dev = 0;
+    const attn_status_t dvs = current_device_ok(&dev);
+    if (dvs != ATTN_OK) return dvs;
+    if (B == 0 || total_q == 0) return ATTN_OK;
+
+    CUtensorMap mq, mdo, mk, mv;
+    const uint64_t rowq = (uint64_t)Hq * D * 2;
+    const uint64_t dq4[4] = {(uint64_t)D, (uint64_t)Hq, (uint64_t)total_q, 1};
+    const uint64_t sq3[3] = {(uint64_t)D * 2, rowq, rowq * (uint64_t)total_q};
+    const uint64_t rowk = (uint64_t)Hkv * D * 2;
+    const uint64_t nk = (uint64_t)std::max(total_k, 1);
+    const uint64_t dk4[4] = {(uint64_t)D, (uint64_t)Hkv, nk, 1};
+    const uint64_t sk3[3] = {(uint64_t)D * 2, rowk, rowk * nk};
+    const uint32_t box[4] = {64, 1, 128, 1};
+    attn_status_t s;
+    if ((s = get_map(&mq, q, ATTN_BF16, dq4, sq3, box)) != ATTN_OK) return s;
+    if ((s = get_map(&mdo, dout, ATTN_BF16, dq4, sq3, box)) != ATTN_OK) return s;
+    if ((s = get_map(&mk, k, ATTN_BF16, dk4, sk3, box)) != ATTN_OK) return s;
+    if ((s = get_map(&mv, v, ATTN_BF16, dk4, sk3, box)) != ATTN_OK) return s;
+
+    BwdArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.B = B;
+    a.Hq = Hq;
+    a.Hkv = Hkv;
+    a.group = Hq / Hkv;
+    a.mask = mask;
+    a.window = window_left < 0 ? -1 : window_left;
+    a.cu_q = cu_seqlens_q;
+    a.cu_k = cu_seqlens_k;
+    a.lse = lse;
+    a.delta = static_cast<float*>(workspace);
+    a.scale = resolve_scale(softmax_scale, D);
+    a.dq = static_cast<__nv_bfloat16*>(dq);
+    a.dk = static_cast<__nv_bfloat16*>(dk);
+    a.dv = static_cast<__nv_bfloat16*>(dv);
+    a.total_q = total_q;
+    a.nqt = (max_seqlen_q + 127) / 128;
+    a.nkt = (max_seqlen_k + 127) / 128;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    float* delta = static_cast<float*>(workspace);
+    if (D == 128) return launch_backward<128>(mq, mdo, mk, mv, a, o, dout, delta, sm_count(dev), st);
+    return launch_backward<64>(mq, mdo, mk, mv, a, o, dout, delta, sm_count(dev), st);
 }
 
 attn_status_t attn_decode_paged_noalloc(const void* q, const void* k_cache, const void* v_cache,

@@ -18,6 +18,8 @@ Carried in the same line:
   "kv_append":   paged KV append of every token of the varlen prefill
                  workload (GB/s of new K/V read + cache rows written), and
                  one decode step with its one-token append (GB/s as decode).
+  "backward":    dQ, dK, dV of the varlen causal GQA workload (packed K/V,
+                 same lengths) -> TFLOP/s at 10*D per allowed pair per head.
 
 Timing: W warm-up steps, then K steps each bracketed by CUDA events on the
 launching stream, a 256 MiB L2 flush between steps outside the events, and a
@@ -82,7 +84,8 @@ def parse_args():
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-prefill", action="store_true")
-    p.add_argument("--workload", choices=["all", "decode", "prefill", "fp8", "window", "append"],
+    p.add_argument("--workload", choices=["all", "decode", "prefill", "fp8", "window", "append",
+                                          "backward"],
                    default="all",
                    help="run only one workload (profiling runs); the JSON line then carries "
                         "only what ran")
@@ -367,6 +370,8 @@ def run_ours(args, rank, world, local):
         run_window(args, A, W, dev, world, flush, peaks, peak_kind, line)
     if args.workload in ("all", "append"):
         run_append(args, A, W, dev, world, flush, peaks, peak_kind, line)
+    if args.workload in ("all", "backward") and not args.no_prefill:
+        run_backward(args, A, W, dev, world, flush, peaks, peak_kind, line)
     if args.workload in ("all", "decode") and rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
     if rank == 0:
@@ -654,6 +659,46 @@ def run_append(args, A, W, dev, world, flush, peaks, peak_kind, line):
                          "unit": "GB/s", "frac": round(dgbs / peaks["hbm_gbs"], 4),
                          "traffic": None, "peak_kind": peak_kind}},
     }
+
+
+def run_backward(args, A, W, dev, world, flush, peaks, peak_kind, line):
+    """dQ, dK, dV of the varlen causal GQA workload (packed K/V)."""
+    wp = W.varlen_paged_prefill(seed=args.seed)
+    Pp = wp.params
+    lens = wp.tensors["seqused_k"]
+    cu = W.cu_from_lens(lens).to(dev)
+    total, Hq, Hkv, D = Pp["total_q"], Pp["Hq"], Pp["Hkv"], Pp["D"]
+    q = W.randn_bf16((total, Hq, D), args.seed, 51).to(dev)
+    k = W.randn_bf16((total, Hkv, D), args.seed, 52).to(dev)
+    v = W.randn_bf16((total, Hkv, D), args.seed, 53).to(dev)
+    do = W.randn_bf16((total, Hq, D), args.seed, 54).to(dev)
+    maxlen = int(lens.max())
+    o, lse = A.attn_fwd_varlen_paged(q, k, v, cu_seqlens_q=cu, cu_seqlens_k=cu,
+                                     max_seqlen_q=maxlen, mask=A.MASK_CAUSAL, scale=Pp["scale"])
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(A.lib().attn_bwd_workspace_size(Hq, total), dtype=torch.uint8, device=dev)
+
+    def bwd_step():
+        A.attn_bwd_varlen(q, k, v, o, do, lse, cu_seqlens_q=cu, cu_seqlens_k=cu,
+                          max_seqlen_q=maxlen, max_seqlen_k=maxlen, mask=A.MASK_CAUSAL,
+                          scale=Pp["scale"], dq=dq, dk=dk, dv=dv, workspace=ws)
+
+    bms = statistics.mean(time_steps(bwd_step, args.steps, args.warmup, world, flush))
+    flops = 2.5 * causal_flops(lens.numpy(), Hq, D)
+    tf = flops / (bms * 1e-3) / 1e12
+    line["backward"] = {
+        "workload": "varlen causal GQA backward: 16 seqs, L ~ U[64,4096] (seed %d: %d tokens), "
+                    "Hq=32, Hkv=8, D=128, packed K/V, bf16" % (args.seed, total),
+        "value": round(tf, 2), "unit": "TFLOP/s", "ms_per_step": round(bms, 5),
+        "flops_per_step": flops,
+        "flops_convention": "10*D per allowed (q,k) pair per query head (five GEMMs; the "
+                            "kernels run seven, recomputing S and dP for dQ)",
+        "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": peaks["bf16_tflops"],
+                     "unit": "TFLOP/s", "frac": round(tf / peaks["bf16_tflops"], 4),
+                     "traffic": None, "kernel": "bwd_dkdv_kernel<128> + bwd_dq_kernel<128> "
+                                                "(+ bwd_delta_kernel)", "peak_kind": peak_kind},
+    }
+    del q, k, v, do, o, dq, dk, dv
 
 
 def cpu_baseline(w):

@@ -244,6 +244,40 @@ attn_status_t attn_decode_paged_append(
     void *o, float *lse, void *workspace, size_t workspace_bytes, attn_stream_t stream);
 
 /*
+ * Bytes of workspace attn_bwd_varlen needs (fp32 Delta per query row and head).
+ * Returns 0 for invalid sizes.
+ */
+size_t attn_bwd_workspace_size(int num_heads_q, int total_q);
+
+/*
+ * Attention backward: the gradients dQ, dK, dV of the varlen forward, for the
+ * training path of the pages (BLT trains through the FlexAttention autograd;
+ * "Rope dim" lists the FlashAttnVarlenFunc backward).  With
+ * P = exp(scale Q K^T - LSE) under the mask and Delta_i = dO_i . O_i:
+ *   dV = P^T dO,  dS = P (dO V^T - Delta) scale,  dQ = dS K,  dK = dS^T Q,
+ * dK and dV summed over each KV head's query heads.
+ *   q, o, dout, dq [total_q, Hq, D] bf16, contiguous (o and lse from the
+ *                  forward on the same inputs, lse [Hq, total_q] fp32).
+ *   k, v, dk, dv   [total_k, Hkv, D] bf16, contiguous (packed; no paging).
+ *   cu_seqlens_q, cu_seqlens_k int32 [B+1]; max_seqlen_q / max_seqlen_k bound
+ *                  the per-sequence lengths (they size the grids).
+ *   mask           ATTN_MASK_NONE or ATTN_MASK_CAUSAL (bottom-right aligned),
+ *                  window_left as in the forward (causal only); no softcap
+ *                  and no patch mask (ATTN_ERR_UNSUPPORTED).
+ *   workspace      >= attn_bwd_workspace_size(Hq, total_q) bytes, 16-byte
+ *                  aligned (receives Delta).
+ * Every output row is written (rows whose query saw no key get dQ = 0; keys
+ * no query saw get dK = dV = 0).  Supported: head_dim in {64, 128}.
+ */
+attn_status_t attn_bwd_varlen(
+    const void *q, const void *k, const void *v, const void *o, const void *dout,
+    const float *lse, void *dq, void *dk, void *dv,
+    const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
+    int B, int total_q, int total_k, int max_seqlen_q, int max_seqlen_k,
+    int num_heads_q, int num_heads_kv, int head_dim, float softmax_scale,
+    int mask, int window_left, void *workspace, size_t workspace_bytes, attn_stream_t stream);
+
+/*
  * attn_decode_paged without any device allocation by the caller: the same
  * paged decode (automatic split choice), with its scratch taken from a fixed
  * 8 MiB array that this library keeps in device memory.  No counterpart on
