@@ -309,9 +309,6 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                     if (slot * kPageRows < Lk && slot < a.max_blocks)
                         page = a.block_table[(long long)b * a.max_blocks + slot];
                 }
-                int pages[PPT];
-#pragma unroll
-                for (int p = 0; p < PPT; ++p) pages[p] = __shfl_sync(0xffffffffu, page, p);
                 int npv = 0;
 #pragma unroll
                 for (int p = 0; p < PPT; ++p) npv += (j * kBN + p * kPageRows < Lk) ? 1 : 0;
@@ -320,48 +317,46 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                 bool ok = mbar_wait(&k_empty[st], ph ^ 1, kErrProdKEmpty);
                 ok = __all_sync(0xffffffffu, ok);
                 if (!ok) break;
-                if (lane == 0) {
-                    mbar_arrive_expect_tx(&k_full[st], bytes);
-                    uint8_t* dst = sK + st * C::KVB;
-                    if (a.paged) {
-#pragma unroll
-                        for (int p = 0; p < PPT; ++p) {
-                            if (j * kBN + p * kPageRows >= Lk) continue;
-#pragma unroll
-                            for (int c = 0; c < C::NCHUNK; ++c)
-                                tma_load_4d_hint(&tmK, &k_full[st],
-                                                 dst + c * kBN * 128 + p * kPageRows * 128,
-                                                 c * C::CHUNK_E, g, pages[p] * kPageRows, 0, pol);
-                        }
-                    } else {
+                if (a.paged) {
+                    // the tile's byte count first, then each page lane issues its own page's boxes
+                    if (lane == 0) mbar_arrive_expect_tx(&k_full[st], bytes);
+                    __syncwarp();
+                    if (lane < PPT && j * kBN + lane * kPageRows < Lk) {
+                        uint8_t* dst = sK + st * C::KVB + lane * kPageRows * 128;
 #pragma unroll
                         for (int c = 0; c < C::NCHUNK; ++c)
-                            tma_load_4d_hint(&tmK, &k_full[st], dst + c * kBN * 128,
-                                             c * C::CHUNK_E, g, k_off + j * kBN, bcoord, pol);
+                            tma_load_4d_hint(&tmK, &k_full[st], dst + c * kBN * 128, c * C::CHUNK_E, g,
+                                             page * kPageRows, 0, pol);
                     }
+                } else if (lane == 0) {
+                    mbar_arrive_expect_tx(&k_full[st], bytes);
+                    uint8_t* dst = sK + st * C::KVB;
+#pragma unroll
+                    for (int c = 0; c < C::NCHUNK; ++c)
+                        tma_load_4d_hint(&tmK, &k_full[st], dst + c * kBN * 128,
+                                         c * C::CHUNK_E, g, k_off + j * kBN, bcoord, pol);
                 }
                 ok = mbar_wait(&v_empty[st], ph ^ 1, kErrProdVEmpty);
                 ok = __all_sync(0xffffffffu, ok);
                 if (!ok) { ++issued; break; }
-                if (lane == 0) {
-                    mbar_arrive_expect_tx(&v_full[st], bytes);
-                    uint8_t* dst = sV + st * C::KVB;
-                    if (a.paged) {
-#pragma unroll
-                        for (int p = 0; p < PPT; ++p) {
-                            if (j * kBN + p * kPageRows >= Lk) continue;
-#pragma unroll
-                            for (int c = 0; c < C::NCHUNK; ++c)
-                                tma_load_4d_hint(&tmV, &v_full[st],
-                                                 dst + c * kBN * 128 + p * kPageRows * 128,
-                                                 c * C::CHUNK_E, g, pages[p] * kPageRows, 0, pol);
-                        }
-                    } else {
+                if (a.paged) {
+                    // the tile's byte count first, then each page lane issues its own page's boxes
+                    if (lane == 0) mbar_arrive_expect_tx(&v_full[st], bytes);
+                    __syncwarp();
+                    if (lane < PPT && j * kBN + lane * kPageRows < Lk) {
+                        uint8_t* dst = sV + st * C::KVB + lane * kPageRows * 128;
 #pragma unroll
                         for (int c = 0; c < C::NCHUNK; ++c)
-                            tma_load_4d_hint(&tmV, &v_full[st], dst + c * kBN * 128,
-                                             c * C::CHUNK_E, g, k_off + j * kBN, bcoord, pol);
+                            tma_load_4d_hint(&tmV, &v_full[st], dst + c * kBN * 128, c * C::CHUNK_E, g,
+                                             page * kPageRows, 0, pol);
                     }
+                } else if (lane == 0) {
+                    mbar_arrive_expect_tx(&v_full[st], bytes);
+                    uint8_t* dst = sV + st * C::KVB;
+#pragma unroll
+                    for (int c = 0; c < C::NCHUNK; ++c)
+                        tma_load_4d_hint(&tmV, &v_full[st], dst + c * kBN * 128,
+                                         c * C::CHUNK_E, g, k_off + j * kBN, bcoord, pol);
                 }
             }
             // Let every copy this warp started land before the CTA can exit.
