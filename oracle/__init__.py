@@ -59,6 +59,8 @@ def bind(lib):
                                     D, I, P, I, D, P, P, I, I]
     lib.attn_oracle_combine.restype = None
     lib.attn_oracle_combine.argtypes = [P, P, I, I, I, P, P]
+    lib.attn_oracle_fwd_qv.restype = I
+    lib.attn_oracle_fwd_qv.argtypes = [P, P, P, P, P, P, I, I, I, I, D, I, I, P, P, I, I]
     lib.attn_oracle_bwd.restype = I
     lib.attn_oracle_bwd.argtypes = [P, P, P, P, P, P, I, I, I, I, D, I, I, P, P, P, I]
     return lib
@@ -217,3 +219,26 @@ def attn_bwd_dense(q, k, v, do, *, scale, causal, window_left=-1, nthreads=None)
                                  mask=MASK_CAUSAL if causal else MASK_NONE,
                                  window_left=window_left, nthreads=nthreads)
     return dq.reshape(B, Lq, Hq, D), dk.reshape(B, Lk, Hkv, D), dv.reshape(B, Lk, Hkv, D)
+
+
+def attn_varlen_qv(q, qv, k, v, *, cu_seqlens_q, cu_seqlens_k, num_heads_kv, scale,
+                   mask=MASK_NONE, only_qv=False, nthreads=None):
+    """Forward with the extra Qv score term: s = scale * (q.k + qv.v) (only_qv: scale * qv.v).
+
+    q, qv [total_q, Hq, D] (q ignored with only_qv); k, v [total_k, Hkv, D].
+    Returns (O [total_q, Hq, D], LSE [Hq, total_q]).
+    """
+    lib = _load()
+    qva, ka, va = _f64(qv), _f64(k), _f64(v)
+    qa = None if only_qv else _f64(q)
+    total_q, Hq, D = qva.shape
+    cq, ck = _i32(cu_seqlens_q), _i32(cu_seqlens_k)
+    B = len(cq) - 1
+    o = np.zeros((total_q, Hq, D), np.float64)
+    lse = np.zeros((Hq, total_q), np.float64)
+    rc = lib.attn_oracle_fwd_qv(_ptr(qa), _ptr(qva), _ptr(ka), _ptr(va), _ptr(cq), _ptr(ck), B, Hq,
+                                int(num_heads_kv), D, float(scale), int(mask), int(bool(only_qv)),
+                                _ptr(o), _ptr(lse), total_q, int(nthreads or os.cpu_count() or 1))
+    if rc != 0:
+        raise ValueError("oracle rejected its arguments (rc=%d)" % rc)
+    return o, lse

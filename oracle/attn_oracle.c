@@ -46,7 +46,11 @@
  *     attention", Testing) are read as: a causal row keeps only the keys
  *     i' - W <= j <= i' (i' = i + Lk - Lq, W >= 0; W < 0 means no window),
  *     and a softcap c > 0 maps each scaled score s to c * tanh(s / c)
- *     (c = 0 means none).
+ *     (c = 0 means none);
+ *   - the Qv term of "Rope dim" (overview: Qv GEMM, only_qv) is read as an
+ *     extra dot product of a query-side vector qv with the value row,
+ *     s_ij = scale * (q.k_j + qv.v_j), with only_qv dropping q.k_j; qv has the
+ *     value head dimension, equal to the key one here (attn_oracle_fwd_qv).
  */
 #include <math.h>
 #include <stdint.h>
@@ -160,6 +164,77 @@ int attn_oracle_fwd(const double *q, const double *k, const double *v,
             *lse_i = M + log(Z);
         }
         free(s);
+    }
+    return bad ? -2 : 0;
+}
+
+/*
+ * Forward with the extra "Qv" score term of "Rope dim" (vllm-project
+ * flash-attention PR 172, overview: the Qv GEMM, and an only_qv mode that
+ * skips the Q/K loads and the QK GEMM and zero-initialises the score with the
+ * Qv GEMM).  Reading: for query i and key j (packed varlen, no paging, the
+ * masks above), with qv [total_q][Hq][D] paired with the value rows,
+ *   s_ij = scale * (q_i . k_j + qv_i . v_j)        (only_qv: the first term is dropped)
+ * then the same softmax, O and LSE as attn_oracle_fwd.  Written out plainly
+ * (explicit score row, max-subtracted softmax).
+ */
+int attn_oracle_fwd_qv(const double *q, const double *qv, const double *k, const double *v,
+                       const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k, int B, int Hq,
+                       int Hkv, int D, double scale, int mask, int only_qv, double *o,
+                       double *lse, int total_q, int nthreads) {
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || Hq % Hkv != 0) return -1;
+    if (!qv || !cu_seqlens_q || !cu_seqlens_k || (!only_qv && !q)) return -1;
+    if (mask != ORACLE_MASK_NONE && mask != ORACLE_MASK_CAUSAL) return -1;
+    const int group = Hq / Hkv;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+    (void)nthreads;
+#endif
+    int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(|| : bad)
+    for (long long task = 0; task < (long long)B * Hq; ++task) {
+        const int b = (int)(task / Hq), h = (int)(task % Hq);
+        const int g = h / group;
+        const int q0 = cu_seqlens_q[b], k0 = cu_seqlens_k[b];
+        const int Lq = cu_seqlens_q[b + 1] - q0, Lk = cu_seqlens_k[b + 1] - k0;
+        double *srow = (double *)malloc(sizeof(double) * (size_t)(Lk > 0 ? Lk : 1));
+        if (!srow) { bad = 1; continue; }
+        for (int i = 0; i < Lq; ++i) {
+            const double *qi = only_qv ? NULL : q + ((long long)(q0 + i) * Hq + h) * D;
+            const double *qvi = qv + ((long long)(q0 + i) * Hq + h) * D;
+            double *oi = o + ((long long)(q0 + i) * Hq + h) * D;
+            double *lse_i = lse + (long long)h * total_q + (q0 + i);
+            for (int j = 0; j < Lk; ++j) {
+                const double *kj = k + ((long long)(k0 + j) * Hkv + g) * D;
+                const double *vj = v + ((long long)(k0 + j) * Hkv + g) * D;
+                double qk = 0.0, qvv = 0.0;
+                if (!only_qv)
+                    for (int d = 0; d < D; ++d) qk += qi[d] * kj[d];
+                for (int d = 0; d < D; ++d) qvv += qvi[d] * vj[d];
+                srow[j] = scale * (qk + qvv);
+            }
+            double M = -INFINITY;
+            int any = 0;
+            for (int j = 0; j < Lk; ++j) {
+                if (!allowed(mask, i, j, Lq, Lk, NULL, -1)) continue;
+                if (!any || srow[j] > M) M = srow[j];
+                any = 1;
+            }
+            for (int d = 0; d < D; ++d) oi[d] = 0.0;
+            if (!any) { *lse_i = -INFINITY; continue; }
+            double Z = 0.0;
+            for (int j = 0; j < Lk; ++j) {
+                if (!allowed(mask, i, j, Lq, Lk, NULL, -1)) continue;
+                const double pj = exp(srow[j] - M);
+                const double *vj = v + ((long long)(k0 + j) * Hkv + g) * D;
+                Z += pj;
+                for (int d = 0; d < D; ++d) oi[d] += pj * vj[d];
+            }
+            for (int d = 0; d < D; ++d) oi[d] /= Z;
+            *lse_i = M + log(Z);
+        }
+        free(srow);
     }
     return bad ? -2 : 0;
 }
