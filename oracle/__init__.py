@@ -60,7 +60,8 @@ def bind(lib):
     lib.attn_oracle_combine.restype = None
     lib.attn_oracle_combine.argtypes = [P, P, I, I, I, P, P]
     lib.attn_oracle_fwd_qv.restype = I
-    lib.attn_oracle_fwd_qv.argtypes = [P, P, P, P, P, P, I, I, I, I, D, I, I, P, P, I, I]
+    lib.attn_oracle_fwd_qv.argtypes = [P, P, P, P, P, I, I, P, P, P, I, I, I, I, D, I, P, I, D, I,
+                                       P, P, I, I]
     lib.attn_oracle_bwd.restype = I
     lib.attn_oracle_bwd.argtypes = [P, P, P, P, P, P, I, I, I, I, D, I, I, P, P, P, I]
     return lib
@@ -221,24 +222,38 @@ def attn_bwd_dense(q, k, v, do, *, scale, causal, window_left=-1, nthreads=None)
     return dq.reshape(B, Lq, Hq, D), dk.reshape(B, Lk, Hkv, D), dv.reshape(B, Lk, Hkv, D)
 
 
-def attn_varlen_qv(q, qv, k, v, *, cu_seqlens_q, cu_seqlens_k, num_heads_kv, scale,
-                   mask=MASK_NONE, only_qv=False, nthreads=None):
+def attn_varlen_qv(q, qv, k, v, *, cu_seqlens_q, num_heads_kv, scale, cu_seqlens_k=None,
+                   block_table=None, seqused_k=None, mask=MASK_NONE, patch_kv_range=None,
+                   window_left=-1, softcap=0.0, only_qv=False, nthreads=None):
     """Forward with the extra Qv score term: s = scale * (q.k + qv.v) (only_qv: scale * qv.v).
 
-    q, qv [total_q, Hq, D] (q ignored with only_qv); k, v [total_k, Hkv, D].
+    q, qv [total_q, Hq, D] (q and k may be None with only_qv); k, v packed
+    [total_k, Hkv, D] addressed by cu_seqlens_k, or paged [num_blocks, bs, Hkv, D]
+    through block_table.  Masks, window and softcap as attn_varlen.
     Returns (O [total_q, Hq, D], LSE [Hq, total_q]).
     """
     lib = _load()
-    qva, ka, va = _f64(qv), _f64(k), _f64(v)
+    qva, va = _f64(qv), _f64(v)
     qa = None if only_qv else _f64(q)
+    ka = None if only_qv else _f64(k)
     total_q, Hq, D = qva.shape
-    cq, ck = _i32(cu_seqlens_q), _i32(cu_seqlens_k)
+    cq = _i32(cu_seqlens_q)
+    ck = None if cu_seqlens_k is None else _i32(cu_seqlens_k)
+    bt = None if block_table is None else _i32(block_table)
+    su = None if seqused_k is None else _i32(seqused_k)
+    pr = None if patch_kv_range is None else _i32(patch_kv_range)
     B = len(cq) - 1
+    mbps = 0 if bt is None else bt.shape[1]
+    bs = 0 if bt is None else va.shape[1]
     o = np.zeros((total_q, Hq, D), np.float64)
     lse = np.zeros((Hq, total_q), np.float64)
-    rc = lib.attn_oracle_fwd_qv(_ptr(qa), _ptr(qva), _ptr(ka), _ptr(va), _ptr(cq), _ptr(ck), B, Hq,
-                                int(num_heads_kv), D, float(scale), int(mask), int(bool(only_qv)),
-                                _ptr(o), _ptr(lse), total_q, int(nthreads or os.cpu_count() or 1))
+    if scale is None or scale <= 0:
+        scale = default_scale(D)
+    rc = lib.attn_oracle_fwd_qv(_ptr(qa), _ptr(qva), _ptr(ka), _ptr(va), _ptr(bt), mbps, bs, _ptr(cq),
+                                _ptr(ck), _ptr(su), B, Hq, int(num_heads_kv), D, float(scale),
+                                int(mask), _ptr(pr), int(window_left), float(softcap),
+                                int(bool(only_qv)), _ptr(o), _ptr(lse), total_q,
+                                int(nthreads or os.cpu_count() or 1))
     if rc != 0:
         raise ValueError("oracle rejected its arguments (rc=%d)" % rc)
     return o, lse

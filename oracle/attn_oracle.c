@@ -172,19 +172,26 @@ int attn_oracle_fwd(const double *q, const double *k, const double *v,
  * Forward with the extra "Qv" score term of "Rope dim" (vllm-project
  * flash-attention PR 172, overview: the Qv GEMM, and an only_qv mode that
  * skips the Q/K loads and the QK GEMM and zero-initialises the score with the
- * Qv GEMM).  Reading: for query i and key j (packed varlen, no paging, the
- * masks above), with qv [total_q][Hq][D] paired with the value rows,
+ * Qv GEMM).  Reading: for query i and key j, with qv [total_q][Hq][D] paired
+ * with the value rows,
  *   s_ij = scale * (q_i . k_j + qv_i . v_j)        (only_qv: the first term is dropped)
- * then the same softmax, O and LSE as attn_oracle_fwd.  Written out plainly
- * (explicit score row, max-subtracted softmax).
+ * then the softcap, masks, softmax, O and LSE exactly as attn_oracle_fwd, over
+ * the same packed or paged stores (k is not read with only_qv and may be NULL).
+ * Written out plainly (explicit score row, max-subtracted softmax).
  */
 int attn_oracle_fwd_qv(const double *q, const double *qv, const double *k, const double *v,
-                       const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k, int B, int Hq,
-                       int Hkv, int D, double scale, int mask, int only_qv, double *o,
-                       double *lse, int total_q, int nthreads) {
+                       const int32_t *block_table, int max_blocks_per_seq, int block_size,
+                       const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
+                       const int32_t *seqused_k, int B, int Hq, int Hkv, int D, double scale,
+                       int mask, const int32_t *patch_kv_range, int window_left, double softcap,
+                       int only_qv, double *o, double *lse, int total_q, int nthreads) {
     if (B < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || Hq % Hkv != 0) return -1;
-    if (!qv || !cu_seqlens_q || !cu_seqlens_k || (!only_qv && !q)) return -1;
-    if (mask != ORACLE_MASK_NONE && mask != ORACLE_MASK_CAUSAL) return -1;
+    if (!qv || !v || (!only_qv && (!q || !k))) return -1;
+    if (window_left >= 0 && mask != ORACLE_MASK_CAUSAL) return -1;
+    if (!(softcap >= 0.0)) return -1;
+    if (!seqused_k && !cu_seqlens_k) return -1;
+    if (!block_table && !cu_seqlens_k) return -1;
+    if (mask == ORACLE_MASK_PATCH && !patch_kv_range) return -1;
     const int group = Hq / Hkv;
 #ifdef _OPENMP
     if (nthreads > 0) omp_set_num_threads(nthreads);
@@ -196,28 +203,34 @@ int attn_oracle_fwd_qv(const double *q, const double *qv, const double *k, const
     for (long long task = 0; task < (long long)B * Hq; ++task) {
         const int b = (int)(task / Hq), h = (int)(task % Hq);
         const int g = h / group;
-        const int q0 = cu_seqlens_q[b], k0 = cu_seqlens_k[b];
-        const int Lq = cu_seqlens_q[b + 1] - q0, Lk = cu_seqlens_k[b + 1] - k0;
+        const int q0 = cu_seqlens_q[b];
+        const int Lq = cu_seqlens_q[b + 1] - q0;
+        const int Lk = seqused_k ? seqused_k[b] : cu_seqlens_k[b + 1] - cu_seqlens_k[b];
         double *srow = (double *)malloc(sizeof(double) * (size_t)(Lk > 0 ? Lk : 1));
         if (!srow) { bad = 1; continue; }
         for (int i = 0; i < Lq; ++i) {
             const double *qi = only_qv ? NULL : q + ((long long)(q0 + i) * Hq + h) * D;
             const double *qvi = qv + ((long long)(q0 + i) * Hq + h) * D;
+            const int32_t *range_i = patch_kv_range ? patch_kv_range + 2LL * (q0 + i) : NULL;
             double *oi = o + ((long long)(q0 + i) * Hq + h) * D;
             double *lse_i = lse + (long long)h * total_q + (q0 + i);
             for (int j = 0; j < Lk; ++j) {
-                const double *kj = k + ((long long)(k0 + j) * Hkv + g) * D;
-                const double *vj = v + ((long long)(k0 + j) * Hkv + g) * D;
+                const double *vj = kv_row(v, b, j, g, Hkv, D, block_table, max_blocks_per_seq,
+                                          block_size, cu_seqlens_k);
                 double qk = 0.0, qvv = 0.0;
-                if (!only_qv)
+                if (!only_qv) {
+                    const double *kj = kv_row(k, b, j, g, Hkv, D, block_table, max_blocks_per_seq,
+                                              block_size, cu_seqlens_k);
                     for (int d = 0; d < D; ++d) qk += qi[d] * kj[d];
+                }
                 for (int d = 0; d < D; ++d) qvv += qvi[d] * vj[d];
                 srow[j] = scale * (qk + qvv);
+                if (softcap > 0.0) srow[j] = softcap * tanh(srow[j] / softcap);
             }
             double M = -INFINITY;
             int any = 0;
             for (int j = 0; j < Lk; ++j) {
-                if (!allowed(mask, i, j, Lq, Lk, NULL, -1)) continue;
+                if (!allowed(mask, i, j, Lq, Lk, range_i, window_left)) continue;
                 if (!any || srow[j] > M) M = srow[j];
                 any = 1;
             }
@@ -225,9 +238,10 @@ int attn_oracle_fwd_qv(const double *q, const double *qv, const double *k, const
             if (!any) { *lse_i = -INFINITY; continue; }
             double Z = 0.0;
             for (int j = 0; j < Lk; ++j) {
-                if (!allowed(mask, i, j, Lq, Lk, NULL, -1)) continue;
+                if (!allowed(mask, i, j, Lq, Lk, range_i, window_left)) continue;
                 const double pj = exp(srow[j] - M);
-                const double *vj = v + ((long long)(k0 + j) * Hkv + g) * D;
+                const double *vj = kv_row(v, b, j, g, Hkv, D, block_table, max_blocks_per_seq,
+                                          block_size, cu_seqlens_k);
                 Z += pj;
                 for (int d = 0; d < D; ++d) oi[d] += pj * vj[d];
             }

@@ -78,6 +78,57 @@ def test_matches_sdpa_on_concatenated_head_dims(causal, only_qv):
     np.testing.assert_allclose(lse, lse_ref, atol=1e-12, rtol=0)
 
 
+def _to_pages(x, lens, bs, num_blocks, seed):
+    rng = np.random.default_rng(seed)
+    mbps = max(1, max((n + bs - 1) // bs for n in lens))
+    perm = rng.permutation(num_blocks)[:len(lens) * mbps].reshape(len(lens), mbps).astype(np.int32)
+    store = rng.standard_normal((num_blocks, bs) + x.shape[1:])
+    cu = _cu(lens)
+    for b, n in enumerate(lens):
+        for t in range(n):
+            store[perm[b, t // bs], t % bs] = x[cu[b] + t]
+    return store, perm
+
+
+@pytest.mark.parametrize("only_qv", [False, True])
+@pytest.mark.parametrize("mods", ["paged_window_softcap", "patch"])
+def test_concatenated_head_dims_through_the_plain_forward(only_qv, mods):
+    """[q|qv].[k|v]^T with values [v|0] through the (separately pinned) plain forward:
+    the first D columns of its O and its LSE are the Qv forward's, for every mask,
+    window, softcap and the paged store."""
+    lens_q, lens_k = [7, 3, 12], [19, 3, 12]
+    Hq, Hkv, D, scale, bs = 4, 2, 5, 0.45, 4
+    q, qv, k, v = _data(lens_q, lens_k, Hq, Hkv, D, seed=31 + only_qv)
+    cq, ck = _cu(lens_q), _cu(lens_k)
+    qq = qv if only_qv else np.concatenate([q, qv], -1)
+    kk = v if only_qv else np.concatenate([k, v], -1)
+    vv = v if only_qv else np.concatenate([v, np.zeros_like(v)], -1)
+    kw = dict(num_heads_kv=Hkv, scale=scale)
+    if mods == "patch":
+        rng = np.random.default_rng(5)
+        pr = np.zeros((sum(lens_q), 2), np.int32)
+        for b in range(3):
+            for i in range(lens_q[b]):
+                s0 = int(rng.integers(0, lens_k[b]))
+                pr[cq[b] + i] = (s0, int(rng.integers(s0, lens_k[b] + 1)))
+        kw.update(mask=2, patch_kv_range=pr)
+        got = oracle.attn_varlen_qv(q, qv, k, v, cu_seqlens_q=cq, cu_seqlens_k=ck, only_qv=only_qv, **kw)
+        ref = oracle.attn_varlen(qq, kk, vv, cu_seqlens_q=cq, cu_seqlens_k=ck, **kw)
+    else:
+        kw.update(mask=1, window_left=4, softcap=1.7)
+        su = np.array(lens_k, np.int32)
+        ks, bt = _to_pages(k, lens_k, bs, 24, 1)
+        vs, _ = _to_pages(v, lens_k, bs, 24, 1)
+        kks, _ = _to_pages(kk, lens_k, bs, 24, 1)
+        vvs, _ = _to_pages(vv, lens_k, bs, 24, 1)
+        got = oracle.attn_varlen_qv(q, qv, ks, vs, cu_seqlens_q=cq, block_table=bt, seqused_k=su,
+                                    only_qv=only_qv, **kw)
+        ref = oracle.attn_varlen(qq, kks, vvs, cu_seqlens_q=cq, block_table=bt, block_size=bs,
+                                 seqused_k=su, **kw)
+    np.testing.assert_allclose(got[0], ref[0][..., :D], atol=1e-13, rtol=0)
+    np.testing.assert_allclose(got[1], ref[1], atol=1e-13, rtol=0)
+
+
 @pytest.mark.parametrize("causal", [False, True])
 def test_zero_qv_is_the_plain_forward(causal):
     lens = [6, 3, 11]
@@ -96,7 +147,7 @@ def test_only_qv_is_the_plain_forward_with_keys_equal_to_values(causal):
     lens_q, lens_k = [4, 9], [10, 9]
     q, qv, k, v = _data(lens_q, lens_k, 6, 2, 4, seed=22)
     cq, ck = _cu(lens_q), _cu(lens_k)
-    o, lse = oracle.attn_varlen_qv(None, qv, k, v, cu_seqlens_q=cq, cu_seqlens_k=ck, num_heads_kv=2,
+    o, lse = oracle.attn_varlen_qv(None, qv, None, v, cu_seqlens_q=cq, cu_seqlens_k=ck, num_heads_kv=2,
                                    scale=0.8, mask=int(causal), only_qv=True)
     o_ref, lse_ref = oracle.attn_varlen(qv, v, v, cu_seqlens_q=cq, cu_seqlens_k=ck, num_heads_kv=2,
                                         scale=0.8, mask=int(causal))
@@ -114,19 +165,21 @@ def test_empty_rows_and_sequences():
 
 
 PINS = [lambda: [test_matches_sdpa_on_concatenated_head_dims(c, oq) for c in (False, True) for oq in (False, True)],
+        lambda: [test_concatenated_head_dims_through_the_plain_forward(oq, m) for oq in (False, True)
+                 for m in ("paged_window_softcap", "patch")],
         lambda: [test_zero_qv_is_the_plain_forward(c) for c in (False, True)],
         lambda: [test_only_qv_is_the_plain_forward_with_keys_equal_to_values(c) for c in (False, True)]]
 
+_VROW = ("const double *vj = kv_row(v, b, j, g, Hkv, D, block_table, max_blocks_per_seq,\n"
+         "                                          block_size, cu_seqlens_k);\n"
+         "                double qk = 0.0, qvv = 0.0;")
 MUTATIONS = {
     "qk_term_dropped": ("srow[j] = scale * (qk + qvv);", "srow[j] = scale * qvv;"),
     "qv_term_dropped": ("srow[j] = scale * (qk + qvv);", "srow[j] = scale * qk;"),
     "qv_term_unscaled": ("srow[j] = scale * (qk + qvv);", "srow[j] = scale * qk + qvv;"),
-    "qv_against_keys": ("for (int d = 0; d < D; ++d) qvv += qvi[d] * vj[d];",
-                        "for (int d = 0; d < D; ++d) qvv += qvi[d] * kj[d];"),
-    "q_in_place_of_qv": ("for (int d = 0; d < D; ++d) qvv += qvi[d] * vj[d];",
-                         "for (int d = 0; d < D; ++d) qvv += (only_qv ? qvi : qi)[d] * vj[d];"),
-    "only_qv_keeps_qk": ("                if (!only_qv)\n                    for (int d = 0; d < D; ++d) qk += qi[d] * kj[d];",
-                         "                for (int d = 0; d < D; ++d) qk += (only_qv ? qvi : qi)[d] * kj[d];"),
+    "query_in_place_of_qv": ("qvv += qvi[d] * vj[d];", "qvv += (only_qv ? qvi : qi)[d] * vj[d];"),
+    "qv_against_the_wrong_kv_head": (_VROW, _VROW.replace("kv_row(v, b, j, g,", "kv_row(v, b, j, h % Hkv,")),
+    "softcap_skipped": ("if (softcap > 0.0) srow[j] = softcap * tanh(srow[j] / softcap);", ""),
 }
 
 
