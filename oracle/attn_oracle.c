@@ -192,7 +192,6 @@ int attn_oracle_fwd_qv(const double *q, const double *qv, const double *k, const
     if (!seqused_k && !cu_seqlens_k) return -1;
     if (!block_table && !cu_seqlens_k) return -1;
     if (mask == ORACLE_MASK_PATCH && !patch_kv_range) return -1;
-    const int group = Hq / Hkv;
 #ifdef _OPENMP
     if (nthreads > 0) omp_set_num_threads(nthreads);
 #else
@@ -202,7 +201,7 @@ int attn_oracle_fwd_qv(const double *q, const double *qv, const double *k, const
 #pragma omp parallel for schedule(dynamic, 1) reduction(|| : bad)
     for (long long task = 0; task < (long long)B * Hq; ++task) {
         const int b = (int)(task / Hq), h = (int)(task % Hq);
-        const int g = h / group;
+        const int g = h / (Hq / Hkv);   /* the KV head query head h reads */
         const int q0 = cu_seqlens_q[b];
         const int Lq = cu_seqlens_q[b + 1] - q0;
         const int Lk = seqused_k ? seqused_k[b] : cu_seqlens_k[b + 1] - cu_seqlens_k[b];
@@ -215,7 +214,7 @@ int attn_oracle_fwd_qv(const double *q, const double *qv, const double *k, const
             double *oi = o + ((long long)(q0 + i) * Hq + h) * D;
             double *lse_i = lse + (long long)h * total_q + (q0 + i);
             for (int j = 0; j < Lk; ++j) {
-                const double *vj = kv_row(v, b, j, g, Hkv, D, block_table, max_blocks_per_seq,
+                const double *v_j = kv_row(v, b, j, g, Hkv, D, block_table, max_blocks_per_seq,
                                           block_size, cu_seqlens_k);
                 double qk = 0.0, qvv = 0.0;
                 if (!only_qv) {
@@ -223,7 +222,7 @@ int attn_oracle_fwd_qv(const double *q, const double *qv, const double *k, const
                                               block_size, cu_seqlens_k);
                     for (int d = 0; d < D; ++d) qk += qi[d] * kj[d];
                 }
-                for (int d = 0; d < D; ++d) qvv += qvi[d] * vj[d];
+                for (int d = 0; d < D; ++d) qvv += qvi[d] * v_j[d];
                 srow[j] = scale * (qk + qvv);
                 if (softcap > 0.0) srow[j] = softcap * tanh(srow[j] / softcap);
             }
@@ -240,13 +239,13 @@ int attn_oracle_fwd_qv(const double *q, const double *qv, const double *k, const
             for (int j = 0; j < Lk; ++j) {
                 if (!allowed(mask, i, j, Lq, Lk, range_i, window_left)) continue;
                 const double pj = exp(srow[j] - M);
-                const double *vj = kv_row(v, b, j, g, Hkv, D, block_table, max_blocks_per_seq,
+                const double *v_j = kv_row(v, b, j, g, Hkv, D, block_table, max_blocks_per_seq,
                                           block_size, cu_seqlens_k);
                 Z += pj;
-                for (int d = 0; d < D; ++d) oi[d] += pj * vj[d];
+                for (int d = 0; d < D; ++d) oi[d] += pj * v_j[d];
             }
-            for (int d = 0; d < D; ++d) oi[d] /= Z;
-            *lse_i = M + log(Z);
+            for (int d = 0; d < D; ++d) oi[d] = oi[d] / Z;
+            *lse_i = log(Z) + M;
         }
         free(srow);
     }

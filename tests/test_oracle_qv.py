@@ -170,14 +170,14 @@ PINS = [lambda: [test_matches_sdpa_on_concatenated_head_dims(c, oq) for c in (Fa
         lambda: [test_zero_qv_is_the_plain_forward(c) for c in (False, True)],
         lambda: [test_only_qv_is_the_plain_forward_with_keys_equal_to_values(c) for c in (False, True)]]
 
-_VROW = ("const double *vj = kv_row(v, b, j, g, Hkv, D, block_table, max_blocks_per_seq,\n"
+_VROW = ("const double *v_j = kv_row(v, b, j, g, Hkv, D, block_table, max_blocks_per_seq,\n"
          "                                          block_size, cu_seqlens_k);\n"
          "                double qk = 0.0, qvv = 0.0;")
 MUTATIONS = {
     "qk_term_dropped": ("srow[j] = scale * (qk + qvv);", "srow[j] = scale * qvv;"),
     "qv_term_dropped": ("srow[j] = scale * (qk + qvv);", "srow[j] = scale * qk;"),
     "qv_term_unscaled": ("srow[j] = scale * (qk + qvv);", "srow[j] = scale * qk + qvv;"),
-    "query_in_place_of_qv": ("qvv += qvi[d] * vj[d];", "qvv += (only_qv ? qvi : qi)[d] * vj[d];"),
+    "query_in_place_of_qv": ("qvv += qvi[d] * v_j[d];", "qvv += (only_qv ? qvi : qi)[d] * v_j[d];"),
     "qv_against_the_wrong_kv_head": (_VROW, _VROW.replace("kv_row(v, b, j, g,", "kv_row(v, b, j, h % Hkv,")),
     "softcap_skipped": ("if (softcap > 0.0) srow[j] = softcap * tanh(srow[j] / softcap);", ""),
 }
