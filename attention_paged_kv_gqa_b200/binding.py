@@ -55,6 +55,12 @@ def lib():
         L.attn_fwd_varlen_paged.argtypes = [P, P, P, P, I, I, I, P, P, P, I, I, I, I, I, I, I,
                                             F, I, P, I, F, I, P, P, P, P, P, P, Z, P]
         L.attn_fwd_varlen_paged.restype = I
+        L.attn_fwd_varlen_paged_only_qv.argtypes = [P, P, P, I, I, I, P, P, P, I, I, I, I, I, I, I,
+                                                    F, I, P, I, F, I, P, P, P, P, P]
+        L.attn_fwd_varlen_paged_only_qv.restype = I
+        L.attn_decode_paged_only_qv.argtypes = [P, P, P, I, I, I, P, I, I, I, I, F, I, F, I, I, P, P,
+                                                P, Z, P]
+        L.attn_decode_paged_only_qv.restype = I
         L.attn_decode_workspace_size.argtypes = [I, I, I, I, I, I, I]
         L.attn_decode_workspace_size.restype = Z
         L.attn_decode_paged.argtypes = [P, P, P, P, I, I, I, P, I, I, I, I, F, I, F, I, I, P, P,
@@ -189,6 +195,35 @@ def attn_fwd_varlen_paged(q, k_cache, v_cache, *, cu_seqlens_q, max_seqlen_q, bl
     return out, lse
 
 
+def attn_fwd_varlen_paged_only_qv(qv, v_cache, *, cu_seqlens_q, max_seqlen_q, block_table=None,
+                                  cu_seqlens_k=None, seqused_k=None, mask=MASK_NONE, scale=None,
+                                  patch_kv_range=None, window_left=-1, softcap=0.0,
+                                  descale_qv=None, descale_v=None, out=None, lse=None,
+                                  return_lse=True, stream=None):
+    """The only_qv score (scale * qv . v): qv [total_q, Hq, D]; v paged or packed as in
+    attn_fwd_varlen_paged.  Returns (o [total_q, Hq, D] bf16, lse [Hq, total_q] fp32)."""
+    total_q, Hq, D = qv.shape
+    B = cu_seqlens_q.numel() - 1
+    if block_table is not None:
+        num_blocks, block_size, Hkv = v_cache.shape[0], v_cache.shape[1], v_cache.shape[2]
+        mbps, total_k = block_table.shape[1], 0
+    else:
+        num_blocks, block_size, mbps = 0, 0, 0
+        total_k, Hkv = v_cache.shape[0], v_cache.shape[1]
+    if out is None:
+        out = torch.empty((total_q, Hq, D), dtype=torch.bfloat16, device=qv.device)
+    if lse is None and return_lse:
+        lse = torch.empty((Hq, total_q), dtype=torch.float32, device=qv.device)
+    st = lib().attn_fwd_varlen_paged_only_qv(
+        _ptr(qv), _ptr(v_cache), _ptr(block_table), mbps, num_blocks, block_size,
+        _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), _ptr(seqused_k), B, total_q, total_k,
+        int(max_seqlen_q), Hq, Hkv, D, _scale(scale), int(mask), _ptr(patch_kv_range),
+        int(window_left), float(softcap), _dtype_code(qv), _ptr(descale_qv), _ptr(descale_v),
+        _ptr(out), _ptr(lse), _stream(stream))
+    _check(st, "attn_fwd_varlen_paged_only_qv")
+    return out, lse
+
+
 def attn_decode_workspace_size(B, num_heads_q, num_heads_kv, head_dim, max_blocks_per_seq,
                                block_size=16, num_splits=0) -> int:
     return int(lib().attn_decode_workspace_size(B, num_heads_q, num_heads_kv, head_dim,
@@ -220,6 +255,29 @@ def attn_decode_paged(q, k_cache, v_cache, block_table, seqused_k, *, scale=None
                                  _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(),
                                  _stream(stream))
     _check(st, "attn_decode_paged")
+    return out, lse
+
+
+def attn_decode_paged_only_qv(qv, v_cache, block_table, seqused_k, *, scale=None, num_splits=0,
+                              window_left=-1, softcap=0.0, out=None, lse=None, workspace=None,
+                              return_lse=True, stream=None):
+    """Paged decode with the only_qv score: qv [B, Hq, D] -> (o [B, Hq, D] bf16, lse [B, Hq])."""
+    B, Hq, D = qv.shape
+    num_blocks, block_size, Hkv = v_cache.shape[0], v_cache.shape[1], v_cache.shape[2]
+    mbps = block_table.shape[1]
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=torch.bfloat16, device=qv.device)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=qv.device)
+    ws_bytes = attn_decode_workspace_size(B, Hq, Hkv, D, mbps, block_size, num_splits)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=qv.device)
+    st = lib().attn_decode_paged_only_qv(_ptr(qv), _ptr(v_cache), _ptr(block_table), mbps,
+                                         num_blocks, block_size, _ptr(seqused_k), B, Hq, Hkv, D,
+                                         _scale(scale), int(window_left), float(softcap),
+                                         int(num_splits), _dtype_code(qv), _ptr(out), _ptr(lse),
+                                         _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(st, "attn_decode_paged_only_qv")
     return out, lse
 
 

@@ -43,7 +43,7 @@ attn_status_t check_device_uncached(int device) {
     cudaGetDevice(&prev);
     if (prev != device) cudaSetDevice(device);
     cudaFuncAttributes fa;
-    const cudaError_t e = cudaFuncGetAttributes(&fa, prefill_kernel<128, false, false>);
+    const cudaError_t e = cudaFuncGetAttributes(&fa, prefill_kernel<128, false, false, false>);
     if (prev != device && prev >= 0) cudaSetDevice(prev);
     if (e != cudaSuccess) {
         cudaGetLastError();
@@ -221,7 +221,7 @@ attn_status_t launch_maybe_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, 
 }
 
 // ------------------------------------------------------------------ prefill dispatch
-template <int D, bool FP8, bool CAP>
+template <int D, bool FP8, bool CAP, bool OQ>
 attn_status_t launch_prefill_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                                const PrefillArgs& a, long long grid, cudaStream_t stream) {
     using Cfg = PrefillCfg<D, FP8>;
@@ -230,11 +230,11 @@ attn_status_t launch_prefill_t(const CUtensorMap& mq, const CUtensorMap& mk, con
     cudaGetDevice(&dev);
     const uint64_t bit = 1ull << (dev & 63);
     if (!(attr_mask.load() & bit)) {
-        const attn_status_t s = set_smem(prefill_kernel<D, FP8, CAP>, Cfg::SMEM_BYTES);
+        const attn_status_t s = set_smem(prefill_kernel<D, FP8, CAP, OQ>, Cfg::SMEM_BYTES);
         if (s != ATTN_OK) return s;
         attr_mask.fetch_or(bit);
     }
-    prefill_kernel<D, FP8, CAP><<<static_cast<unsigned>(grid), kPrefillThreads, Cfg::SMEM_BYTES, stream>>>(
+    prefill_kernel<D, FP8, CAP, OQ><<<static_cast<unsigned>(grid), kPrefillThreads, Cfg::SMEM_BYTES, stream>>>(
         mq, mk, mv, a);
     return launch_status();
 }
@@ -245,15 +245,27 @@ attn_status_t launch_prefill(int D, int dtype, const CUtensorMap& mq, const CUte
     if (grid <= 0) return ATTN_OK;
     if (grid >= (1LL << 31)) return ATTN_ERR_UNSUPPORTED;
     const bool cap = a.softcap > 0.0f;
+    if (a.only_qv) {
+        if (dtype == ATTN_BF16 && D == 128)
+            return cap ? launch_prefill_t<128, false, true, true>(mq, mk, mv, a, grid, stream)
+                       : launch_prefill_t<128, false, false, true>(mq, mk, mv, a, grid, stream);
+        if (dtype == ATTN_BF16 && D == 64)
+            return cap ? launch_prefill_t<64, false, true, true>(mq, mk, mv, a, grid, stream)
+                       : launch_prefill_t<64, false, false, true>(mq, mk, mv, a, grid, stream);
+        if (dtype == ATTN_FP8_E4M3 && D == 128)
+            return cap ? launch_prefill_t<128, true, true, true>(mq, mk, mv, a, grid, stream)
+                       : launch_prefill_t<128, true, false, true>(mq, mk, mv, a, grid, stream);
+        return ATTN_ERR_UNSUPPORTED;
+    }
     if (dtype == ATTN_BF16 && D == 128)
-        return cap ? launch_prefill_t<128, false, true>(mq, mk, mv, a, grid, stream)
-                   : launch_prefill_t<128, false, false>(mq, mk, mv, a, grid, stream);
+        return cap ? launch_prefill_t<128, false, true, false>(mq, mk, mv, a, grid, stream)
+                   : launch_prefill_t<128, false, false, false>(mq, mk, mv, a, grid, stream);
     if (dtype == ATTN_BF16 && D == 64)
-        return cap ? launch_prefill_t<64, false, true>(mq, mk, mv, a, grid, stream)
-                   : launch_prefill_t<64, false, false>(mq, mk, mv, a, grid, stream);
+        return cap ? launch_prefill_t<64, false, true, false>(mq, mk, mv, a, grid, stream)
+                   : launch_prefill_t<64, false, false, false>(mq, mk, mv, a, grid, stream);
     if (dtype == ATTN_FP8_E4M3 && D == 128)
-        return cap ? launch_prefill_t<128, true, true>(mq, mk, mv, a, grid, stream)
-                   : launch_prefill_t<128, true, false>(mq, mk, mv, a, grid, stream);
+        return cap ? launch_prefill_t<128, true, true, false>(mq, mk, mv, a, grid, stream)
+                   : launch_prefill_t<128, true, false, false>(mq, mk, mv, a, grid, stream);
     return ATTN_ERR_UNSUPPORTED;
 }
 
@@ -269,18 +281,19 @@ void unit_grid(PrefillArgs& a, int max_seqlen_q, long long* grid) {
 // when at least two 64-key stages fit in half of the SM's shared memory,
 // otherwise one CTA with as many stages as fit.
 template <int D>
-bool decode_geometry(int G, int B, int* ns_out, int* ctas_per_sm, int* smem_out) {
+bool decode_geometry(int G, int B, int* ns_out, int* ctas_per_sm, int* smem_out, bool vonly) {
     using Cfg = DecodeCfg<D>;
     const int half = (228 * 1024 - 2 * 1024) / 2;
     const int whole = 227 * 1024;
+    const int max_ns = vonly ? 32 : 16;     // V-only stages are half as large: twice as many
     for (int per_sm : {2, 1}) {
         const int cap = per_sm == 2 ? half : whole;
         int ns = 0;
-        while (ns < 16 && Cfg::smem_bytes(G, B, ns + 1) <= cap) ++ns;
+        while (ns < max_ns && Cfg::smem_bytes(G, B, ns + 1, vonly) <= cap) ++ns;
         if (ns >= 2) {
             *ns_out = ns;
             *ctas_per_sm = per_sm;
-            *smem_out = Cfg::smem_bytes(G, B, ns);
+            *smem_out = Cfg::smem_bytes(G, B, ns, vonly);
             return true;
         }
     }
@@ -301,7 +314,7 @@ attn_status_t launch_decode(const CUtensorMap& mk, const CUtensorMap& mv, Decode
         attr_mask.fetch_or(bit);
     }
     int ns = 0, per_sm = 0, smem = 0;
-    if (!decode_geometry<D>(a.group, a.B, &ns, &per_sm, &smem)) return ATTN_ERR_UNSUPPORTED;
+    if (!decode_geometry<D>(a.group, a.B, &ns, &per_sm, &smem, a.only_qv != 0)) return ATTN_ERR_UNSUPPORTED;
     a.nstages = ns;
     const int grid = (int)std::min<long long>((long long)sms * per_sm, std::max<long long>(items_max, 1));
     attn_status_t s = launch_maybe_pdl(decode_split_kernel<D>, dim3(grid), dim3(kDecThreads), smem, st,
@@ -376,7 +389,7 @@ attn_status_t launch_decode_pages(const CUtensorMap& mk, const CUtensorMap& mv, 
         if (s != ATTN_OK) return s;
         attr_mask.fetch_or(bit);
     }
-    const int smem = DecodePagesCfg<D>::smem_bytes(a.Hkv, a.B, a.nstages);
+    const int smem = DecodePagesCfg<D>::smem_bytes(a.Hkv, a.B, a.nstages, a.only_qv != 0);
     attn_status_t s = launch_maybe_pdl(decode_pages_kernel<D>, dim3(grid), dim3(32 * (a.Hkv + 1)),
                                        smem, st, pdl, mk, mv, a);
     if (s != ATTN_OK) return s;
@@ -581,16 +594,15 @@ attn_status_t attn_fwd_dense(const void* q, const void* k, const void* v, void* 
     return launch_prefill(D, dtype, mq, mk, mv, a, grid, static_cast<cudaStream_t>(stream));
 }
 
-attn_status_t attn_fwd_varlen_paged(
+// The varlen / paged forward; with `only_qv` the score is q . v (k_cache is the
+// value store, and the kernel reads the value tile as the score GEMM's operand).
+static attn_status_t fwd_varlen_paged_impl(
     const void* q, const void* k_cache, const void* v_cache, const int32_t* block_table,
     int max_blocks_per_seq, int num_blocks, int block_size, const int32_t* cu_seqlens_q,
     const int32_t* cu_seqlens_k, const int32_t* seqused_k, int B, int total_q, int total_k,
     int max_seqlen_q, int Hq, int Hkv, int D, float softmax_scale, int mask,
     const int32_t* patch_kv_range, int window_left, float softcap, int dtype, const float* dq,
-    const float* dk, const float* dv, void* o, float* lse, void* workspace,
-    size_t workspace_bytes, attn_stream_t stream) {
-    (void)workspace;
-    (void)workspace_bytes;
+    const float* dk, const float* dv, void* o, float* lse, attn_stream_t stream, int only_qv) {
     if (!q || !k_cache || !v_cache || !o || !cu_seqlens_q) return ATTN_ERR_INVALID_ARG;
     if (B < 0 || total_q < 0 || max_seqlen_q < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0)
         return ATTN_ERR_INVALID_ARG;
@@ -634,8 +646,9 @@ attn_status_t attn_fwd_varlen_paged(
     const uint32_t bkv[4] = {(uint32_t)chunk, 1, (uint32_t)(paged ? kPageRows : kBN), 1};
     attn_status_t s;
     if ((s = get_map(&mq, q, dtype, dq4, sq3, bq)) != ATTN_OK) return s;
-    if ((s = get_map(&mk, k_cache, dtype, dk4, sk3, bkv)) != ATTN_OK) return s;
     if ((s = get_map(&mv, v_cache, dtype, dk4, sk3, bkv)) != ATTN_OK) return s;
+    if (only_qv) mk = mv;   // no key store: its map is never used
+    else if ((s = get_map(&mk, k_cache, dtype, dk4, sk3, bkv)) != ATTN_OK) return s;
 
     PrefillArgs a;
     std::memset(&a, 0, sizeof(a));
@@ -648,6 +661,7 @@ attn_status_t attn_fwd_varlen_paged(
     a.softcap = softcap;
     a.varlen = 1;
     a.paged = paged ? 1 : 0;
+    a.only_qv = only_qv ? 1 : 0;
     a.cu_q = cu_seqlens_q;
     a.cu_k = cu_seqlens_k;
     a.seqused_k = seqused_k;
@@ -667,6 +681,38 @@ attn_status_t attn_fwd_varlen_paged(
     long long grid;
     unit_grid(a, max_seqlen_q, &grid);
     return launch_prefill(D, dtype, mq, mk, mv, a, grid, static_cast<cudaStream_t>(stream));
+}
+
+attn_status_t attn_fwd_varlen_paged(
+    const void* q, const void* k_cache, const void* v_cache, const int32_t* block_table,
+    int max_blocks_per_seq, int num_blocks, int block_size, const int32_t* cu_seqlens_q,
+    const int32_t* cu_seqlens_k, const int32_t* seqused_k, int B, int total_q, int total_k,
+    int max_seqlen_q, int Hq, int Hkv, int D, float softmax_scale, int mask,
+    const int32_t* patch_kv_range, int window_left, float softcap, int dtype, const float* dq,
+    const float* dk, const float* dv, void* o, float* lse, void* workspace,
+    size_t workspace_bytes, attn_stream_t stream) {
+    (void)workspace;
+    (void)workspace_bytes;
+    return fwd_varlen_paged_impl(q, k_cache, v_cache, block_table, max_blocks_per_seq, num_blocks,
+                                 block_size, cu_seqlens_q, cu_seqlens_k, seqused_k, B, total_q,
+                                 total_k, max_seqlen_q, Hq, Hkv, D, softmax_scale, mask,
+                                 patch_kv_range, window_left, softcap, dtype, dq, dk, dv, o, lse,
+                                 stream, 0);
+}
+
+attn_status_t attn_fwd_varlen_paged_only_qv(
+    const void* qv, const void* v_cache, const int32_t* block_table, int max_blocks_per_seq,
+    int num_blocks, int block_size, const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+    const int32_t* seqused_k, int B, int total_q, int total_k, int max_seqlen_q, int Hq, int Hkv,
+    int D, float softmax_scale, int mask, const int32_t* patch_kv_range, int window_left,
+    float softcap, int dtype, const float* descale_qv, const float* descale_v, void* o,
+    float* lse, attn_stream_t stream) {
+    // the value codes stand in the key slot, so the score's key descale is the value one
+    return fwd_varlen_paged_impl(qv, v_cache, v_cache, block_table, max_blocks_per_seq, num_blocks,
+                                 block_size, cu_seqlens_q, cu_seqlens_k, seqused_k, B, total_q,
+                                 total_k, max_seqlen_q, Hq, Hkv, D, softmax_scale, mask,
+                                 patch_kv_range, window_left, softcap, dtype, descale_qv, descale_v,
+                                 descale_v, o, lse, stream, 1);
 }
 
 // Split-KV heuristic: enough CTAs to fill every SM about twice with sequences
@@ -691,13 +737,14 @@ static void decode_splits(int B, int Hkv, int max_tokens, int requested, int* nu
     *num_splits = (max_tokens + t - 1) / t;
 }
 
-static int decode_pages_stages(int D, int Hkv, int B) {
+static int decode_pages_stages(int D, int Hkv, int B, bool vonly = false) {
     const int cap = 227 * 1024;
+    const int max_ns = vonly ? 16 : 8;      // V-only stages are half as large: twice as many
     int ns = 0;
     if (D == 128)
-        while (ns < 8 && DecodePagesCfg<128>::smem_bytes(Hkv, B, ns + 1) <= cap) ++ns;
+        while (ns < max_ns && DecodePagesCfg<128>::smem_bytes(Hkv, B, ns + 1, vonly) <= cap) ++ns;
     else
-        while (ns < 8 && DecodePagesCfg<64>::smem_bytes(Hkv, B, ns + 1) <= cap) ++ns;
+        while (ns < max_ns && DecodePagesCfg<64>::smem_bytes(Hkv, B, ns + 1, vonly) <= cap) ++ns;
     return ns;
 }
 
@@ -743,7 +790,7 @@ static attn_status_t decode_paged_impl(const void* q, const void* k_cache, const
                                        int window_left, float softcap, int num_splits, int dtype,
                                        const float* dq, const float* dk, const float* dv, void* o,
                                        float* lse, void* workspace, size_t workspace_bytes,
-                                       attn_stream_t stream, bool pdl) {
+                                       attn_stream_t stream, bool pdl, int only_qv = 0) {
     (void)dq;
     (void)dk;
     (void)dv;
@@ -789,8 +836,9 @@ static attn_status_t decode_paged_impl(const void* q, const void* k_cache, const
         const uint64_t ps[3] = {rowk, (uint64_t)D * 2, rowk * kPageRows};
         const uint32_t pbox[4] = {64, (uint32_t)kPageRows, (uint32_t)Hkv, 1};
         attn_status_t s;
-        if ((s = get_map(&pk, k_cache, ATTN_BF16, pd, ps, pbox)) != ATTN_OK) return s;
         if ((s = get_map(&pv, v_cache, ATTN_BF16, pd, ps, pbox)) != ATTN_OK) return s;
+        if (only_qv) pk = pv;   // no key store: its map is never used
+        else if ((s = get_map(&pk, k_cache, ATTN_BF16, pd, ps, pbox)) != ATTN_OK) return s;
         const int grid = sm_count(dev);
         const size_t slots = (size_t)grid + B;
         const size_t need_pg = slots * Hq * (D + 1) * sizeof(float) + (size_t)(B + 2) * sizeof(int);
@@ -812,7 +860,8 @@ static attn_status_t decode_paged_impl(const void* q, const void* k_cache, const
         pa.o_part = static_cast<float*>(workspace);
         pa.lse_part = pa.o_part + slots * Hq * D;
         pa.meta = reinterpret_cast<int*>(pa.lse_part + slots * Hq);
-        pa.nstages = decode_pages_stages(D, Hkv, B);
+        pa.nstages = decode_pages_stages(D, Hkv, B, only_qv != 0);
+        pa.only_qv = only_qv ? 1 : 0;
         if (D == 128)
             return launch_decode_pages<128>(pk, pv, pa, grid, stp, static_cast<__nv_bfloat16*>(o), lse, pdl);
         return launch_decode_pages<64>(pk, pv, pa, grid, stp, static_cast<__nv_bfloat16*>(o), lse, pdl);
@@ -824,8 +873,9 @@ static attn_status_t decode_paged_impl(const void* q, const void* k_cache, const
     const uint64_t sk3[3] = {(uint64_t)D * 2, rowk, rowk * nrows};
     const uint32_t bkv[4] = {64, 1, (uint32_t)kPageRows, 1};
     attn_status_t s;
-    if ((s = get_map(&mk, k_cache, ATTN_BF16, dk4, sk3, bkv)) != ATTN_OK) return s;
     if ((s = get_map(&mv, v_cache, ATTN_BF16, dk4, sk3, bkv)) != ATTN_OK) return s;
+    if (only_qv) mk = mv;
+    else if ((s = get_map(&mk, k_cache, ATTN_BF16, dk4, sk3, bkv)) != ATTN_OK) return s;
 
     DecodeArgs a;
     std::memset(&a, 0, sizeof(a));
@@ -845,6 +895,7 @@ static attn_status_t decode_paged_impl(const void* q, const void* k_cache, const
     a.o = static_cast<__nv_bfloat16*>(o);
     a.lse = lse;
     a.direct = ns == 1 ? 1 : 0;
+    a.only_qv = only_qv ? 1 : 0;
     if (ns > 1) {
         a.o_part = static_cast<float*>(workspace);
         a.lse_part = a.o_part + (size_t)ns * B * Hq * D;
@@ -872,6 +923,19 @@ attn_status_t attn_decode_paged(const void* q, const void* k_cache, const void* 
                              block_size, seqused_k, B, Hq, Hkv, D, softmax_scale, window_left,
                              softcap, num_splits, dtype, dq, dk, dv, o, lse, workspace,
                              workspace_bytes, stream, false);
+}
+
+attn_status_t attn_decode_paged_only_qv(const void* qv, const void* v_cache,
+                                        const int32_t* block_table, int max_blocks_per_seq,
+                                        int num_blocks, int block_size, const int32_t* seqused_k,
+                                        int B, int Hq, int Hkv, int D, float softmax_scale,
+                                        int window_left, float softcap, int num_splits, int dtype,
+                                        void* o, float* lse, void* workspace,
+                                        size_t workspace_bytes, attn_stream_t stream) {
+    return decode_paged_impl(qv, v_cache, v_cache, block_table, max_blocks_per_seq, num_blocks,
+                             block_size, seqused_k, B, Hq, Hkv, D, softmax_scale, window_left,
+                             softcap, num_splits, dtype, nullptr, nullptr, nullptr, o, lse,
+                             workspace, workspace_bytes, stream, false, 1);
 }
 
 // Shared checks and launch of the KV append; `one_per_seq` means

@@ -45,6 +45,7 @@ struct DecodeArgs {
     float* lse;               // [B][Hq]     (direct mode, nullable)
     int direct;               // 1: single split, write the final result
     int nstages;              // stage ring depth (runtime: sized from G and B)
+    int only_qv;              // 1: score = q . v (no K loads; the score reads the V rows)
 };
 
 template <int D>
@@ -62,8 +63,10 @@ struct DecodeCfg {
     __host__ __device__ static constexpr int tail_bytes(int G, int B, int ns) {
         return merge_bytes(G) + table_bytes(B) + 2 * ns * 8;
     }
-    __host__ __device__ static constexpr int smem_bytes(int G, int B, int ns) {
-        return 1024 + ns * STAGE + tail_bytes(G, B, ns);
+    // vonly: stages of V alone (the only_qv score reads no K)
+    __host__ __device__ static constexpr int stage_bytes(bool vonly) { return vonly ? STAGE_K : STAGE; }
+    __host__ __device__ static constexpr int smem_bytes(int G, int B, int ns, bool vonly = false) {
+        return 1024 + ns * stage_bytes(vonly) + tail_bytes(G, B, ns);
     }
 };
 
@@ -129,14 +132,19 @@ __global__ void __launch_bounds__(kDecThreads, 2)
     using C = DecodeCfg<D>;
     const int NS = a.nstages;
     const int G = a.group;
+    // A stage is K then V (STAGE_K bytes each), or with only_qv V alone: stage st's
+    // K and V sit at STAGE_K multiples kslot(st) and vslot(st).
+    const int STG = C::stage_bytes(a.only_qv);
+    auto kslot = [&](int st) { return a.only_qv ? st : 2 * st; };
+    auto vslot = [&](int st) { return a.only_qv ? st : 2 * st + 1; };
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
-    float* mo = reinterpret_cast<float*>(smem + NS * C::STAGE);       // [4][G][D]
+    float* mo = reinterpret_cast<float*>(smem + NS * STG);            // [4][G][D]
     float* mm = mo + 4 * G * D;                                        // [4][16]
     float* ml = mm + 4 * kDecRows;                                     // [4][16]
     int* prefix = reinterpret_cast<int*>(ml + 4 * kDecRows);           // [B+1] split-count prefix
     int* lenv = prefix + (a.B + 1);                                    // [B] keys per sequence
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + NS * C::STAGE + C::merge_bytes(G) +
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + NS * STG + C::merge_bytes(G) +
                                                  C::table_bytes(a.B));
     uint64_t* empty = full + NS;
 
@@ -219,17 +227,18 @@ __global__ void __launch_bounds__(kDecThreads, 2)
                     int npv = 0;
 #pragma unroll
                     for (int p = 0; p < 4; ++p) npv += ((sbase + p) * kPageRows < it.t_end) ? 1 : 0;
-                    mbar_arrive_expect_tx(&full[st], 2 * npv * kPageRows * C::ROWB);
-                    uint8_t* dk = smem + st * C::STAGE;
-                    uint8_t* dv = dk + C::STAGE_K;
+                    mbar_arrive_expect_tx(&full[st], (a.only_qv ? 1 : 2) * npv * kPageRows * C::ROWB);
+                    uint8_t* dk = smem + kslot(st) * C::STAGE_K;
+                    uint8_t* dv = smem + vslot(st) * C::STAGE_K;
 #pragma unroll
                     for (int p = 0; p < 4; ++p) {
                         if ((sbase + p) * kPageRows >= it.t_end) continue;
 #pragma unroll
                         for (int c = 0; c < C::NCHUNK; ++c) {
                             const int off = c * kDecStageTok * 128 + p * kPageRows * 128;
-                            tma_load_4d_hint(&tmK, &full[st], dk + off, c * 64, it.g,
-                                             pages[p] * kPageRows, 0, pol);
+                            if (!a.only_qv)
+                                tma_load_4d_hint(&tmK, &full[st], dk + off, c * 64, it.g,
+                                                 pages[p] * kPageRows, 0, pol);
                             tma_load_4d_hint(&tmV, &full[st], dv + off, c * 64, it.g,
                                              pages[p] * kPageRows, 0, pol);
                         }
@@ -285,8 +294,8 @@ __global__ void __launch_bounds__(kDecThreads, 2)
                     ok = __all_sync(0xffffffffu, ok);
                 }
                 const int tok0 = it.t_begin + s * kDecStageTok + warp * 16;   // this warp's 16 keys
-                uint8_t* sk = smem + st * C::STAGE;
-                uint8_t* sv = sk + C::STAGE_K;
+                uint8_t* sv = smem + vslot(st) * C::STAGE_K;
+                uint8_t* sk = smem + kslot(st) * C::STAGE_K;
                 const int lrow0 = warp * 16;
                 if (ok && tok0 < it.t_end) {
                     if (tok0 + 16 > it.t_end) {
@@ -465,17 +474,21 @@ struct DecodePagesArgs {
     float* lse_part;          // [grid + B][Hq]
     int* meta;                // [B + 1] page prefix, then pages per CTA (written by CTA 0)
     int nstages;
+    int only_qv;              // 1: score = q . v (no K loads; the score reads the V rows)
 };
 
 template <int D>
 struct DecodePagesCfg {
     static constexpr int ROWB = D * 2;
     static constexpr int NCHUNK = ROWB / 128;
-    // stage = one page of K and V for all heads: 2 * 16 * Hkv * D * 2 bytes
-    __host__ __device__ static constexpr int stage_bytes(int Hkv) { return 2 * kPageRows * Hkv * ROWB; }
+    // stage = one page of K and V for all heads: 2 * 16 * Hkv * D * 2 bytes (half: V alone,
+    // for the only_qv score)
+    __host__ __device__ static constexpr int stage_bytes(int Hkv, bool vonly = false) {
+        return (vonly ? 1 : 2) * kPageRows * Hkv * ROWB;
+    }
     __host__ __device__ static constexpr int table_bytes(int B) { return ((2 * B + 2) * 4 + 15) / 16 * 16; }
-    __host__ __device__ static constexpr int smem_bytes(int Hkv, int B, int ns) {
-        return 1024 + ns * stage_bytes(Hkv) + table_bytes(B) + 2 * ns * 8;
+    __host__ __device__ static constexpr int smem_bytes(int Hkv, int B, int ns, bool vonly = false) {
+        return 1024 + ns * stage_bytes(Hkv, vonly) + table_bytes(B) + 2 * ns * 8;
     }
 };
 
@@ -486,7 +499,8 @@ __global__ void __launch_bounds__(32 * (kPgMaxWarps + 1), 1)
     using C = DecodePagesCfg<D>;
     const int NS = a.nstages;
     const int Hkv = a.Hkv, G = a.group;
-    const int SB = C::stage_bytes(Hkv);
+    const int SB = C::stage_bytes(Hkv, a.only_qv);          // K and V of a page, or V alone
+    const int VOFF = a.only_qv ? 0 : SB / 2;                 // V's offset inside a stage
     const int rows = kPageRows * Hkv;            // rows of one 128-byte column of a stage tensor
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
@@ -574,10 +588,11 @@ __global__ void __launch_bounds__(32 * (kPgMaxWarps + 1), 1)
                 if (lane == 0) {
                     mbar_arrive_expect_tx(&full[st], SB);
                     uint8_t* dk = smem + st * SB;
-                    uint8_t* dv = dk + SB / 2;
+                    uint8_t* dv = dk + VOFF;
 #pragma unroll
                     for (int c = 0; c < C::NCHUNK; ++c) {
-                        tma_load_4d_hint(&tmK, &full[st], dk + c * rows * 128, c * 64, 0, 0, page, pol);
+                        if (!a.only_qv)
+                            tma_load_4d_hint(&tmK, &full[st], dk + c * rows * 128, c * 64, 0, 0, page, pol);
                         tma_load_4d_hint(&tmV, &full[st], dv + c * rows * 128, c * 64, 0, 0, page, pol);
                     }
                 }
@@ -667,8 +682,8 @@ __global__ void __launch_bounds__(32 * (kPgMaxWarps + 1), 1)
                 ok = __all_sync(0xffffffffu, ok);
             }
             const int tok0 = kb + (g - prefix[b]) * kPageRows;     // first key of this page
-            uint8_t* sk = smem + st * SB;
-            uint8_t* sv = sk + SB / 2;
+            uint8_t* sv = smem + st * SB + VOFF;
+            uint8_t* sk = a.only_qv ? sv : smem + st * SB;
             const int r0 = h * kPageRows;                      // this head's first row in the stage
             if (ok) {
                 if (tok0 + kPageRows > L) {

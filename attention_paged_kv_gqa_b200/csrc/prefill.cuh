@@ -71,6 +71,7 @@ struct PrefillArgs {
     float softcap;       // > 0: logit s -> softcap * tanh(s / softcap); 0: none
     int varlen;          // 1: rows addressed through cu_seqlens (batch coordinate 0)
     int paged;           // 1: K/V through block_table, 16-token pages
+    int only_qv;         // 1: score = Qv . V (selects the OQ kernel instance)
     int Lq, Lk;          // dense sizes (varlen == 0)
     const int* cu_q;
     const int* cu_k;
@@ -119,8 +120,12 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 }
 
 // CAP: the score softcap is compiled in (a separate instance, so that the
-// uncapped kernel carries none of its code).
-template <int D, bool FP8, bool CAP>
+// uncapped kernel carries none of its code).  OQ: the only_qv score, Qv . V --
+// no key tiles are fetched, the value tile is the score GEMM's B operand, and
+// the key stages and barriers deepen the value ring to 2 NS slots.  Both are
+// template parameters because the single MMA-issuing thread's control path is
+// on the critical path: runtime switches there cost measurable throughput.
+template <int D, bool FP8, bool CAP, bool OQ>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const PrefillArgs a) {
@@ -143,6 +148,12 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     uint64_t* o_final = p_full + 2;
     uint64_t* mma_done = o_final + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+    // Value ring: the NS value stages, and with only_qv (no key tiles) the NS key
+    // stages and their barriers too, so that 2 NS value tiles can be in flight.
+    constexpr int vring = OQ ? 2 * NS : NS;
+    auto vslot_buf = [&](int st) { return st < NS ? sV + st * C::KVB : sK + (st - NS) * C::KVB; };
+    auto vslot_full = [&](int st) { return st < NS ? &v_full[st] : &k_full[st - NS]; };
+    auto vslot_empty = [&](int st) { return st < NS ? &v_empty[st] : &k_empty[st - NS]; };
     int* sched = reinterpret_cast<int*>(tmem_slot + 2);   // [t][0]=min start, [t][1]=max end
 
     const int warp = threadIdx.x >> 5;
@@ -302,6 +313,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                 const int it = j - lo;
                 const int st = it % NS;
                 const uint32_t ph = (it / NS) & 1;
+                const int vst = it % vring;                 // value ring (2 NS deep with only_qv)
+                const uint32_t vph = (it / vring) & 1;
+                uint64_t* vfull = vslot_full(vst);
+                uint8_t* vbuf = vslot_buf(vst);
                 int page = -1;
                 constexpr int PPT = kBN / kPageRows;   // pages per tile
                 if (a.paged && lane < PPT) {
@@ -314,58 +329,60 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                 for (int p = 0; p < PPT; ++p) npv += (j * kBN + p * kPageRows < Lk) ? 1 : 0;
                 const uint32_t bytes = a.paged ? npv * kPageRows * C::ROWB : C::KVB;
 
-                bool ok = mbar_wait(&k_empty[st], ph ^ 1, kErrProdKEmpty);
-                ok = __all_sync(0xffffffffu, ok);
-                if (!ok) break;
-                if (a.paged) {
-                    // the tile's byte count first, then each page lane issues its own page's boxes
-                    if (lane == 0) mbar_arrive_expect_tx(&k_full[st], bytes);
-                    __syncwarp();
-                    if (lane < PPT && j * kBN + lane * kPageRows < Lk) {
-                        uint8_t* dst = sK + st * C::KVB + lane * kPageRows * 128;
+                bool ok = true;
+                if constexpr (!OQ) {
+                    ok = mbar_wait(&k_empty[st], ph ^ 1, kErrProdKEmpty);
+                    ok = __all_sync(0xffffffffu, ok);
+                    if (!ok) break;
+                    if (a.paged) {
+                        // the tile's byte count first, then each page lane issues its own page's boxes
+                        if (lane == 0) mbar_arrive_expect_tx(&k_full[st], bytes);
+                        __syncwarp();
+                        if (lane < PPT && j * kBN + lane * kPageRows < Lk) {
+                            uint8_t* dst = sK + st * C::KVB + lane * kPageRows * 128;
+#pragma unroll
+                            for (int c = 0; c < C::NCHUNK; ++c)
+                                tma_load_4d_hint(&tmK, &k_full[st], dst + c * kBN * 128, c * C::CHUNK_E, g,
+                                                 page * kPageRows, 0, pol);
+                        }
+                    } else if (lane == 0) {
+                        mbar_arrive_expect_tx(&k_full[st], bytes);
+                        uint8_t* dst = sK + st * C::KVB;
 #pragma unroll
                         for (int c = 0; c < C::NCHUNK; ++c)
-                            tma_load_4d_hint(&tmK, &k_full[st], dst + c * kBN * 128, c * C::CHUNK_E, g,
-                                             page * kPageRows, 0, pol);
+                            tma_load_4d_hint(&tmK, &k_full[st], dst + c * kBN * 128,
+                                             c * C::CHUNK_E, g, k_off + j * kBN, bcoord, pol);
                     }
-                } else if (lane == 0) {
-                    mbar_arrive_expect_tx(&k_full[st], bytes);
-                    uint8_t* dst = sK + st * C::KVB;
-#pragma unroll
-                    for (int c = 0; c < C::NCHUNK; ++c)
-                        tma_load_4d_hint(&tmK, &k_full[st], dst + c * kBN * 128,
-                                         c * C::CHUNK_E, g, k_off + j * kBN, bcoord, pol);
                 }
-                ok = mbar_wait(&v_empty[st], ph ^ 1, kErrProdVEmpty);
+                ok = mbar_wait(vslot_empty(vst), vph ^ 1, kErrProdVEmpty);
                 ok = __all_sync(0xffffffffu, ok);
-                if (!ok) { ++issued; break; }
+                if (!ok) { if (!OQ) ++issued; break; }
                 if (a.paged) {
                     // the tile's byte count first, then each page lane issues its own page's boxes
-                    if (lane == 0) mbar_arrive_expect_tx(&v_full[st], bytes);
+                    if (lane == 0) mbar_arrive_expect_tx(vfull, bytes);
                     __syncwarp();
                     if (lane < PPT && j * kBN + lane * kPageRows < Lk) {
-                        uint8_t* dst = sV + st * C::KVB + lane * kPageRows * 128;
+                        uint8_t* dst = vbuf + lane * kPageRows * 128;
 #pragma unroll
                         for (int c = 0; c < C::NCHUNK; ++c)
-                            tma_load_4d_hint(&tmV, &v_full[st], dst + c * kBN * 128, c * C::CHUNK_E, g,
+                            tma_load_4d_hint(&tmV, vfull, dst + c * kBN * 128, c * C::CHUNK_E, g,
                                              page * kPageRows, 0, pol);
                     }
                 } else if (lane == 0) {
-                    mbar_arrive_expect_tx(&v_full[st], bytes);
-                    uint8_t* dst = sV + st * C::KVB;
+                    mbar_arrive_expect_tx(vfull, bytes);
 #pragma unroll
                     for (int c = 0; c < C::NCHUNK; ++c)
-                        tma_load_4d_hint(&tmV, &v_full[st], dst + c * kBN * 128,
+                        tma_load_4d_hint(&tmV, vfull, vbuf + c * kBN * 128,
                                          c * C::CHUNK_E, g, k_off + j * kBN, bcoord, pol);
                 }
             }
             // Let every copy this warp started land before the CTA can exit.
             if (lane == 0) {
-                for (int st = 0; st < NS && st < issued; ++st) {
-                    const int last = st + ((issued - 1 - st) / NS) * NS;
-                    const uint32_t ph = (last / NS) & 1;
-                    mbar_wait(&k_full[st], ph, kErrProdDrain);
-                    mbar_wait(&v_full[st], ph, kErrProdDrain);
+                for (int st = 0; st < vring && st < issued; ++st) {
+                    const int last = st + ((issued - 1 - st) / vring) * vring;
+                    const uint32_t ph = (last / vring) & 1;
+                    if (!OQ) mbar_wait(&k_full[st], ph, kErrProdDrain);
+                    mbar_wait(vslot_full(st), ph, kErrProdDrain);
                 }
             }
         }
@@ -374,24 +391,26 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         if (any_tiles && lane == 0) {
             const uint32_t tS[2] = {tbase, tbase + 128};
             const uint32_t tO[2] = {tbase + 256, tbase + 256 + D};
-            const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
+            const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK);
             auto part = [&](int t, int j) { return lo_t[t] <= j && j < hi_t[t]; };
-            auto issue_s = [&](int t, int st) {
+            // score GEMM: B operand at kb (the key tile; with only_qv the value tile, whose
+            // slot is released by the P.V GEMM that reads it last)
+            auto issue_s = [&](int t, uint32_t kb) {
 #pragma unroll
                 for (int kk = 0; kk < C::QK_STEPS; ++kk) {
                     const uint32_t cb = (kk * 32) / 128, off = (kk * 32) % 128;
                     const uint32_t qa = sQa + t * C::QB + cb * kBM * 128 + off;
-                    const uint32_t ka = sKa + st * C::KVB + cb * kBN * 128 + off;
+                    const uint32_t ka = kb + cb * kBN * 128 + off;
                     const uint64_t da = smem_desc(qa, 16, 1024, 2);
                     const uint64_t db = smem_desc(ka, 16, 1024, 2);
                     if constexpr (FP8) mma_f8_ss(tS[t], da, db, C::IDESC_QK, kk > 0);
                     else mma_f16_ss(tS[t], da, db, C::IDESC_QK, kk > 0);
                 }
             };
-            auto issue_pv = [&](int t, int st, bool acc) {
+            auto issue_pv = [&](int t, uint32_t vb, bool acc) {
 #pragma unroll
                 for (int kk = 0; kk < C::PV_STEPS; ++kk) {
-                    const uint32_t va = sVa + st * C::KVB + kk * (C::KSTEP / 8) * 1024;
+                    const uint32_t va = vb + kk * (C::KSTEP / 8) * 1024;
                     const uint64_t db = smem_desc(va, kBN * 128, 1024, 2);
                     const uint32_t pa = tS[t] + kk * 8;
                     if constexpr (FP8) mma_f8_ts(tO[t], pa, db, C::IDESC_PV, (acc || kk > 0) ? 1u : 0u);
@@ -401,16 +420,17 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             bool ok = mbar_wait(q_full, 0, kErrMmaQ);
             bool started[2] = {false, false};
             int pcount[2] = {0, 0};
-            if (ok) ok = mbar_wait(&k_full[0], 0, kErrMmaK);
+            if (ok) ok = mbar_wait(OQ ? vslot_full(0) : &k_full[0], 0, kErrMmaK);
             if (ok) {
                 tc_fence_after();
+                const uint32_t kb0 = OQ ? smem_u32(vslot_buf(0)) : sKa;
 #pragma unroll
                 for (int t = 0; t < 2; ++t)
                     if (part(t, lo)) {
-                        issue_s(t, 0);
+                        issue_s(t, kb0);
                         mma_commit(&s_full[t]);
                     }
-                mma_commit(&k_empty[0]);
+                if (!OQ) mma_commit(&k_empty[0]);
             }
             for (int j = lo; ok && j < hi; ++j) {
                 const int it = j - lo;
@@ -418,32 +438,36 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                 const uint32_t ph = (it / NS) & 1;
                 const int st1 = (it + 1) % NS;
                 const uint32_t ph1 = ((it + 1) / NS) & 1;
+                const int vst = it % vring, vst1 = (it + 1) % vring;
+                const uint32_t vph = (it / vring) & 1, vph1 = ((it + 1) / vring) & 1;
                 const bool next = j + 1 < hi;
                 bool k1 = false;
-                if (!(ok = mbar_wait(&v_full[st], ph, kErrMmaV))) break;
+                if (!(ok = mbar_wait(vslot_full(vst), vph, kErrMmaV))) break;
 #pragma unroll
                 for (int t = 0; t < 2; ++t) {
                     if (part(t, j)) {
                         if (!(ok = mbar_wait(&p_full[t], pcount[t] & 1, kErrMmaP))) break;
                         ++pcount[t];
                         tc_fence_after();
-                        issue_pv(t, st, started[t]);
+                        issue_pv(t, smem_u32(vslot_buf(vst)), started[t]);
                         started[t] = true;
                         if (j == hi_t[t] - 1) mma_commit(&o_final[t]);
                     }
                     if (next && part(t, j + 1)) {
                         if (!k1) {
-                            if (!(ok = mbar_wait(&k_full[st1], ph1, kErrMmaK))) break;
+                            ok = OQ ? mbar_wait(vslot_full(vst1), vph1, kErrMmaK)
+                                           : mbar_wait(&k_full[st1], ph1, kErrMmaK);
+                            if (!ok) break;
                             tc_fence_after();
                             k1 = true;
                         }
-                        issue_s(t, st1);
+                        issue_s(t, OQ ? smem_u32(vslot_buf(vst1)) : sKa + st1 * C::KVB);
                         mma_commit(&s_full[t]);
                     }
                 }
                 if (!ok) break;
-                mma_commit(&v_empty[st]);
-                if (next) {
+                mma_commit(vslot_empty(vst));
+                if (next && !OQ) {
                     if (!k1 && !(ok = mbar_wait(&k_full[st1], ph1, kErrMmaK))) break;
                     mma_commit(&k_empty[st1]);
                 }
@@ -596,11 +620,11 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                 const int zt = (lo_t[0] <= j && j < hi_t[0]) ? 0 : 1;
                 if (zt == t) {
                     const int it = j - lo;
-                    const int st = it % NS;
-                    ok = mbar_wait(&v_full[st], (it / NS) & 1, kErrSmV);
+                    const int st = it % vring;
+                    ok = mbar_wait(vslot_full(st), (it / vring) & 1, kErrSmV);
                     if (ok) {
                         const int first = Lk - j * kBN;
-                        uint8_t* base = sV + st * C::KVB;
+                        uint8_t* base = vslot_buf(st);
                         const int nrow = kBN - first;
                         const int n16 = nrow * C::NCHUNK * 8;     // 16-byte pieces
                         for (int i = r; i < n16; i += kBM) {

@@ -85,7 +85,7 @@ def parse_args():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-prefill", action="store_true")
     p.add_argument("--workload", choices=["all", "decode", "prefill", "fp8", "window", "append",
-                                          "backward"],
+                                          "backward", "only_qv"],
                    default="all",
                    help="run only one workload (profiling runs); the JSON line then carries "
                         "only what ran")
@@ -372,6 +372,8 @@ def run_ours(args, rank, world, local):
         run_append(args, A, W, dev, world, flush, peaks, peak_kind, line)
     if args.workload in ("all", "backward") and not args.no_prefill:
         run_backward(args, A, W, dev, world, flush, peaks, peak_kind, line)
+    if args.workload in ("all", "only_qv") and not args.no_prefill:
+        run_only_qv(args, A, W, dev, world, flush, peaks, peak_kind, line)
     if args.workload in ("all", "decode") and rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
     if rank == 0:
@@ -699,6 +701,63 @@ def run_backward(args, A, W, dev, world, flush, peaks, peak_kind, line):
                                                 "(+ bwd_delta_kernel)", "peak_kind": peak_kind},
     }
     del q, k, v, do, o, dq, dk, dv
+
+
+def run_only_qv(args, A, W, dev, world, flush, peaks, peak_kind, line):
+    """The only_qv score path (score = scale * qv . v) on the decode and prefill workloads:
+    the query tensor serves as qv and the value cache as the only KV store."""
+    w = W.paged_decode(seed=args.seed)
+    t, P = w.tensors, w.params
+    d = {k: v.to(dev) for k, v in t.items() if k != "k_cache"}
+    ws = torch.empty(max(A.attn_decode_workspace_size(P["B"], P["Hq"], P["Hkv"], P["D"],
+                                                      P["max_blocks_per_seq"]), 16),
+                     dtype=torch.uint8, device=dev)
+    o = torch.empty(P["B"], P["Hq"], P["D"], dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(P["B"], P["Hq"], dtype=torch.float32, device=dev)
+
+    def dec_step():
+        A.attn_decode_paged_only_qv(d["q"], d["v_cache"], d["block_table"], d["seqused_k"],
+                                    scale=P["scale"], out=o, lse=lse, workspace=ws)
+
+    dms = statistics.mean(time_steps(dec_step, args.steps, args.warmup, world, flush))
+    # algorithmic bytes: decode_bytes with the V half of the K/V stream only
+    lens = t["seqused_k"].numpy().astype(np.int64)
+    nb = decode_bytes(t, P["Hq"], P["Hkv"], P["D"]) - int(lens.sum()) * P["Hkv"] * P["D"] * 2
+    gbs = nb / (dms * 1e-3) / 1e9
+    out = {"decode": {"value": round(gbs, 2), "unit": "GB/s", "ms_per_step": round(dms, 5),
+                      "bytes_per_step": nb,
+                      "roofline": {"bound": "hbm", "achieved": round(gbs, 1),
+                                   "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                   "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": None,
+                                   "peak_kind": peak_kind}}}
+    del d
+
+    wp = W.varlen_paged_prefill(seed=args.seed)
+    tp, Pp = wp.tensors, wp.params
+    dp = {k: v.to(dev) for k, v in tp.items() if k != "k_cache"}
+    op = torch.empty(Pp["total_q"], Pp["Hq"], Pp["D"], dtype=torch.bfloat16, device=dev)
+    lp = torch.empty(Pp["Hq"], Pp["total_q"], dtype=torch.float32, device=dev)
+
+    def pf_step():
+        A.attn_fwd_varlen_paged_only_qv(dp["q"], dp["v_cache"], cu_seqlens_q=dp["cu_seqlens_q"],
+                                        max_seqlen_q=Pp["max_seqlen_q"],
+                                        block_table=dp["block_table"], seqused_k=dp["seqused_k"],
+                                        mask=A.MASK_CAUSAL, scale=Pp["scale"], out=op, lse=lp)
+
+    pms = statistics.mean(time_steps(pf_step, args.steps, args.warmup, world, flush))
+    fl = causal_flops(tp["seqused_k"].numpy(), Pp["Hq"], Pp["D"])
+    tf = fl / (pms * 1e-3) / 1e12
+    out["prefill"] = {"value": round(tf, 2), "unit": "TFLOP/s", "ms_per_step": round(pms, 5),
+                      "flops_per_step": fl,
+                      "roofline": {"bound": "tensor", "achieved": round(tf, 1),
+                                   "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                                   "frac": round(tf / peaks["bf16_tflops"], 4), "traffic": None,
+                                   "peak_kind": peak_kind}}
+    del dp
+    out["workloads"] = ("the paged GQA decode and varlen paged GQA causal prefill workloads "
+                        "above with the query tensor as qv and the value cache as the only "
+                        "KV store; decode bytes count V once (no K stream)")
+    line["only_qv"] = out
 
 
 def cpu_baseline(w):

@@ -165,6 +165,27 @@ attn_status_t attn_fwd_varlen_paged(
     void *o, float *lse, void *workspace, size_t workspace_bytes, attn_stream_t stream);
 
 /*
+ * The only_qv score path of "Rope dim" (vllm-project flash-attention PR 172,
+ * overview: the mode that skips the Q and K loads and the QK GEMM and
+ * zero-initialises the score with the Qv GEMM).  The score of query i and key
+ * j is scale * (qv_i . v_j): the value rows serve as the score's second
+ * operand, and there is no key store.  Everything else (masks, window,
+ * softcap, LSE, paging, varlen, fp8) is as in attn_fwd_varlen_paged, with
+ *   qv           in place of q: [total_q, Hq, D], the value head dimension.
+ *   v_cache      the only KV store, laid out as v_cache there.
+ *   descale_qv, descale_v   fp8 only; the score uses descale_qv * descale_v.
+ * No key tile is fetched: each value tile is read once and feeds both the
+ * score GEMM and the P.V GEMM.
+ */
+attn_status_t attn_fwd_varlen_paged_only_qv(
+    const void *qv, const void *v_cache, const int32_t *block_table, int max_blocks_per_seq,
+    int num_blocks, int block_size, const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
+    const int32_t *seqused_k, int B, int total_q, int total_k, int max_seqlen_q,
+    int num_heads_q, int num_heads_kv, int head_dim, float softmax_scale, int mask,
+    const int32_t *patch_kv_range, int window_left, float softcap, int dtype,
+    const float *descale_qv, const float *descale_v, void *o, float *lse, attn_stream_t stream);
+
+/*
  * Bytes of workspace attn_decode_paged needs for these sizes (fp32 partial O
  * and LSE per split).  num_splits <= 0 means "as chosen automatically for
  * max_blocks_per_seq".  Returns 0 for invalid sizes.
@@ -193,6 +214,20 @@ attn_status_t attn_decode_paged(
     int window_left, float softcap, int num_splits, int dtype,
     const float *descale_q, const float *descale_k, const float *descale_v,
     void *o, float *lse, void *workspace, size_t workspace_bytes, attn_stream_t stream);
+
+/*
+ * Paged decode with the only_qv score (as attn_fwd_varlen_paged_only_qv): the
+ * score of key j is scale * (qv . v_j), read from the one value store; each
+ * page of V is fetched once.  Arguments as attn_decode_paged with qv in place
+ * of q and without the key store; workspace sized by attn_decode_workspace_size.
+ * Supported: bf16, head_dim in {64, 128}, Hq/Hkv <= 16.
+ */
+attn_status_t attn_decode_paged_only_qv(
+    const void *qv, const void *v_cache, const int32_t *block_table, int max_blocks_per_seq,
+    int num_blocks, int block_size, const int32_t *seqused_k, int B, int num_heads_q,
+    int num_heads_kv, int head_dim, float softmax_scale, int window_left, float softcap,
+    int num_splits, int dtype, void *o, float *lse, void *workspace, size_t workspace_bytes,
+    attn_stream_t stream);
 
 /*
  * Paged KV append: writes new tokens' keys and values into the paged cache

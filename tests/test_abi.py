@@ -127,3 +127,27 @@ def test_window_and_softcap_rules(L):
     st = L.attn_decode_paged(p, p, p, p, 4, 100, 16, p, 1, 8, 2, 128, 0.0, 5, -2.0, 0, 0, None,
                              None, None, p, None, p, 1 << 20, None)
     assert st == 1                                 # negative softcap in decode
+
+
+def test_only_qv_entry_points_check_arguments(L):
+    """The only_qv calls share the forward's and the decode's checks (no launch on a bad call)."""
+    p = ctypes.c_void_p(1 << 20)
+    cu = ctypes.c_void_p(1 << 21)
+    # qv missing
+    st = L.attn_fwd_varlen_paged_only_qv(None, p, p, 4, 100, 16, cu, None, cu, 1, 16, 0, 16, 2, 2,
+                                         64, 0.0, 1, None, -1, 0.0, 0, None, None, p, None, None)
+    assert st == 1
+    # block_size 32 -> unsupported; fp8 without descales -> invalid
+    st = L.attn_fwd_varlen_paged_only_qv(p, p, p, 4, 100, 32, cu, None, cu, 1, 16, 0, 16, 2, 2,
+                                         64, 0.0, 1, None, -1, 0.0, 0, None, None, p, None, None)
+    assert st == 2
+    st = L.attn_fwd_varlen_paged_only_qv(p, p, p, 4, 100, 16, cu, None, cu, 1, 16, 0, 16, 2, 2,
+                                         128, 0.0, 1, None, -1, 0.0, 1, None, None, p, None, None)
+    assert st == 1
+    # decode: group beyond 16 rows -> unsupported; missing seqused_k -> invalid
+    st = L.attn_decode_paged_only_qv(p, p, p, 4, 100, 16, p, 1, 32, 1, 128, 0.0, -1, 0.0, 1, 0,
+                                     p, None, p, 1 << 20, None)
+    assert st == 2
+    st = L.attn_decode_paged_only_qv(p, p, p, 4, 100, 16, None, 1, 8, 2, 128, 0.0, -1, 0.0, 1, 0,
+                                     p, None, p, 1 << 20, None)
+    assert st == 1
