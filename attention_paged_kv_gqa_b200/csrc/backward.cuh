@@ -31,9 +31,20 @@
 
 namespace attn {
 
-constexpr int kBwdThreads = 192;   // warps 0-3 compute (thread = TMEM lane), 4 TMA, 5 MMA
-constexpr int kBwdProducerWarp = 4;
-constexpr int kBwdMmaWarp = 5;
+// Warps 0-7: two compute warpgroups (thread = TMEM lane; warpgroup h takes the
+// score columns [64 h, 64 h + 64)), 8: TMA, 9: MMA.  Warpgroup h writes its bf16
+// results (8 columns per 16 score columns) into columns it has already read:
+// [32 h + 16 c, ...) for its c-th 32-column block, i.e. columns [0, 32) and
+// [64, 96); the accumulating GEMMs read their A operand there.
+constexpr int kBwdThreads = 320;
+constexpr int kBwdProducerWarp = 8;
+constexpr int kBwdMmaWarp = 9;
+constexpr int kBwdComputeThreads = 256;
+
+// TMEM column of the bf16 results of 32-column block c4 (0..3) of a score tile.
+__device__ __forceinline__ uint32_t bwd_out_col(int c4) { return 16 * c4 + (c4 >= 2 ? 32 : 0); }
+// ... and of k-step kk (16 rows, 8 columns) of the accumulating GEMM's A operand.
+__device__ __forceinline__ uint32_t bwd_a_col(int kk) { return 8 * kk + (kk >= 4 ? 32 : 0); }
 
 enum : int {
     kErrBwdLoad = 601, kErrBwdMma = 602, kErrBwdCompute = 603, kErrBwdDrain = 604,
@@ -162,7 +173,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             mbar_init(&kv_empty[i], 1);
         }
         mbar_init(s_full, 1);
-        mbar_init(p_full, 128);
+        mbar_init(p_full, kBwdComputeThreads);
         mbar_init(mma_done, 1);
         fence_mbar_init();
     }
@@ -237,7 +248,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
                 for (int kk = 0; kk < 128 / C::KSTEP; ++kk) {
                     const uint64_t db = smem_desc(sKa + st * C::TILE + kk * 2 * 1024, 128 * 128, 1024, 2);
-                    mma_f16_ts(tdQ, tS + kk * 8, db, C::IDESC_TS, (it > 0 || kk > 0) ? 1u : 0u);
+                    mma_f16_ts(tdQ, tS + bwd_a_col(kk), db, C::IDESC_TS, (it > 0 || kk > 0) ? 1u : 0u);
                 }
                 mma_commit(&kv_empty[st]);
             }
@@ -245,9 +256,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             mbar_wait(mma_done, 0, kErrBwdMma);
         }
     } else {
-        // ---------------------------------------------------- compute warpgroup: dS, then dQ out
-        const int r = warp * 32 + lane;
-        const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+        // ---------------------------------------------------- compute warpgroups: dS, then dQ out
+        const int quad = warp & 3, hf = warp >> 2;   // TMEM lane quarter; score column half
+        const int r = quad * 32 + lane;
+        const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
         const int qi = q0 + r;
         const bool row_ok = qi < Lq;
         float lse2 = INFINITY, dlt = 0.0f;         // rows past the sequence: P = 0
@@ -269,7 +281,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             const int kbase = j * 128;
             const bool partial = kbase < klo || kbase + 128 > khi;
 #pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) {
+            for (int cc = 0; cc < 2; ++cc) {
+                const int c4 = 2 * hf + cc;
                 uint32_t us[32], ud[32];
                 tmem_ld32(tS + lane_off + c4 * 32, us);
                 tmem_ld32(tdP + lane_off + c4 * 32, ud);
@@ -287,8 +300,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     }
                     pk[c] = pack_bf16(ds[0], ds[1]);
                 }
-                // dS chunk c4 -> columns [16 c4, 16 c4 + 16), all already read
-                tmem_st16(tS + lane_off + c4 * 16, pk);
+                // dS of block c4 -> columns this warpgroup has already read
+                tmem_st16(tS + lane_off + bwd_out_col(c4), pk);
             }
             tmem_wait_st();
             tc_fence_before();
@@ -302,9 +315,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         __nv_bfloat16* dst = a.dq + ((long long)(q_off + qi) * a.Hq + h) * D;
         __syncwarp();
+        // warpgroup hf writes the D columns [D/2 hf, D/2 hf + D/2) of its rows
         if (have) {
 #pragma unroll
-            for (int c4 = 0; c4 < D / 32; ++c4) {
+            for (int cc = 0; cc < D / 64; ++cc) {
+                const int c4 = hf * (D / 64) + cc;
                 uint32_t u[32];
                 tmem_ld32(tdQ + lane_off + c4 * 32, u);
                 tmem_wait_ld();
@@ -321,7 +336,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 }
             }
         } else if (row_ok) {
-            for (int v4 = 0; v4 < D / 8; ++v4) reinterpret_cast<uint4*>(dst)[v4] = make_uint4(0, 0, 0, 0);
+            for (int v4 = hf * (D / 16); v4 < (hf + 1) * (D / 16); ++v4)
+                reinterpret_cast<uint4*>(dst)[v4] = make_uint4(0, 0, 0, 0);
         }
         tc_fence_before();
     }
@@ -390,7 +406,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             mbar_init(&st_empty[i], 1);
         }
         mbar_init(s_full, 1);
-        mbar_init(p_full, 128);
+        mbar_init(p_full, kBwdComputeThreads);
         mbar_init(mma_done, 1);
         fence_mbar_init();
     }
@@ -490,9 +506,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
                 for (int kk = 0; kk < 128 / C::KSTEP; ++kk) {
                     const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
-                    mma_f16_ts(tdV, tST + kk * 8, smem_desc(sdOa + kk * 2 * 1024, 128 * 128, 1024, 2),
+                    mma_f16_ts(tdV, tST + bwd_a_col(kk), smem_desc(sdOa + kk * 2 * 1024, 128 * 128, 1024, 2),
                                C::IDESC_TS, acc);
-                    mma_f16_ts(tdK, tdPT + kk * 8, smem_desc(sQa + kk * 2 * 1024, 128 * 128, 1024, 2),
+                    mma_f16_ts(tdK, tdPT + bwd_a_col(kk), smem_desc(sQa + kk * 2 * 1024, 128 * 128, 1024, 2),
                                C::IDESC_TS, acc);
                 }
                 mma_commit(&st_empty[st]);
@@ -501,9 +517,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             mbar_wait(mma_done, 0, kErrBwdMma);
         }
     } else {
-        // ---------------------------------------------------- compute warpgroup (thread = key)
-        const int r = warp * 32 + lane;
-        const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+        // ---------------------------------------------------- compute warpgroups (thread = key)
+        const int quad = warp & 3, hf = warp >> 2;   // TMEM lane quarter; query column half
+        const int r = quad * 32 + lane;
+        const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
         const int j = k0 + r;
         const bool key_ok = j < Lk;
         const float sl2 = a.scale * kLog2e;
@@ -522,38 +539,55 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             const float* sL = stL(st);
             const float* sDl = stDl(st);
             const int ibase = qt * 128;
-            // key j is allowed for row i iff (causal) j <= i + dl and (window) j >= i + dl - W
+            // key j is allowed for row i iff (causal) j <= i + dl and (window) j >= i + dl - W;
+            // a tile whose every (row, key) pair is allowed skips the per-element test
+            // (rows past the sequence have LSE = +inf, so P = 0 there anyway)
             const bool causal = a.mask == kMaskCausal;
+            bool all_ok = k0 + 128 <= Lk;
+            if (causal) {
+                all_ok = all_ok && k0 + 127 <= ibase + dl;
+                if (a.window >= 0) all_ok = all_ok && k0 >= ibase + 127 + dl - a.window;
+            }
 #pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) {
+            for (int cc = 0; cc < 2; ++cc) {
+                const int c4 = 2 * hf + cc;
                 uint32_t us[32], ud[32];
                 tmem_ld32(tST + lane_off + c4 * 32, us);
                 tmem_ld32(tdPT + lane_off + c4 * 32, ud);
                 tmem_wait_ld();
                 uint32_t pp[16], dd[16];
+                float4 lv, dv;   // 4 rows of LSE (base 2) and Delta, broadcast from shared memory
 #pragma unroll
                 for (int c = 0; c < 16; ++c) {
+                    if ((c & 1) == 0) {
+                        lv = reinterpret_cast<const float4*>(sL + c4 * 32)[c / 2];
+                        dv = reinterpret_cast<const float4*>(sDl + c4 * 32)[c / 2];
+                    }
+                    const float l4[4] = {lv.x, lv.y, lv.z, lv.w};
+                    const float d4[4] = {dv.x, dv.y, dv.z, dv.w};
                     float p2[2], ds2[2];
 #pragma unroll
                     for (int e = 0; e < 2; ++e) {
-                        const int col = c4 * 32 + 2 * c + e;
-                        const int i = ibase + col;
-                        float p = ex2(fmaf(__uint_as_float(us[2 * c + e]), sl2, -sL[col]));
-                        bool allowed = key_ok;
-                        if (causal) {
-                            allowed = allowed && j <= i + dl;
-                            if (a.window >= 0) allowed = allowed && j >= i + dl - a.window;
+                        const int col = 2 * c + e;
+                        const int i = ibase + c4 * 32 + col;
+                        float p = ex2(fmaf(__uint_as_float(us[col]), sl2, -l4[col & 3]));
+                        if (!all_ok) {
+                            bool allowed = key_ok;
+                            if (causal) {
+                                allowed = allowed && j <= i + dl;
+                                if (a.window >= 0) allowed = allowed && j >= i + dl - a.window;
+                            }
+                            if (!allowed) p = 0.0f;
                         }
-                        if (!allowed) p = 0.0f;
                         p2[e] = p;
-                        ds2[e] = p * (__uint_as_float(ud[2 * c + e]) - sDl[col]) * a.scale;
+                        ds2[e] = p * (__uint_as_float(ud[col]) - d4[col & 3]) * a.scale;
                     }
                     pp[c] = pack_bf16(p2[0], p2[1]);
                     dd[c] = pack_bf16(ds2[0], ds2[1]);
                 }
-                // chunk c4 -> columns [16 c4, 16 c4 + 16) of S^T / dP^T, all already read
-                tmem_st16(tST + lane_off + c4 * 16, pp);
-                tmem_st16(tdPT + lane_off + c4 * 16, dd);
+                // block c4 -> columns this warpgroup has already read
+                tmem_st16(tST + lane_off + bwd_out_col(c4), pp);
+                tmem_st16(tdPT + lane_off + bwd_out_col(c4), dd);
             }
             tmem_wait_st();
             tc_fence_before();
@@ -566,8 +600,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             tc_fence_after();
         }
         __syncwarp();
-#pragma unroll
-        for (int which = 0; which < 2; ++which) {
+        // warpgroup 0 writes dV, warpgroup 1 dK
+        {
+            const int which = hf;
             const uint32_t tacc = which == 0 ? tdV : tdK;
             __nv_bfloat16* dst = (which == 0 ? a.dv : a.dk) + ((long long)(k_off + j) * a.Hkv + g) * D;
             if (have) {
