@@ -31,20 +31,22 @@
 
 namespace attn {
 
-// Warps 0-7: two compute warpgroups (thread = TMEM lane; warpgroup h takes the
-// score columns [64 h, 64 h + 64)), 8: TMA, 9: MMA.  Warpgroup h writes its bf16
-// results (8 columns per 16 score columns) into columns it has already read:
-// [32 h + 16 c, ...) for its c-th 32-column block, i.e. columns [0, 32) and
-// [64, 96); the accumulating GEMMs read their A operand there.
-constexpr int kBwdThreads = 320;
-constexpr int kBwdProducerWarp = 8;
-constexpr int kBwdMmaWarp = 9;
-constexpr int kBwdComputeThreads = 256;
+// Warps 0 .. 4 kBwdWG - 1: compute warpgroups (thread = TMEM lane; warpgroup h
+// takes the 32-column blocks c4 = h, h + kBwdWG, .. of a 128-column score
+// tile); then the TMA warp and the MMA warp.  A block's bf16 results (16
+// columns) are written over the first half of the block itself, which its
+// warpgroup has already read, so no warpgroup writes where another reads; the
+// accumulating GEMMs read their A operand there.
+constexpr int kBwdWG = 4;
+constexpr int kBwdComputeThreads = 128 * kBwdWG;
+constexpr int kBwdProducerWarp = 4 * kBwdWG;
+constexpr int kBwdMmaWarp = 4 * kBwdWG + 1;
+constexpr int kBwdThreads = kBwdComputeThreads + 64;
 
 // TMEM column of the bf16 results of 32-column block c4 (0..3) of a score tile.
-__device__ __forceinline__ uint32_t bwd_out_col(int c4) { return 16 * c4 + (c4 >= 2 ? 32 : 0); }
+__device__ __forceinline__ uint32_t bwd_out_col(int c4) { return 32 * c4; }
 // ... and of k-step kk (16 rows, 8 columns) of the accumulating GEMM's A operand.
-__device__ __forceinline__ uint32_t bwd_a_col(int kk) { return 8 * kk + (kk >= 4 ? 32 : 0); }
+__device__ __forceinline__ uint32_t bwd_a_col(int kk) { return 32 * (kk >> 1) + 8 * (kk & 1); }
 
 enum : int {
     kErrBwdLoad = 601, kErrBwdMma = 602, kErrBwdCompute = 603, kErrBwdDrain = 604,
@@ -257,7 +259,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
     } else {
         // ---------------------------------------------------- compute warpgroups: dS, then dQ out
-        const int quad = warp & 3, hf = warp >> 2;   // TMEM lane quarter; score column half
+        const int quad = warp & 3, hf = warp >> 2;   // TMEM lane quarter; warpgroup
         const int r = quad * 32 + lane;
         const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
         const int qi = q0 + r;
@@ -281,8 +283,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             const int kbase = j * 128;
             const bool partial = kbase < klo || kbase + 128 > khi;
 #pragma unroll
-            for (int cc = 0; cc < 2; ++cc) {
-                const int c4 = 2 * hf + cc;
+            for (int cc = 0; cc < 4 / kBwdWG; ++cc) {
+                const int c4 = hf + cc * kBwdWG;
                 uint32_t us[32], ud[32];
                 tmem_ld32(tS + lane_off + c4 * 32, us);
                 tmem_ld32(tdP + lane_off + c4 * 32, ud);
@@ -315,11 +317,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         __nv_bfloat16* dst = a.dq + ((long long)(q_off + qi) * a.Hq + h) * D;
         __syncwarp();
-        // warpgroup hf writes the D columns [D/2 hf, D/2 hf + D/2) of its rows
+        // warpgroup hf writes the 32-column blocks hf, hf + kBwdWG, .. of its rows' dQ
         if (have) {
 #pragma unroll
-            for (int cc = 0; cc < D / 64; ++cc) {
-                const int c4 = hf * (D / 64) + cc;
+            for (int c4 = hf; c4 < D / 32; c4 += kBwdWG) {
                 uint32_t u[32];
                 tmem_ld32(tdQ + lane_off + c4 * 32, u);
                 tmem_wait_ld();
@@ -336,8 +337,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 }
             }
         } else if (row_ok) {
-            for (int v4 = hf * (D / 16); v4 < (hf + 1) * (D / 16); ++v4)
-                reinterpret_cast<uint4*>(dst)[v4] = make_uint4(0, 0, 0, 0);
+            for (int c4 = hf; c4 < D / 32; c4 += kBwdWG)
+                for (int v4 = 0; v4 < 4; ++v4)
+                    reinterpret_cast<uint4*>(dst + c4 * 32)[v4] = make_uint4(0, 0, 0, 0);
         }
         tc_fence_before();
     }
@@ -518,7 +520,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
     } else {
         // ---------------------------------------------------- compute warpgroups (thread = key)
-        const int quad = warp & 3, hf = warp >> 2;   // TMEM lane quarter; query column half
+        const int quad = warp & 3, hf = warp >> 2;   // TMEM lane quarter; warpgroup
         const int r = quad * 32 + lane;
         const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
         const int j = k0 + r;
@@ -549,8 +551,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 if (a.window >= 0) all_ok = all_ok && k0 >= ibase + 127 + dl - a.window;
             }
 #pragma unroll
-            for (int cc = 0; cc < 2; ++cc) {
-                const int c4 = 2 * hf + cc;
+            for (int cc = 0; cc < 4 / kBwdWG; ++cc) {
+                const int c4 = hf + cc * kBwdWG;
                 uint32_t us[32], ud[32];
                 tmem_ld32(tST + lane_off + c4 * 32, us);
                 tmem_ld32(tdPT + lane_off + c4 * 32, ud);
@@ -600,14 +602,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             tc_fence_after();
         }
         __syncwarp();
-        // warpgroup 0 writes dV, warpgroup 1 dK
-        {
-            const int which = hf;
+        // the 2 D/32 output blocks (dV's, then dK's) go round the warpgroups
+        for (int blk = hf; blk < 2 * (D / 32); blk += kBwdWG) {
+            const int which = blk / (D / 32), c4 = blk % (D / 32);
             const uint32_t tacc = which == 0 ? tdV : tdK;
             __nv_bfloat16* dst = (which == 0 ? a.dv : a.dk) + ((long long)(k_off + j) * a.Hkv + g) * D;
             if (have) {
-#pragma unroll
-                for (int c4 = 0; c4 < D / 32; ++c4) {
+                {
                     uint32_t u[32];
                     tmem_ld32(tacc + lane_off + c4 * 32, u);
                     tmem_wait_ld();
@@ -624,7 +625,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     }
                 }
             } else if (key_ok) {
-                for (int v4 = 0; v4 < D / 8; ++v4) reinterpret_cast<uint4*>(dst)[v4] = make_uint4(0, 0, 0, 0);
+                for (int v4 = 0; v4 < 4; ++v4)
+                    reinterpret_cast<uint4*>(dst + c4 * 32)[v4] = make_uint4(0, 0, 0, 0);
             }
         }
         tc_fence_before();
