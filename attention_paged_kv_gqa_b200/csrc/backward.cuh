@@ -187,7 +187,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = *tmem_slot;
-    const uint32_t tS = tbase, tdP = tbase + 128, tdQ = tbase + 256;
+    // S is double-buffered (tile it in S[it & 1]); dP and the dQ accumulator are single
+    const uint32_t tdP = tbase + 128, tdQ = tbase + 256;
+    auto tSb = [&](int it) { return tbase + ((it & 1) ? 384u : 0u); };
 
     if (warp == kBwdProducerWarp) {
         // ---------------------------------------------------- TMA: Q, dO once; K/V tiles stream
@@ -228,29 +230,54 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         // ---------------------------------------------------- MMA issuer
         if (any_tiles && lane == 0) {
             const uint32_t sQa = smem_u32(sQ), sdOa = smem_u32(sdO), sKa = smem_u32(sK), sVa = smem_u32(sV);
-            bool ok = mbar_wait(q_full, 0, kErrBwdMma);
-            for (int j = lo; ok && j < hi; ++j) {
-                const int it = j - lo, st = it % NS;
-                if (!(ok = mbar_wait(&kv_full[st], (it / NS) & 1, kErrBwdMma))) break;
-                tc_fence_after();
-                // S = Q K^T and dP = dO V^T (both K-major, K = D)
+            // Order per key tile it: S(it+1) into the other S buffer, then (once the compute
+            // warps have turned S(it), dP(it) into dS(it)) dP(it+1), the signal for the next
+            // compute, and dQ += dS(it) K(it) -- so dQ(it) runs beside the next tile's compute.
+            auto issue_s = [&](int it, int st) {       // S = Q K^T (K-major, K = D)
 #pragma unroll
                 for (int kk = 0; kk < D / C::KSTEP; ++kk) {
                     const uint32_t cb = (kk * 32) / 128, off = (kk * 32) % 128;
                     const uint32_t ro = cb * 128 * 128 + off;
-                    mma_f16_ss(tS, smem_desc(sQa + ro, 16, 1024, 2),
+                    mma_f16_ss(tSb(it), smem_desc(sQa + ro, 16, 1024, 2),
                                smem_desc(sKa + st * C::TILE + ro, 16, 1024, 2), C::IDESC_SS, kk > 0);
+                }
+            };
+            auto issue_dp = [&](int st) {              // dP = dO V^T
+#pragma unroll
+                for (int kk = 0; kk < D / C::KSTEP; ++kk) {
+                    const uint32_t cb = (kk * 32) / 128, off = (kk * 32) % 128;
+                    const uint32_t ro = cb * 128 * 128 + off;
                     mma_f16_ss(tdP, smem_desc(sdOa + ro, 16, 1024, 2),
                                smem_desc(sVa + st * C::TILE + ro, 16, 1024, 2), C::IDESC_SS, kk > 0);
                 }
+            };
+            bool ok = mbar_wait(q_full, 0, kErrBwdMma);
+            if (ok) ok = mbar_wait(&kv_full[0], 0, kErrBwdMma);
+            if (ok) {
+                tc_fence_after();
+                issue_s(0, 0);
+                issue_dp(0);
                 mma_commit(s_full);
+            }
+            for (int j = lo; ok && j < hi; ++j) {
+                const int it = j - lo, st = it % NS, st1 = (it + 1) % NS;
+                const bool next = j + 1 < hi;
+                if (next) {
+                    if (!(ok = mbar_wait(&kv_full[st1], ((it + 1) / NS) & 1, kErrBwdMma))) break;
+                    tc_fence_after();
+                    issue_s(it + 1, st1);
+                }
                 if (!(ok = mbar_wait(p_full, it & 1, kErrBwdMma))) break;
                 tc_fence_after();
-                // dQ += dS K: A = dS (bf16 over S in TMEM), B = the key tile read MN-major (K = keys)
+                if (next) {
+                    issue_dp(st1);
+                    mma_commit(s_full);
+                }
+                // dQ += dS K: A = dS (bf16 over S(it) in TMEM), B = the key tile read MN-major (K = keys)
 #pragma unroll
                 for (int kk = 0; kk < 128 / C::KSTEP; ++kk) {
                     const uint64_t db = smem_desc(sKa + st * C::TILE + kk * 2 * 1024, 128 * 128, 1024, 2);
-                    mma_f16_ts(tdQ, tS + bwd_a_col(kk), db, C::IDESC_TS, (it > 0 || kk > 0) ? 1u : 0u);
+                    mma_f16_ts(tdQ, tSb(it) + bwd_a_col(kk), db, C::IDESC_TS, (it > 0 || kk > 0) ? 1u : 0u);
                 }
                 mma_commit(&kv_empty[st]);
             }
@@ -286,7 +313,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             for (int cc = 0; cc < 4 / kBwdWG; ++cc) {
                 const int c4 = hf + cc * kBwdWG;
                 uint32_t us[32], ud[32];
-                tmem_ld32(tS + lane_off + c4 * 32, us);
+                tmem_ld32(tSb(it) + lane_off + c4 * 32, us);
                 tmem_ld32(tdP + lane_off + c4 * 32, ud);
                 tmem_wait_ld();
                 uint32_t pk[16];
@@ -303,7 +330,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     pk[c] = pack_bf16(ds[0], ds[1]);
                 }
                 // dS of block c4 -> columns this warpgroup has already read
-                tmem_st16(tS + lane_off + bwd_out_col(c4), pk);
+                tmem_st16(tSb(it) + lane_off + bwd_out_col(c4), pk);
             }
             tmem_wait_st();
             tc_fence_before();
