@@ -408,27 +408,39 @@ def run_decode(args, A, W, dev, world, flush, peaks, peak_kind, line):
                                            P["max_blocks_per_seq"]) <= 16 else 2
 
     # end to end through the binding with host buffers: q, block_table, seqused_k in
-    # (pinned), O and LSE out; the paged cache is resident device state.
-    qh = t["q"].pin_memory()
-    bth = t["block_table"].pin_memory()
-    suh = t["seqused_k"].pin_memory()
-    oh = torch.empty(o.shape, dtype=o.dtype).pin_memory()
-    lh = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
-    qd, btd, sud = torch.empty_like(d["q"]), torch.empty_like(d["block_table"]), torch.empty_like(d["seqused_k"])
+    # (pinned), O and LSE out; the paged cache is resident device state.  The inputs
+    # travel packed in one pinned buffer (one copy in) and O | LSE come back in one
+    # buffer (one copy out), as a serving loop would stage a step's metadata.
+    def views_of(buf, like):
+        out, off = [], 0
+        for x in like:
+            n = x.numel() * x.element_size()
+            out.append(buf[off:off + n].view(x.dtype).view(x.shape))
+            off += n
+        return out
+
+    ins = [t["q"], t["block_table"], t["seqused_k"]]
+    n_in = sum(x.numel() * x.element_size() for x in ins)
+    hin = torch.empty(n_in, dtype=torch.uint8).pin_memory()
+    for v, x in zip(views_of(hin, ins), ins):
+        v.copy_(x)
+    din = torch.empty(n_in, dtype=torch.uint8, device=dev)
+    qd, btd, sud = views_of(din, ins)
+    dout = torch.empty(o.numel() * o.element_size() + lse.numel() * lse.element_size(),
+                       dtype=torch.uint8, device=dev)
+    od, ld = views_of(dout, [o, lse])
+    hout = torch.empty(dout.numel(), dtype=torch.uint8).pin_memory()
 
     def e2e_step():
-        qd.copy_(qh, non_blocking=True)
-        btd.copy_(bth, non_blocking=True)
-        sud.copy_(suh, non_blocking=True)
-        A.attn_decode_paged(qd, d["k_cache"], d["v_cache"], btd, sud, scale=P["scale"], out=o,
-                            lse=lse, workspace=ws)
-        oh.copy_(o, non_blocking=True)
-        lh.copy_(lse, non_blocking=True)
+        din.copy_(hin, non_blocking=True)
+        A.attn_decode_paged(qd, d["k_cache"], d["v_cache"], btd, sud, scale=P["scale"], out=od,
+                            lse=ld, workspace=ws)
+        hout.copy_(dout, non_blocking=True)
 
     e2e_times = time_steps(e2e_step, args.steps, args.warmup, world, flush)
     e2e_ms = max_over_ranks(sum(e2e_times), world) / args.steps
-    h2d = qh.numel() * 2 + bth.numel() * 4 + suh.numel() * 4
-    d2h = oh.numel() * 2 + lh.numel() * 4
+    h2d = hin.numel()
+    d2h = hout.numel()
 
     line.update({
         "value": round(value, 2), "ms_per_step": round(ms_max, 5),
@@ -451,7 +463,8 @@ def run_decode(args, A, W, dev, world, flush, peaks, peak_kind, line):
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": round(e2e_ms, 5),
                 "note": "paged K/V cache resident on the device; q, block_table, seqused_k "
-                        "copied in and O, LSE copied out every step"},
+                        "copied in (one packed pinned buffer) and O, LSE copied out (one "
+                        "buffer) every step"},
         "gpu_launches": args.steps * ns,
         "clocks": clocks,
     })
