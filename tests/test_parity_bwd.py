@@ -102,3 +102,34 @@ def test_bwd_dense_wrapper_matches_varlen():
     _check(dq, rq, "dense dQ")
     _check(dk, rk, "dense dK")
     _check(dv, rv, "dense dV")
+
+
+def test_bwd_config_varlen_causal_gqa_full():
+    """The bench's backward workload at full size (16 sequences, L ~ U[64,4096], Hq=32, Hkv=8,
+    D=128, causal): the GPU runs the whole batch; the oracle checks every gradient of the
+    shortest sequence and of the fourth shortest (sequences are independent)."""
+    wp = W.FULL_SIZE["varlen_paged_gqa_prefill_causal_bf16"]()
+    lens = wp.tensors["seqused_k"].numpy().astype(np.int64)
+    cu = W.cu_from_lens(lens)
+    total, Hq, Hkv, D, scale = int(cu[-1]), 32, 8, 128, wp.params["scale"]
+    q = W.randn_bf16((total, Hq, D), 0, 51)
+    k = W.randn_bf16((total, Hkv, D), 0, 52)
+    v = W.randn_bf16((total, Hkv, D), 0, 53)
+    do = W.randn_bf16((total, Hq, D), 0, 54)
+    qd, kd, vd, dod, cud = q.to(DEV), k.to(DEV), v.to(DEV), do.to(DEV), cu.to(DEV)
+    maxlen = int(lens.max())
+    o, lse = A.attn_fwd_varlen_paged(qd, kd, vd, cu_seqlens_q=cud, cu_seqlens_k=cud, max_seqlen_q=maxlen,
+                                     mask=A.MASK_CAUSAL, scale=scale)
+    dq, dk, dv = A.attn_bwd_varlen(qd, kd, vd, o, dod, lse, cu_seqlens_q=cud, cu_seqlens_k=cud,
+                                   max_seqlen_q=maxlen, max_seqlen_k=maxlen, mask=A.MASK_CAUSAL, scale=scale)
+    torch.cuda.synchronize()
+    assert A.attn_device_error() == 0
+    order = np.argsort(lens)
+    for b in (int(order[0]), int(order[3])):
+        sl = slice(int(cu[b]), int(cu[b + 1]))
+        c1 = np.array([0, lens[b]], np.int32)
+        rq, rk, rv = oracle.attn_bwd_varlen(q[sl], k[sl], v[sl], do[sl], cu_seqlens_q=c1, cu_seqlens_k=c1,
+                                            num_heads_kv=Hkv, scale=scale, mask=1)
+        _check(dq[sl], rq, "dQ seq %d" % b)
+        _check(dk[sl], rk, "dK seq %d" % b)
+        _check(dv[sl], rv, "dV seq %d" % b)

@@ -185,3 +185,59 @@ def test_decode_only_qv_equals_decode_with_keys_equal_to_values():
     o2, l2 = A.attn_decode_paged(q, v, v, bt, su, scale=0.05)
     torch.cuda.synchronize()
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def _compact(v_cache, bt_row, n_keys):
+    """The pages one sequence uses, as a small pool with its own (identity) block table."""
+    n = (int(n_keys) + 15) // 16
+    return v_cache[bt_row[:n].long()], torch.arange(n, dtype=torch.int32)[None]
+
+
+def test_config_only_qv_decode_full():
+    """only_qv paged decode at the bench's size: B=32, Hq=32, Hkv=8, D=128, L ~ U[1,8192],
+    20000-page pool, automatic splits (sampled sequences)."""
+    w = W.FULL_SIZE["paged_gqa_decode_bf16"]()
+    t = w.tensors
+    o, lse = A.attn_decode_paged_only_qv(t["q"].to(DEV), t["v_cache"].to(DEV), t["block_table"].to(DEV),
+                                         t["seqused_k"].to(DEV), scale=w.params["scale"])
+    torch.cuda.synchronize()
+    assert A.attn_device_error() == 0
+    lens = t["seqused_k"].numpy()
+    sample = sorted(set([int(np.argmax(lens)), int(np.argmin(lens))] +
+                        list(np.random.default_rng(2).choice(len(lens), 5, replace=False))))
+    for b in sample:
+        vc, bt = _compact(t["v_cache"], t["block_table"][b], lens[b])
+        o_ref, lse_ref = oracle.attn_varlen_qv(None, t["q"][b:b + 1], None, vc, cu_seqlens_q=[0, 1],
+                                               block_table=bt, seqused_k=[int(lens[b])], num_heads_kv=8,
+                                               scale=w.params["scale"], mask=0, only_qv=True)
+        _cmp(o[b:b + 1], lse[b:b + 1].T.contiguous(), o_ref, lse_ref, TOL_O_BF16, TOL_LSE_BF16,
+             "only_qv decode b%d" % b)
+
+
+def test_config_only_qv_prefill_full():
+    """only_qv varlen paged causal prefill at the bench's size (sampled rows: row i of a
+    sequence is unmasked only_qv attention over its keys 0..i)."""
+    w = W.FULL_SIZE["varlen_paged_gqa_prefill_causal_bf16"]()
+    t = w.tensors
+    o, lse = A.attn_fwd_varlen_paged_only_qv(t["q"].to(DEV), t["v_cache"].to(DEV),
+                                             cu_seqlens_q=t["cu_seqlens_q"].to(DEV),
+                                             max_seqlen_q=w.params["max_seqlen_q"],
+                                             block_table=t["block_table"].to(DEV),
+                                             seqused_k=t["seqused_k"].to(DEV), mask=A.MASK_CAUSAL,
+                                             scale=w.params["scale"])
+    torch.cuda.synchronize()
+    assert A.attn_device_error() == 0
+    o = o.float().cpu().numpy()
+    lse = lse.cpu().numpy()
+    cu = t["cu_seqlens_q"].numpy()
+    rng = np.random.default_rng(3)
+    for b in range(0, 16, 3):
+        L = cu[b + 1] - cu[b]
+        for i in sorted(set([0, L - 1, int(rng.integers(0, L)), min(128, L - 1)])):
+            r = cu[b] + i
+            vc, bt = _compact(t["v_cache"], t["block_table"][b], i + 1)
+            o_ref, lse_ref = oracle.attn_varlen_qv(None, t["q"][r:r + 1], None, vc, cu_seqlens_q=[0, 1],
+                                                   block_table=bt, seqused_k=[i + 1], num_heads_kv=8,
+                                                   scale=w.params["scale"], mask=0, only_qv=True)
+            assert np.max(np.abs(o[r] - o_ref[0])) <= TOL_O_BF16, (b, i)
+            assert np.max(np.abs(lse[:, r] - lse_ref[:, 0])) <= TOL_LSE_BF16, (b, i)
