@@ -61,6 +61,8 @@ def lib():
         L.attn_decode_paged_only_qv.argtypes = [P, P, P, I, I, I, P, I, I, I, I, F, I, F, I, I, P, P,
                                                 P, Z, P]
         L.attn_decode_paged_only_qv.restype = I
+        L.attn_fwd_patch.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, F, I, I, P, P, P, P, P, P]
+        L.attn_fwd_patch.restype = I
         L.attn_decode_workspace_size.argtypes = [I, I, I, I, I, I, I]
         L.attn_decode_workspace_size.restype = Z
         L.attn_decode_paged.argtypes = [P, P, P, P, I, I, I, P, I, I, I, I, F, I, F, I, I, P, P,
@@ -221,6 +223,26 @@ def attn_fwd_varlen_paged_only_qv(qv, v_cache, *, cu_seqlens_q, max_seqlen_q, bl
         int(window_left), float(softcap), _dtype_code(qv), _ptr(descale_qv), _ptr(descale_v),
         _ptr(out), _ptr(lse), _stream(stream))
     _check(st, "attn_fwd_varlen_paged_only_qv")
+    return out, lse
+
+
+def attn_fwd_patch(q, k, v, *, cu_seqlens_q, cu_seqlens_k, patch_kv_range, max_seqlen_q,
+                   max_interval, scale=None, descale_q=None, descale_k=None, descale_v=None,
+                   out=None, lse=None, return_lse=True, stream=None):
+    """Patch cross-attention with intervals of at most max_interval keys (see the header):
+    q [total_q, Hq, D], packed k/v [total_k, Hkv, D] -> (o, lse [Hq, total_q])."""
+    total_q, Hq, D = q.shape
+    total_k, Hkv = k.shape[0], k.shape[1]
+    B = cu_seqlens_q.numel() - 1
+    if out is None:
+        out = torch.empty((total_q, Hq, D), dtype=torch.bfloat16, device=q.device)
+    if lse is None and return_lse:
+        lse = torch.empty((Hq, total_q), dtype=torch.float32, device=q.device)
+    st = lib().attn_fwd_patch(_ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens_q), _ptr(cu_seqlens_k),
+                              _ptr(patch_kv_range), B, total_q, total_k, int(max_seqlen_q), Hq, Hkv, D,
+                              _scale(scale), int(max_interval), _dtype_code(q), _ptr(descale_q),
+                              _ptr(descale_k), _ptr(descale_v), _ptr(out), _ptr(lse), _stream(stream))
+    _check(st, "attn_fwd_patch")
     return out, lse
 
 

@@ -20,6 +20,7 @@
 
 #include "attn_b200.h"
 #include "decode.cuh"
+#include "patch.cuh"
 #include "prefill.cuh"
 #include "append.cuh"
 #include "backward.cuh"
@@ -713,6 +714,68 @@ attn_status_t attn_fwd_varlen_paged_only_qv(
                                  total_k, max_seqlen_q, Hq, Hkv, D, softmax_scale, mask,
                                  patch_kv_range, window_left, softcap, dtype, descale_qv, descale_v,
                                  descale_v, o, lse, stream, 1);
+}
+
+attn_status_t attn_fwd_patch(const void* q, const void* k, const void* v,
+                             const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                             const int32_t* patch_kv_range, int B, int total_q, int total_k,
+                             int max_seqlen_q, int Hq, int Hkv, int D, float softmax_scale,
+                             int max_interval, int dtype, const float* dq, const float* dk,
+                             const float* dv, void* o, float* lse, attn_stream_t stream) {
+    if (max_interval < 0) return ATTN_ERR_INVALID_ARG;
+    // Long intervals, or fp8: the tiled tensor-core kernel with the patch mask.
+    if (max_interval > kPatchShortMax || dtype != ATTN_BF16)
+        return fwd_varlen_paged_impl(q, k, v, nullptr, 0, 0, 0, cu_seqlens_q, cu_seqlens_k, nullptr, B,
+                                     total_q, total_k, max_seqlen_q, Hq, Hkv, D, softmax_scale,
+                                     ATTN_MASK_PATCH, patch_kv_range, -1, 0.0f, dtype, dq, dk, dv, o,
+                                     lse, stream, 0);
+    if (!q || !k || !v || !o || !cu_seqlens_q || !cu_seqlens_k || !patch_kv_range) return ATTN_ERR_INVALID_ARG;
+    if (B < 0 || total_q < 0 || total_k < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0)
+        return ATTN_ERR_INVALID_ARG;
+    if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return ATTN_ERR_INVALID_ARG;
+    int dev = 0;
+    const attn_status_t dvs = current_device_ok(&dev);
+    if (dvs != ATTN_OK) return dvs;
+    if (B == 0 || total_q == 0) return ATTN_OK;
+    PatchArgs pa;
+    std::memset(&pa, 0, sizeof(pa));
+    pa.q = static_cast<const __nv_bfloat16*>(q);
+    pa.k = static_cast<const __nv_bfloat16*>(k);
+    pa.v = static_cast<const __nv_bfloat16*>(v);
+    pa.cu_q = cu_seqlens_q;
+    pa.cu_k = cu_seqlens_k;
+    pa.range = patch_kv_range;
+    pa.B = B;
+    pa.Hq = Hq;
+    pa.Hkv = Hkv;
+    pa.group = Hq / Hkv;
+    pa.total_q = total_q;
+    pa.scale = resolve_scale(softmax_scale, D);
+    pa.o = static_cast<__nv_bfloat16*>(o);
+    pa.lse = lse;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // a warp per query (all heads) where a lane's share of the heads' columns is small;
+    // otherwise a warp per (query, head)
+    const long long qblocks = std::min<long long>((total_q + kPatchWarps - 1) / kPatchWarps,
+                                                  (long long)sm_count(dev) * 16);
+    if (Hq == 16 && D == 64) {
+        patch_query_kernel<64, 16><<<(unsigned)qblocks, 32 * kPatchWarps, 0, st>>>(pa);
+        return launch_status();
+    }
+    if (Hq == 8 && D == 128) {
+        patch_query_kernel<128, 8><<<(unsigned)qblocks, 32 * kPatchWarps, 0, st>>>(pa);
+        return launch_status();
+    }
+    if (Hq == 8 && D == 64) {
+        patch_query_kernel<64, 8><<<(unsigned)qblocks, 32 * kPatchWarps, 0, st>>>(pa);
+        return launch_status();
+    }
+    const long long items = (long long)total_q * Hq;
+    const long long blocks = std::min<long long>((items + kPatchWarps - 1) / kPatchWarps, (long long)sm_count(dev) * 8);
+    if (D == 128) patch_kernel<128><<<(unsigned)blocks, 32 * kPatchWarps, 0, st>>>(pa);
+    else patch_kernel<64><<<(unsigned)blocks, 32 * kPatchWarps, 0, st>>>(pa);
+    return launch_status();
 }
 
 // Split-KV heuristic: enough CTAs to fill every SM about twice with sequences

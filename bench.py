@@ -85,7 +85,7 @@ def parse_args():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--no-prefill", action="store_true")
     p.add_argument("--workload", choices=["all", "decode", "prefill", "fp8", "window", "append",
-                                          "backward", "only_qv"],
+                                          "backward", "only_qv", "patch"],
                    default="all",
                    help="run only one workload (profiling runs); the JSON line then carries "
                         "only what ran")
@@ -374,6 +374,8 @@ def run_ours(args, rank, world, local):
         run_backward(args, A, W, dev, world, flush, peaks, peak_kind, line)
     if args.workload in ("all", "only_qv") and not args.no_prefill:
         run_only_qv(args, A, W, dev, world, flush, peaks, peak_kind, line)
+    if args.workload in ("all", "patch") and not args.no_prefill:
+        run_patch_and_small(args, A, W, dev, world, flush, peaks, peak_kind, line)
     if args.workload in ("all", "decode") and rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
     if rank == 0:
@@ -771,6 +773,65 @@ def run_only_qv(args, A, W, dev, world, flush, peaks, peak_kind, line):
                         "above with the query tensor as qv and the value cache as the only "
                         "KV store; decode bytes count V once (no K stream)")
     line["only_qv"] = out
+
+
+def run_patch_and_small(args, A, W, dev, world, flush, peaks, peak_kind, line):
+    """The two remaining configurations: patch cross-attention (memory-bound: GB/s against
+    HBM) and the small dense causal case (launch-latency bound: microseconds per call)."""
+    w = W.patch_cross(seed=args.seed)
+    t, P = w.tensors, w.params
+    d = {k: v.to(dev) for k, v in t.items()}
+    o = torch.empty(P["total_q"], P["Hq"], P["D"], dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(P["Hq"], P["total_q"], dtype=torch.float32, device=dev)
+
+    def patch_step():   # patches are clipped to 16 bytes: the short-interval kernel
+        A.attn_fwd_patch(d["q"], d["k"], d["v"], cu_seqlens_q=d["cu_seqlens_q"],
+                         cu_seqlens_k=d["cu_seqlens_k"], patch_kv_range=d["patch_kv_range"],
+                         max_seqlen_q=P["max_seqlen_q"], max_interval=16, scale=P["scale"], out=o,
+                         lse=lse)
+
+    def patch_tiled_step():
+        A.attn_fwd_varlen_paged(d["q"], d["k"], d["v"], cu_seqlens_q=d["cu_seqlens_q"],
+                                cu_seqlens_k=d["cu_seqlens_k"], max_seqlen_q=P["max_seqlen_q"],
+                                mask=A.MASK_PATCH, patch_kv_range=d["patch_kv_range"],
+                                scale=P["scale"], out=o, lse=lse)
+
+    pms = statistics.mean(time_steps(patch_step, args.steps, args.warmup, world, flush))
+    tms = statistics.mean(time_steps(patch_tiled_step, args.steps, args.warmup, world, flush))
+    # algorithmic bytes: every key and value row once (each belongs to one patch), Q and O,
+    # LSE, the per-query ranges and the cumulative lengths
+    nb = (2 * P["total_k"] * P["Hkv"] * P["D"] * 2 + 2 * P["total_q"] * P["Hq"] * P["D"] * 2
+          + P["total_q"] * P["Hq"] * 4 + P["total_q"] * 8 + 2 * (P["B"] + 1) * 4)
+    gbs = nb / (pms * 1e-3) / 1e9
+    out = {"patch": {"workload": "patch cross-attention bf16: B=4 x 8192 byte keys, Geometric(0.22) "
+                                 "patches clipped to [1,16] (seed %d: %d queries), H=16, D=64, "
+                                 "packed K/V" % (args.seed, P["total_q"]),
+                     "value": round(gbs, 2), "unit": "GB/s", "ms_per_step": round(pms, 5),
+                     "bytes_per_step": nb,
+                     "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"],
+                                  "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4),
+                                  "traffic": None, "kernel": "patch_query_kernel<64, 16> (attn_fwd_patch, "
+                                                              "max_interval 16)",
+                                  "peak_kind": peak_kind},
+                     "tiled_kernel": {"value": round(nb / (tms * 1e-3) / 1e9, 2), "unit": "GB/s",
+                                      "ms_per_step": round(tms, 5),
+                                      "note": "the same call through attn_fwd_varlen_paged "
+                                              "(tensor-core tiles with the patch mask)"}}}
+    del d
+    w1 = W.dense(seed=args.seed)
+    t1 = {k: v.to(dev) for k, v in w1.tensors.items()}
+    o1 = torch.empty_like(t1["q"])
+    l1 = torch.empty(2, 2, 128, dtype=torch.float32, device=dev)
+
+    def small_step():
+        A.attn_fwd_dense(t1["q"], t1["k"], t1["v"], causal=True, scale=w1.params["scale"], out=o1, lse=l1)
+
+    sms = statistics.mean(time_steps(small_step, args.steps, args.warmup, world, flush))
+    out["dense_small"] = {"workload": "dense causal bf16: B=2, Hq=Hkv=2, L=128, D=64",
+                          "value": round(sms * 1e3, 2), "unit": "us per call",
+                          "higher_is_better": False,
+                          "note": "8.45 MFLOP: launch- and latency-bound, no roofline"}
+    line["other_configs"] = out
 
 
 def cpu_baseline(w):

@@ -165,6 +165,30 @@ attn_status_t attn_fwd_varlen_paged(
     void *o, float *lse, void *workspace, size_t workspace_bytes, attn_stream_t stream);
 
 /*
+ * Patch-to-byte cross-attention (the patch mask of attn_fwd_varlen_paged) for
+ * intervals the caller knows to be short, as in the byte-latent model of "Cross
+ * Attention does not work on CPU and older GPUs" (one query per patch, each
+ * attending to its own patch's bytes; patches of at most 16 bytes).  Query i of
+ * sequence b sees the keys [patch_kv_range[i][0], patch_kv_range[i][1]) of its
+ * sequence (clamped to [0, Lk_b)); O and LSE as in attn_fwd_varlen_paged, an
+ * empty interval giving O = 0 and LSE = -inf.
+ *   q [total_q, Hq, D], k/v packed [total_k, Hkv, D], cu_seqlens_q/k int32 [B+1],
+ *   patch_kv_range int32 [total_q, 2], o [total_q, Hq, D] bf16, lse [Hq, total_q] or NULL.
+ *   max_interval  the caller's bound on end - start over all queries.  It only
+ *                 chooses the kernel, never the result: up to 64 (bf16) a CUDA-core
+ *                 kernel reads each key and value row once per query head (one
+ *                 warp per query and head); above that, or for fp8, the tiled
+ *                 tensor-core kernel of attn_fwd_varlen_paged runs.
+ * Supported: head_dim in {64, 128}.
+ */
+attn_status_t attn_fwd_patch(
+    const void *q, const void *k, const void *v, const int32_t *cu_seqlens_q,
+    const int32_t *cu_seqlens_k, const int32_t *patch_kv_range, int B, int total_q, int total_k,
+    int max_seqlen_q, int num_heads_q, int num_heads_kv, int head_dim, float softmax_scale,
+    int max_interval, int dtype, const float *descale_q, const float *descale_k,
+    const float *descale_v, void *o, float *lse, attn_stream_t stream);
+
+/*
  * The only_qv score path of "Rope dim" (vllm-project flash-attention PR 172,
  * overview: the mode that skips the Q and K loads and the QK GEMM and
  * zero-initialises the score with the Qv GEMM).  The score of query i and key

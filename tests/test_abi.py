@@ -151,3 +151,17 @@ def test_only_qv_entry_points_check_arguments(L):
     st = L.attn_decode_paged_only_qv(p, p, p, 4, 100, 16, None, 1, 8, 2, 128, 0.0, -1, 0.0, 1, 0,
                                      p, None, p, 1 << 20, None)
     assert st == 1
+
+
+def test_patch_entry_point_checks_arguments(L):
+    p = ctypes.c_void_p(1 << 20)
+    # negative interval bound; missing ranges; head_dim 96
+    st = L.attn_fwd_patch(p, p, p, p, p, p, 1, 16, 16, 16, 2, 2, 64, 0.0, -1, 0, None, None, None,
+                          p, None, None)
+    assert st == 1
+    st = L.attn_fwd_patch(p, p, p, p, p, None, 1, 16, 16, 16, 2, 2, 64, 0.0, 16, 0, None, None, None,
+                          p, None, None)
+    assert st == 1
+    st = L.attn_fwd_patch(p, p, p, p, p, p, 1, 16, 16, 16, 2, 2, 96, 0.0, 16, 0, None, None, None,
+                          p, None, None)
+    assert st == 2
