@@ -565,7 +565,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                 m_run = m_new;
             }
             const float mu = (m_run == -INFINITY) ? 0.0f : m_run;
-            float sums[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+            // x = s * sl2 - mu two lanes at a time (packed f32x2 FMA), and for fp8
+            // the row sums too.
+            const float2 sl2x2 = make_float2(sl2, sl2), nmu2 = make_float2(-mu, -mu);
+            float2 sums2[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
             __syncwarp();
             // P overwrites the first columns of S in TMEM, 32 keys at a time.
 #pragma unroll
@@ -574,14 +577,15 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                     uint32_t pk[8];
 #pragma unroll
                     for (int c = 0; c < 8; ++c) {
-                        const float p0 = row_exp2<FP8>(4 * c + 0, fmaf(s[c4 * 32 + 4 * c + 0], sl2, -mu));
-                        const float p1 = row_exp2<FP8>(4 * c + 1, fmaf(s[c4 * 32 + 4 * c + 1], sl2, -mu));
-                        const float p2 = row_exp2<FP8>(4 * c + 2, fmaf(s[c4 * 32 + 4 * c + 2], sl2, -mu));
-                        const float p3 = row_exp2<FP8>(4 * c + 3, fmaf(s[c4 * 32 + 4 * c + 3], sl2, -mu));
-                        sums[0] += p0;
-                        sums[1] += p1;
-                        sums[2] += p2;
-                        sums[3] += p3;
+                        const float* sc = &s[c4 * 32 + 4 * c];
+                        const float2 x01 = ffma2(make_float2(sc[0], sc[1]), sl2x2, nmu2);
+                        const float2 x23 = ffma2(make_float2(sc[2], sc[3]), sl2x2, nmu2);
+                        const float p0 = row_exp2<FP8>(4 * c + 0, x01.x);
+                        const float p1 = row_exp2<FP8>(4 * c + 1, x01.y);
+                        const float p2 = row_exp2<FP8>(4 * c + 2, x23.x);
+                        const float p3 = row_exp2<FP8>(4 * c + 3, x23.y);
+                        sums2[0] = fadd2(sums2[0], make_float2(p0, p1));
+                        sums2[1] = fadd2(sums2[1], make_float2(p2, p3));
                         pk[c] = pack_e4m3x4(p0, p1, p2, p3);
                     }
                     tmem_st8(tS + c4 * 8, pk);
@@ -589,20 +593,23 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                     uint32_t pk[16];
 #pragma unroll
                     for (int c = 0; c < 16; ++c) {
-                        const float p0 = row_exp2<FP8>(2 * c + 0, fmaf(s[c4 * 32 + 2 * c + 0], sl2, -mu));
-                        const float p1 = row_exp2<FP8>(2 * c + 1, fmaf(s[c4 * 32 + 2 * c + 1], sl2, -mu));
-                        sums[(2 * c) & 3] += p0;
-                        sums[(2 * c + 1) & 3] += p1;
+                        const float2 x = ffma2(make_float2(s[c4 * 32 + 2 * c], s[c4 * 32 + 2 * c + 1]), sl2x2, nmu2);
+                        const float p0 = row_exp2<FP8>(2 * c + 0, x.x);
+                        const float p1 = row_exp2<FP8>(2 * c + 1, x.y);
+                        sums2[c & 1].x += p0;      // (packed adds here cost registers: spills)
+                        sums2[c & 1].y += p1;
                         pk[c] = pack_bf16(p0, p1);
                     }
                     tmem_st16(tS + c4 * 16, pk);
                 }
             }
-            const float sum = (sums[0] + sums[1]) + (sums[2] + sums[3]);
+            const float sum = (sums2[0].x + sums2[0].y) + (sums2[1].x + sums2[1].y);
             if (jj > 0 && __any_sync(0xffffffffu, want)) {
                 // O holds the sum over earlier tiles (their P.V MMAs completed
-                // before this tile's S was committed); rescale this row.
-#pragma unroll
+                // before this tile's S was committed); rescale this row.  Rare
+                // (only when the row max grows past the threshold), so the loop
+                // stays rolled to keep register pressure down.
+#pragma unroll 1
                 for (int c4 = 0; c4 < D / 32; ++c4) {
                     uint32_t u[32];
                     tmem_ld32(tO + c4 * 32, u);
