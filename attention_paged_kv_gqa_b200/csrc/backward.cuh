@@ -317,17 +317,22 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 tmem_ld32(tdP + lane_off + c4 * 32, ud);
                 tmem_wait_ld();
                 uint32_t pk[16];
+                // two columns per packed f32x2 instruction
+                const float2 sl2x2 = make_float2(sl2, sl2), nlse2 = make_float2(-lse2, -lse2);
+                const float2 ndlt2 = make_float2(-dlt, -dlt), scale2 = make_float2(a.scale, a.scale);
 #pragma unroll
                 for (int c = 0; c < 16; ++c) {
-                    float ds[2];
-#pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        const int kv = kbase + c4 * 32 + 2 * c + e;
-                        float p = ex2(fmaf(__uint_as_float(us[2 * c + e]), sl2, -lse2));
-                        if (partial && (kv < klo || kv >= khi)) p = 0.0f;
-                        ds[e] = p * (__uint_as_float(ud[2 * c + e]) - dlt) * a.scale;
+                    const float2 x = ffma2(make_float2(__uint_as_float(us[2 * c]), __uint_as_float(us[2 * c + 1])),
+                                           sl2x2, nlse2);
+                    float2 p = make_float2(ex2(x.x), ex2(x.y));
+                    if (partial) {
+                        const int kv = kbase + c4 * 32 + 2 * c;
+                        if (kv < klo || kv >= khi) p.x = 0.0f;
+                        if (kv + 1 < klo || kv + 1 >= khi) p.y = 0.0f;
                     }
-                    pk[c] = pack_bf16(ds[0], ds[1]);
+                    const float2 dp = fadd2(make_float2(__uint_as_float(ud[2 * c]), __uint_as_float(ud[2 * c + 1])), ndlt2);
+                    const float2 ds = fmul2(p, fmul2(dp, scale2));
+                    pk[c] = pack_bf16(ds.x, ds.y);
                 }
                 // dS of block c4 -> columns this warpgroup has already read
                 tmem_st16(tSb(it) + lane_off + bwd_out_col(c4), pk);
@@ -592,27 +597,28 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                         lv = reinterpret_cast<const float4*>(sL + c4 * 32)[c / 2];
                         dv = reinterpret_cast<const float4*>(sDl + c4 * 32)[c / 2];
                     }
-                    const float l4[4] = {lv.x, lv.y, lv.z, lv.w};
-                    const float d4[4] = {dv.x, dv.y, dv.z, dv.w};
-                    float p2[2], ds2[2];
+                    // columns 2c, 2c+1 are rows with LSE / Delta at lanes (2c & 3), (2c & 3) + 1 of lv / dv
+                    const float2 nl = (c & 1) ? make_float2(-lv.z, -lv.w) : make_float2(-lv.x, -lv.y);
+                    const float2 nd = (c & 1) ? make_float2(-dv.z, -dv.w) : make_float2(-dv.x, -dv.y);
+                    const float2 x = ffma2(make_float2(__uint_as_float(us[2 * c]), __uint_as_float(us[2 * c + 1])),
+                                           make_float2(sl2, sl2), nl);
+                    float2 p = make_float2(ex2(x.x), ex2(x.y));
+                    if (!all_ok) {
 #pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        const int col = 2 * c + e;
-                        const int i = ibase + c4 * 32 + col;
-                        float p = ex2(fmaf(__uint_as_float(us[col]), sl2, -l4[col & 3]));
-                        if (!all_ok) {
+                        for (int e = 0; e < 2; ++e) {
+                            const int i = ibase + c4 * 32 + 2 * c + e;
                             bool allowed = key_ok;
                             if (causal) {
                                 allowed = allowed && j <= i + dl;
                                 if (a.window >= 0) allowed = allowed && j >= i + dl - a.window;
                             }
-                            if (!allowed) p = 0.0f;
+                            if (!allowed) (e == 0 ? p.x : p.y) = 0.0f;
                         }
-                        p2[e] = p;
-                        ds2[e] = p * (__uint_as_float(ud[col]) - d4[col & 3]) * a.scale;
                     }
-                    pp[c] = pack_bf16(p2[0], p2[1]);
-                    dd[c] = pack_bf16(ds2[0], ds2[1]);
+                    const float2 dp = fadd2(make_float2(__uint_as_float(ud[2 * c]), __uint_as_float(ud[2 * c + 1])), nd);
+                    const float2 ds = fmul2(p, fmul2(dp, make_float2(a.scale, a.scale)));
+                    pp[c] = pack_bf16(p.x, p.y);
+                    dd[c] = pack_bf16(ds.x, ds.y);
                 }
                 // block c4 -> columns this warpgroup has already read
                 tmem_st16(tST + lane_off + bwd_out_col(c4), pp);

@@ -434,8 +434,6 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             }
             for (int j = lo; ok && j < hi; ++j) {
                 const int it = j - lo;
-                const int st = it % NS;
-                const uint32_t ph = (it / NS) & 1;
                 const int st1 = (it + 1) % NS;
                 const uint32_t ph1 = ((it + 1) / NS) & 1;
                 const int vst = it % vring, vst1 = (it + 1) % vring;
@@ -533,8 +531,13 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                 for (int c = 0; c < kBN; ++c) s[c] = __uint_as_float(u[c]);
             }
             if constexpr (CAP) {
+                const float kin2 = cap_in * 2.88539008177792681f;   // 2 log2(e) k_in
 #pragma unroll
-                for (int c = 0; c < kBN; ++c) s[c] = softcap_raw(s[c], cap_in, cap_out);
+                for (int c = 0; c < kBN; c += 2) {
+                    const float2 v = softcap_raw2(make_float2(s[c], s[c + 1]), kin2, cap_out);
+                    s[c] = v.x;
+                    s[c + 1] = v.y;
+                }
             }
             const int kbase = j * kBN;
             if (kbase < klo || kbase + kBN > khi) {
@@ -566,7 +569,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             }
             const float mu = (m_run == -INFINITY) ? 0.0f : m_run;
             // x = s * sl2 - mu two lanes at a time (packed f32x2 FMA), and for fp8
-            // the row sums too.
+            // without softcap the row sums too.
             const float2 sl2x2 = make_float2(sl2, sl2), nmu2 = make_float2(-mu, -mu);
             float2 sums2[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
             __syncwarp();
@@ -584,8 +587,15 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                         const float p1 = row_exp2<FP8>(4 * c + 1, x01.y);
                         const float p2 = row_exp2<FP8>(4 * c + 2, x23.x);
                         const float p3 = row_exp2<FP8>(4 * c + 3, x23.y);
-                        sums2[0] = fadd2(sums2[0], make_float2(p0, p1));
-                        sums2[1] = fadd2(sums2[1], make_float2(p2, p3));
+                        if constexpr (CAP) {   // (packed adds here cost registers with the softcap)
+                            sums2[0].x += p0;
+                            sums2[0].y += p1;
+                            sums2[1].x += p2;
+                            sums2[1].y += p3;
+                        } else {
+                            sums2[0] = fadd2(sums2[0], make_float2(p0, p1));
+                            sums2[1] = fadd2(sums2[1], make_float2(p2, p3));
+                        }
                         pk[c] = pack_e4m3x4(p0, p1, p2, p3);
                     }
                     tmem_st8(tS + c4 * 8, pk);

@@ -333,6 +333,34 @@ __device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
     return d;
 }
 
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\t"
+        "mov.b64 rb, {%4, %5};\n\t"
+        "mul.rn.f32x2 rd, ra, rb;\n\t"
+        "mov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+
+__device__ __forceinline__ float rcp_approx(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// softcap_raw on two raw scores: k_out * tanh(k_in * qk) as
+// k_out - 2 k_out / (2^(2 log2(e) k_in qk) + 1), kin2 = 2 log2(e) k_in (the same
+// formula and error as tanh_ex2; 2^x overflowing to inf gives k_out).
+__device__ __forceinline__ float2 softcap_raw2(float2 qk, float kin2, float k_out) {
+    // (only the last step is packed: packing the first two costs registers)
+    const float r0 = rcp_approx(ex2(qk.x * kin2) + 1.0f);
+    const float r1 = rcp_approx(ex2(qk.y * kin2) + 1.0f);
+    return ffma2(make_float2(r0, r1), make_float2(-2.0f * k_out, -2.0f * k_out), make_float2(k_out, k_out));
+}
+
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
     float r;
     asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
