@@ -47,6 +47,8 @@ def lib():
         L.attn_status_string.restype = ctypes.c_char_p
         L.attn_device_error.argtypes = [ctypes.POINTER(I), P]
         L.attn_device_error.restype = I
+        L.attn_selftest_wait_expiry.argtypes = [ctypes.c_longlong, P]
+        L.attn_selftest_wait_expiry.restype = I
         L.attn_selftest_exp2.argtypes = [P, P, I, I, P]
         L.attn_selftest_exp2.restype = I
         L.attn_fwd_dense.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P, P, P, F, I, I, F, I,
@@ -133,6 +135,12 @@ def attn_device_error(stream=None) -> int:
     if st not in (0, 7):
         _check(st, "attn_device_error")
     return code.value
+
+
+def attn_selftest_wait_expiry(limit_ns: int, stream=None):
+    """Launches the bounded-wait test kernel (a wait nothing satisfies, limited to limit_ns)."""
+    _check(lib().attn_selftest_wait_expiry(int(limit_ns), _stream(stream)),
+           "attn_selftest_wait_expiry")
 
 
 def attn_selftest_exp2(x, degree=3, stream=None):

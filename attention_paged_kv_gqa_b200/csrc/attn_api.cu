@@ -350,6 +350,21 @@ __global__ void exp2_selftest_kernel(const float* __restrict__ x, float* __restr
     if (i < n) y[i] = degree >= 3 ? exp2_fma<3>(x[i]) : exp2_fma<2>(x[i]);
 }
 
+// One CTA waits on an mbarrier that nothing ever arrives on, bounded by
+// limit_ns: the wait expires, records kErrSelftestWait in the device error word
+// and the kernel returns (the failure-detection path of every kernel here,
+// made to run out on purpose).
+__global__ void wait_expiry_kernel(unsigned long long limit_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) mbar_wait_for(&bar, 0, kErrSelftestWait, limit_ns);
+    __syncthreads();
+}
+
 // ------------------------------------------------------------------ allocation-free decode
 // Fixed device scratch for attn_decode_paged_noalloc.  Every device that loads
 // this library holds these bytes until the process exits.  Host code must not
@@ -496,6 +511,15 @@ attn_status_t attn_device_error(int* code_out, attn_stream_t stream) {
     }
     *code_out = host;
     return host == 0 ? ATTN_OK : ATTN_ERR_DEVICE_TIMEOUT;
+}
+
+attn_status_t attn_selftest_wait_expiry(long long limit_ns, attn_stream_t stream) {
+    if (limit_ns < 0 || limit_ns > 10000000000LL) return ATTN_ERR_INVALID_ARG;
+    const attn_status_t dvs = current_device_ok(nullptr);
+    if (dvs != ATTN_OK) return dvs;
+    wait_expiry_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<unsigned long long>(limit_ns));
+    return launch_status();
 }
 
 attn_status_t attn_selftest_exp2(const float* x, float* y, int n, int degree, attn_stream_t stream) {
@@ -1181,12 +1205,26 @@ attn_status_t attn_decode_paged_noalloc(const void* q, const void* k_cache, cons
                                         int num_blocks, int block_size, const int32_t* seqused_k,
                                         int B, int Hq, int Hkv, int D, float softmax_scale, int dtype,
                                         void* o, float* lse, attn_stream_t stream) {
-    // Arguments that the shared path would reject are reported by it; here only
-    // what decides whether the fixed scratch can serve the request.
-    if (B < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || Hq % Hkv != 0 || max_blocks_per_seq <= 0 ||
-        block_size <= 0)
+    // The argument checks of attn_decode_paged, in its order, so that a bad call
+    // gets the same status from both entry points; then what decides whether the
+    // fixed scratch can serve the request.
+    if (!q || !k_cache || !v_cache || !block_table || !seqused_k || !o) return ATTN_ERR_INVALID_ARG;
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
+    if (num_blocks <= 0 || max_blocks_per_seq <= 0) return ATTN_ERR_INVALID_ARG;
+    if (!dtype_ok(dtype)) return ATTN_ERR_INVALID_ARG;
+    if (dtype != ATTN_BF16) return ATTN_ERR_UNSUPPORTED;
+    if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+    if (block_size != kPageRows) return ATTN_ERR_UNSUPPORTED;
+    if (Hq / Hkv > kDecRows) return ATTN_ERR_UNSUPPORTED;
+    if (B > kDecMaxSeqs) return ATTN_ERR_UNSUPPORTED;
+    if ((long long)num_blocks * block_size >= (1LL << 31)) return ATTN_ERR_UNSUPPORTED;
+    if ((long long)max_blocks_per_seq * block_size >= (1LL << 30)) return ATTN_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o))
         return ATTN_ERR_INVALID_ARG;
-    if (B == 0) return ATTN_OK;
+    if (B == 0) {
+        const attn_status_t dv0 = current_device_ok(nullptr);
+        return dv0;
+    }
     if (!use_page_stream(B, Hq, Hkv, D, 0)) return ATTN_ERR_UNSUPPORTED;
     int dev = 0;
     const attn_status_t dvs = current_device_ok(&dev);

@@ -62,6 +62,7 @@ enum : int {
     kErrMmaQ = 201, kErrMmaK = 202, kErrMmaV = 203, kErrMmaP = 204, kErrMmaDone = 205,
     kErrSmS = 301, kErrSmV = 302, kErrSmO = 303,
     kErrDecFull = 401, kErrDecEmpty = 402,
+    kErrSelftestWait = 901,
 };
 
 struct PrefillArgs {

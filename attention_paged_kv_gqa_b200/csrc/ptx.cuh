@@ -74,8 +74,12 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Waits until the phase with the given parity has completed.  Bounded.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int code) {
+// Waits until the phase with the given parity has completed, for at most
+// limit_ns of wall time: on expiry it records `code` in the device error word
+// and returns false; it also returns false early once another CTA has
+// recorded an error.
+__device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity, int code,
+                                              uint64_t limit_ns) {
     const uint32_t a = smem_u32(bar);
     if (mbar_try_wait(a, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
@@ -84,12 +88,17 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int co
         if (mbar_try_wait(a, parity)) return true;
         if ((++spins & 63u) == 0) {
             if (error_flagged()) return false;
-            if (globaltimer_ns() - t0 > ATTN_WAIT_LIMIT_NS) {
+            if (globaltimer_ns() - t0 > limit_ns) {
                 record_error(code);
                 return false;
             }
         }
     }
+}
+
+// The kernels' wait: bounded by ATTN_WAIT_LIMIT_NS.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int code) {
+    return mbar_wait_for(bar, parity, code, ATTN_WAIT_LIMIT_NS);
 }
 
 // Makes generic-proxy shared-memory writes visible to the async proxy (TMA, tcgen05).

@@ -109,6 +109,20 @@ const char *attn_status_string(attn_status_t status);
 attn_status_t attn_device_error(int *code_out, attn_stream_t stream);
 
 /*
+ * Test hook for the kernels' failure detection: launches one CTA whose thread
+ * waits on a shared-memory barrier that nothing ever arrives on, bounded by
+ * limit_ns nanoseconds (0 .. 1e10) instead of the kernels' 2 s.  The wait runs
+ * out, records code 901 in the device error word and the kernel returns, so
+ * the stream completes and the context stays usable; attn_device_error then
+ * reports ATTN_ERR_DEVICE_TIMEOUT with that code (and clears it).  Run it with
+ * no other kernel of this library in flight: while the word is set, their
+ * bounded waits give up early.  No counterpart on the pages: the bounded
+ * waits are this library's own protection against hanging the GPU.
+ * Returns ATTN_ERR_INVALID_ARG for a limit outside that range.
+ */
+attn_status_t attn_selftest_wait_expiry(long long limit_ns, attn_stream_t stream);
+
+/*
  * Evaluates, on the device, the polynomial exp2 that the prefill softmax runs
  * on the FMA pipe for part of its exponentials: y[i] ~ 2^x[i] (x <= 127;
  * x below -125, including -inf, gives exactly 0).  degree 3 (bf16 path, max
@@ -353,7 +367,10 @@ attn_status_t attn_bwd_varlen(
  *   query heads per KV head) return ATTN_ERR_UNSUPPORTED.
  *   Set-up: the first call on each device looks up the scratch's device
  *   address (cudaGetSymbolAddress) with that device current; make that first
- *   call before any stream capture.
+ *   call before any stream capture.  The address is kept for the life of the
+ *   process, so this entry point must not be used on a device after
+ *   cudaDeviceReset (or any other teardown of its primary context).
+ *   Errors: bad arguments get the same status as from attn_decode_paged.
  *   Sharing: every call on a device uses the same scratch and leaves its
  *   contents behind (nothing in it needs to start zeroed).  Calls whose
  *   kernels could overlap on the GPU (different streams without ordering)

@@ -165,3 +165,33 @@ def test_patch_entry_point_checks_arguments(L):
     st = L.attn_fwd_patch(p, p, p, p, p, p, 1, 16, 16, 16, 2, 2, 96, 0.0, 16, 0, None, None, None,
                           p, None, None)
     assert st == 2
+
+
+def test_noalloc_decode_reports_bad_arguments_like_the_workspace_decode(L):
+    """attn_decode_paged_noalloc gives the same status as attn_decode_paged for every bad call
+    (also with B == 0), before it looks at its scratch or the device."""
+    p = ctypes.c_void_p(1 << 20)
+    odd = ctypes.c_void_p((1 << 20) + 8)
+    # (q, k, v, block_table, max_blocks, num_blocks, block_size, seqused_k, B, Hq, Hkv, D, dtype, o)
+    good = [p, p, p, p, 4, 100, 16, p, 2, 8, 2, 128, 0, p]
+    cases = {
+        "null q": {0: None}, "null k": {1: None}, "null v": {2: None},
+        "null block_table": {3: None}, "null seqused_k": {7: None}, "null o": {13: None},
+        "null q, B 0": {0: None, 8: 0}, "null o, B 0": {13: None, 8: 0},
+        "negative B": {8: -1}, "Hq not a multiple": {9: 6, 10: 4}, "Hkv 0": {10: 0},
+        "max_blocks 0": {4: 0}, "num_blocks 0": {5: 0}, "dtype 7": {12: 7},
+        "fp8": {12: 1}, "head_dim 96": {11: 96}, "head_dim 96, B 0": {11: 96, 8: 0},
+        "block_size 32": {6: 32}, "group 32": {9: 32, 10: 1}, "B 5000": {8: 5000},
+        "misaligned q": {0: odd}, "misaligned o": {13: odd},
+    }
+    for name, change in cases.items():
+        a = list(good)
+        for i, val in change.items():
+            a[i] = val
+        q, k, v, bt, mb, nb, bs, su, B_, Hq, Hkv, D, dt, o = a
+        ws_status = L.attn_decode_paged(q, k, v, bt, mb, nb, bs, su, B_, Hq, Hkv, D, 0.0, -1, 0.0,
+                                        0, dt, None, None, None, o, None, p, 1 << 24, None)
+        na_status = L.attn_decode_paged_noalloc(q, k, v, bt, mb, nb, bs, su, B_, Hq, Hkv, D, 0.0,
+                                                dt, o, None, None)
+        assert ws_status != 0, name
+        assert na_status == ws_status, name

@@ -4,10 +4,13 @@ It serves callers that cannot allocate device memory while they run (a
 plug-in inside a host program that owns all allocations, or a serving loop
 whose memory is fixed at start-up and must never reach cudaMalloc), by taking
 its split-KV scratch from a fixed array inside the library.  Its results must
-equal those of attn_decode_paged with a caller-provided workspace, also on a
-second call that finds the previous call's data left in that scratch.
+equal those of attn_decode_paged with a caller-provided workspace and those of
+the fp64 oracle, also on a second call that finds the previous call's data
+left in that scratch.
 """
 import ctypes
+
+import oracle
 
 import numpy as np
 import pytest
@@ -47,18 +50,28 @@ def _close(o, l, o_ref, l_ref):
     assert float((l[fin] - l_ref[fin]).abs().max()) <= TOL_LSE
 
 
+def _oracle(w):
+    t = w.tensors
+    o, l = oracle.attn_decode(t["q"], t["k_cache"], t["v_cache"], t["block_table"],
+                              t["seqused_k"], scale=w.params["scale"])
+    return torch.from_numpy(o).to(DEV), torch.from_numpy(l).to(DEV)
+
+
 def test_noalloc_matches_workspace_decode_on_two_calls_in_a_row():
     first = W.paged_decode(B=32, Hq=32, Hkv=8, D=128, num_blocks=6000, lmin=1, lmax=2048, seed=11)
     second = W.paged_decode(B=20, Hq=16, Hkv=4, D=64, num_blocks=3000, lmin=1, lmax=1500,
                             lens=[0, 1, 17, 1500, 33, 0, 700, 16, 15, 999] * 2, seed=12)
     for w in (first, second):
-        _close(*_both(w))
+        o, l, o_ref, l_ref = _both(w)
+        _close(o, l, o_ref, l_ref)                  # against the workspace entry point
+        _close(o, l, *_oracle(w))                   # and against the fp64 oracle
 
 
 def test_noalloc_rejects_requests_beyond_its_scratch():
     """A batch whose partials exceed the fixed 8 MiB scratch is refused with its own status."""
     L = A.lib()
-    st = L.attn_decode_paged_noalloc(None, None, None, None, 4, 16, 16, None, 4000, 32, 8, 128,
-                                     0.0, 0, None, None, None)
+    p = ctypes.c_void_p(1 << 20)      # never dereferenced: the request is refused before launch
+    st = L.attn_decode_paged_noalloc(p, p, p, p, 512, 20000, 16, p, 4000, 32, 8, 128,
+                                     0.0, 0, p, None, None)
     assert st == 8
     assert "scratch" in A.status_string(st)
