@@ -49,8 +49,6 @@ def lib():
         L.attn_device_error.restype = I
         L.attn_selftest_wait_expiry.argtypes = [ctypes.c_longlong, P]
         L.attn_selftest_wait_expiry.restype = I
-        L.attn_selftest_exp2.argtypes = [P, P, I, I, P]
-        L.attn_selftest_exp2.restype = I
         L.attn_fwd_dense.argtypes = [P, P, P, P, P, I, I, I, I, I, I, P, P, P, F, I, I, F, I,
                                      P, P, P, P]
         L.attn_fwd_dense.restype = I
@@ -141,14 +139,6 @@ def attn_selftest_wait_expiry(limit_ns: int, stream=None):
     """Launches the bounded-wait test kernel (a wait nothing satisfies, limited to limit_ns)."""
     _check(lib().attn_selftest_wait_expiry(int(limit_ns), _stream(stream)),
            "attn_selftest_wait_expiry")
-
-
-def attn_selftest_exp2(x, degree=3, stream=None):
-    """The prefill softmax's FMA-pipe exp2 applied to a device fp32 tensor."""
-    y = torch.empty_like(x)
-    _check(lib().attn_selftest_exp2(_ptr(x), _ptr(y), x.numel(), int(degree), _stream(stream)),
-           "attn_selftest_exp2")
-    return y
 
 
 def attn_fwd_dense(q, k, v, *, causal=False, scale=None, window_left=-1, softcap=0.0,
@@ -309,10 +299,6 @@ def attn_decode_paged_only_qv(qv, v_cache, block_table, seqused_k, *, scale=None
                                          _ptr(workspace), workspace.numel(), _stream(stream))
     _check(st, "attn_decode_paged_only_qv")
     return out, lse
-
-
-def default_scale(head_dim: int) -> float:
-    return 1.0 / math.sqrt(head_dim)
 
 
 def attn_decode_paged_noalloc(q, k_cache, v_cache, block_table, seqused_k, *, scale=None,

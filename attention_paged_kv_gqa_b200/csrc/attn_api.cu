@@ -344,12 +344,6 @@ attn_status_t launch_decode(const CUtensorMap& mk, const CUtensorMap& mv, Decode
     return ATTN_OK;
 }
 
-__global__ void exp2_selftest_kernel(const float* __restrict__ x, float* __restrict__ y, int n,
-                                     int degree) {
-    const int i = blockIdx.x * blockDim.x + threadIdx.x;
-    if (i < n) y[i] = degree >= 3 ? exp2_fma<3>(x[i]) : exp2_fma<2>(x[i]);
-}
-
 // One CTA waits on an mbarrier that nothing ever arrives on, bounded by
 // limit_ns: the wait expires, records kErrSelftestWait in the device error word
 // and the kernel returns (the failure-detection path of every kernel here,
@@ -519,15 +513,6 @@ attn_status_t attn_selftest_wait_expiry(long long limit_ns, attn_stream_t stream
     if (dvs != ATTN_OK) return dvs;
     wait_expiry_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
         static_cast<unsigned long long>(limit_ns));
-    return launch_status();
-}
-
-attn_status_t attn_selftest_exp2(const float* x, float* y, int n, int degree, attn_stream_t stream) {
-    if (!x || !y || n < 0 || (degree != 2 && degree != 3)) return ATTN_ERR_INVALID_ARG;
-    const attn_status_t dvs = current_device_ok(nullptr);
-    if (dvs != ATTN_OK) return dvs;
-    if (n == 0) return ATTN_OK;
-    exp2_selftest_kernel<<<(n + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n, degree);
     return launch_status();
 }
 

@@ -27,6 +27,7 @@ constexpr int kDecStageTok = 64;      // keys per stage (4 pages)
 constexpr int kDecRows = 16;          // MMA rows = query heads of one KV group (padded)
 constexpr int kDecMaxSeqs = 4096;     // sequences per call (on-device item table in smem)
 constexpr int kMaxSplits = 256;       // partials merged per (sequence, head)
+constexpr int kCombineRegs = 8;       // partials a combine thread merges from registers
 
 struct DecodeArgs {
     int B, Hq, Hkv, group;
@@ -794,6 +795,35 @@ __global__ void __launch_bounds__(D)
     const int pb = meta[b], pe = meta[b + 1];
     const int c0 = pb / ppc, c1 = (pe - 1) / ppc;
     const int ns = (pe > pb) ? min(c1 - c0 + 1, kMaxSplits) : 0;
+    if (ns <= kCombineRegs) {
+        // Few partials (the common case): every thread loads all of their LSEs and
+        // its own column of each O partial at once, and forms the weights itself,
+        // so the merge costs one round trip to memory.
+        float ls[kCombineRegs], ov[kCombineRegs];
+#pragma unroll
+        for (int s = 0; s < kCombineRegs; ++s) {
+            const long long slot = (long long)(c0 + s + b) * Hq + h;
+            ls[s] = s < ns ? lse_part[slot] : -INFINITY;
+            ov[s] = s < ns ? o_part[slot * D + d] : 0.0f;
+        }
+        float M = -INFINITY;
+#pragma unroll
+        for (int s = 0; s < kCombineRegs; ++s) M = fmaxf(M, ls[s]);
+        float W = 0.0f;
+        if (M != -INFINITY) {
+#pragma unroll
+            for (int s = 0; s < kCombineRegs; ++s) W += __expf(ls[s] - M);
+        }
+        const float out_lse = (M != -INFINITY && W > 0.0f) ? M + __logf(W) : -INFINITY;
+        float acc = 0.0f;
+        if (out_lse != -INFINITY) {
+#pragma unroll
+            for (int s = 0; s < kCombineRegs; ++s) acc += __expf(ls[s] - out_lse) * ov[s];
+        }
+        o[(long long)bh * D + d] = __float2bfloat16_rn(acc);
+        if (lse && d == 0) lse[bh] = out_lse;
+        return;
+    }
     if (threadIdx.x < 32) {
         const int lane = threadIdx.x;
         float M = -INFINITY;

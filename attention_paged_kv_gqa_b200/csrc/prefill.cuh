@@ -38,23 +38,8 @@ constexpr int kPageRows = 16;      // paged KV: tokens per page
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only when the max grows by > 2^8
 constexpr float kLn2 = 0.69314718055994531f;
 constexpr float kLog2e = 1.44269504088896341f;
-// Of every 8 softmax exponentials, this many are evaluated by a polynomial on
-// the FMA pipe (exp2_fma) and the rest by the MUFU unit, so that the two run
-// side by side instead of the MUFU unit bounding the tile.
-#ifndef ATTN_EXP2_EMU_OF_8
-#define ATTN_EXP2_EMU_OF_8 0
-#endif
-constexpr int kEmuOf8 = ATTN_EXP2_EMU_OF_8;
-
-// exp2 of element e of a row (e is a constant after unrolling): MUFU or the
-// FMA polynomial.
-template <bool FP8>
-__device__ __forceinline__ float row_exp2(int e, float x) {
-    if ((e & 7) >= 8 - kEmuOf8) return exp2_fma<FP8 ? 2 : 3>(x);
-    return ex2(x);
-}
-
 enum : int { kMaskNone = 0, kMaskCausal = 1, kMaskPatch = 2 };
+
 
 // Error codes recorded when a bounded wait gives up.
 enum : int {
@@ -157,10 +142,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     auto vslot_empty = [&](int st) { return st < NS ? &v_empty[st] : &k_empty[st - NS]; };
     int* sched = reinterpret_cast<int*>(tmem_slot + 2);   // [t][0]=min start, [t][1]=max end
 
+    // ------------------------------------------------------------ work unit (a1)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-
-    // ------------------------------------------------------------ work unit (a1)
     // Units are enumerated with the query-unit index slowest and descending, so
     // the causal units with the most KV tiles are launched first.
     const int bh = a.B * a.NH;
@@ -584,10 +568,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                         const float* sc = &s[c4 * 32 + 4 * c];
                         const float2 x01 = ffma2(make_float2(sc[0], sc[1]), sl2x2, nmu2);
                         const float2 x23 = ffma2(make_float2(sc[2], sc[3]), sl2x2, nmu2);
-                        const float p0 = row_exp2<FP8>(4 * c + 0, x01.x);
-                        const float p1 = row_exp2<FP8>(4 * c + 1, x01.y);
-                        const float p2 = row_exp2<FP8>(4 * c + 2, x23.x);
-                        const float p3 = row_exp2<FP8>(4 * c + 3, x23.y);
+                        const float p0 = ex2(x01.x);
+                        const float p1 = ex2(x01.y);
+                        const float p2 = ex2(x23.x);
+                        const float p3 = ex2(x23.y);
                         if constexpr (CAP) {   // (packed adds here cost registers with the softcap)
                             sums2[0].x += p0;
                             sums2[0].y += p1;
@@ -605,8 +589,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
 #pragma unroll
                     for (int c = 0; c < 16; ++c) {
                         const float2 x = ffma2(make_float2(s[c4 * 32 + 2 * c], s[c4 * 32 + 2 * c + 1]), sl2x2, nmu2);
-                        const float p0 = row_exp2<FP8>(2 * c + 0, x.x);
-                        const float p1 = row_exp2<FP8>(2 * c + 1, x.y);
+                        const float p0 = ex2(x.x);
+                        const float p1 = ex2(x.y);
                         sums2[c & 1].x += p0;      // (packed adds here cost registers: spills)
                         sums2[c & 1].y += p1;
                         pk[c] = pack_bf16(p0, p1);

@@ -376,30 +376,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
     return r;
 }
 
-// 2^x evaluated on the FMA pipe instead of the MUFU unit, for x <= 127:
-//   j = round(x) (adding 1.5*2^23 leaves round(x) in the low mantissa bits),
-//   f = x - j in [-1/2, 1/2], 2^f ~ polynomial in f, and 2^j is added to the
-//   exponent field (the low bits of x + 1.5*2^23, shifted by 23, are j << 23).
-// x < -125 (including -inf, a masked score) gives exactly 0, like the flush
-// to zero of ex2.approx.ftz; the clamp keeps the bit arithmetic on normal
-// numbers.  Coefficients: Lawson minimax fit of 2^f, relative error 7.5e-5
-// (degree 3) and 1.7e-3 (degree 2); exp2_poly_fit.py reproduces them.
-template <int DEG>
-__device__ __forceinline__ float exp2_fma(float x_in) {
-    const float x = fmaxf(x_in, -125.0f);
-    const float t = x + 12582912.0f;
-    const float f = x - (t - 12582912.0f);
-    float p;
-    if constexpr (DEG >= 3) {
-        p = fmaf(fmaf(fmaf(5.517166853e-02f, f, 2.426111400e-01f), f, 6.932609677e-01f), f,
-                 9.999280572e-01f);
-    } else {
-        p = fmaf(fmaf(2.384289205e-01f, f, 7.034480572e-01f), f, 1.000443101e+00f);
-    }
-    const float r = __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-    return x_in < -125.0f ? 0.0f : r;
-}
-
 // Two fp32 -> packed bf16x2 (lo in the low half), round to nearest even.
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     uint32_t r;

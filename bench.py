@@ -7,23 +7,24 @@ Primary line (one JSON object on stdout, rank 0):
   20000-page pool.  value = algorithmic K/V (+Q, O, LSE, block-table) bytes per
   step / device time per step, in GB/s; one step = one attn_decode_paged call
   (split-KV kernel + combine kernel).
-Carried in the same line:
-  "prefill":     varlen paged GQA prefill, causal, 16 seqs, L ~ U[64, 4096],
-                 Hq=32, Hkv=8, D=128 -> TFLOP/s (4*D*allowed pairs per head)
-  "prefill_fp8": fp8 e4m3 dense causal B=4, H=16, L=4096, D=128 -> TFLOP/s,
-                 with the bf16 kernel on the same data beside it.
-  "window_softcap": the decode and varlen prefill workloads again with a
-                 sliding window of 1024 keys and a softcap of 50 (GB/s and
-                 TFLOP/s over the keys inside each window only).
-  "kv_append":   paged KV append of every token of the varlen prefill
-                 workload (GB/s of new K/V read + cache rows written), and
-                 one decode step with its one-token append (GB/s as decode).
-  "backward":    dQ, dK, dV of the varlen causal GQA workload (packed K/V,
-                 same lengths) -> TFLOP/s at 10*D per allowed pair per head.
+Carried in the same line (compact entries: value, unit, ms per step, and the
+fraction of the measured peak "frac" and of the spec peak "frac_spec"):
+  prefill       varlen paged GQA prefill, causal, 16 seqs, L ~ U[64, 4096],
+                Hq=32, Hkv=8, D=128 -> TFLOP/s (4*D per allowed pair per head)
+  prefill_fp8   fp8 e4m3 dense causal B=4, H=16, L=4096, D=128 -> TFLOP/s, with
+                the bf16 kernel on the same data beside it
+  window_softcap, kv_append, backward, only_qv, other_configs: the remaining
+                hot-path rows on the same workloads.
+  peaks         the denominators: measured HBM copy and bf16 GEMM rates (from
+                MEASURED_PEAKS.json), the fp8 e4m3 GEMM rate measured here with
+                torch._scaled_mm at 8192^3, and the spec figures.
+  cpu_baseline  the fp64 oracle on the host cores: the decode sample (GB/s) and
+                its wall seconds on bounded samples of every configuration.
 
 Timing: W warm-up steps, then K steps each bracketed by CUDA events on the
-launching stream, a 256 MiB L2 flush between steps outside the events, and a
-barrier + synchronize on both sides of the timed region; max over ranks.
+launching stream, a 512 MiB L2 eviction between steps outside the events, and
+a barrier + synchronize on both sides of the timed region; max over ranks.
+The end-to-end decode leg times K steps as one region with host copies in it.
 N > 1 runs N independent replicas (one process per GPU; no collective on the
 data path).  --impl reference times the fp64 CPU oracle instead.
 """
@@ -75,6 +76,50 @@ def measured_traffic(kind):
         return None
     return rec["bytes"]
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# The spec figures of a B200 (dense tensor rates; HBM3e bandwidth).
+SPEC_PEAKS = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0, "fp8_tflops": 4500.0}
+
+
+def measure_fp8_peak(dev, n=8192, reps=10):
+    """Dense e4m3 GEMM rate (TFLOP/s): torch._scaled_mm at n^3, best of `reps`, CUDA events."""
+    try:
+        g = torch.Generator(device="cpu").manual_seed(0)
+        a = torch.randn(n, n, generator=g).to(torch.float8_e4m3fn).to(dev)
+        b = torch.randn(n, n, generator=g).to(torch.float8_e4m3fn).to(dev).t()   # column-major
+        one = torch.ones((), dtype=torch.float32, device=dev)
+        for _ in range(3):
+            torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+        best = float("inf")
+        for _ in range(reps):
+            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s.record()
+            torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+            e.record()
+            torch.cuda.synchronize()
+            best = min(best, s.elapsed_time(e))
+        del a, b
+        return 2.0 * n ** 3 / (best * 1e-3) / 1e12
+    except Exception:
+        return None
+
+
+def entry(value, unit, ms, bound, peaks, dtype="bf16", digits=2):
+    """A compact result: value, unit, ms per step, fraction of the measured and spec peaks."""
+    key = "hbm_gbs" if bound == "hbm" else ("fp8_tflops" if dtype == "fp8" else "bf16_tflops")
+    e = {"value": round(value, digits), "unit": unit, "ms": round(ms, 5)}
+    if peaks.get(key):
+        e["frac"] = round(value / peaks[key], 4)
+    e["frac_spec"] = round(value / SPEC_PEAKS[key], 4)
+    return e
+
+
+def roofline(achieved, unit, bound, peaks, peak_kind, traffic, kernel, dtype="bf16"):
+    key = "hbm_gbs" if bound == "hbm" else ("fp8_tflops" if dtype == "fp8" else "bf16_tflops")
+    peak = peaks[key]
+    return {"bound": bound if bound == "hbm" else "tensor", "achieved": round(achieved, 1),
+            "peak": round(peak, 1), "unit": unit, "frac": round(achieved / peak, 4),
+            "traffic": traffic, "kernel": kernel, "peak_kind": peak_kind,
+            "peak_spec": SPEC_PEAKS[key], "frac_spec": round(achieved / SPEC_PEAKS[key], 4)}
 
 
 def parse_args():
@@ -355,35 +400,47 @@ def run_ours(args, rank, world, local):
     if st != 0:
         raise RuntimeError("device check failed: " + A.status_string(st))
     peaks, peak_kind = load_peaks()
+    fp8 = measure_fp8_peak(dev)
+    peaks["fp8_tflops"] = fp8 if fp8 else 2.0 * peaks["bf16_tflops"]
+    fp8_kind = ("measured here: torch._scaled_mm e4m3 8192^3, best of 10" if fp8 else
+                peak_kind + " bf16 x 2 (nominal fp8/bf16 ratio)")
     flush = torch.ones(512 << 20, dtype=torch.uint8, device=dev)
 
     line = {"metric": METRIC, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16"}
+    ctx = dict(args=args, A=A, W=W, dev=dev, world=world, flush=flush, peaks=peaks,
+               peak_kind=peak_kind, fp8_kind=fp8_kind, line=line, launches=0)
+    w = None
     if args.workload in ("all", "decode"):
-        w = run_decode(args, A, W, dev, world, flush, peaks, peak_kind, line)
+        w = run_decode(ctx)
     if args.workload in ("all", "prefill") and not args.no_prefill:
-        run_prefill(args, A, W, dev, world, flush, peaks, peak_kind, line)
+        run_prefill(ctx)
     if args.workload in ("all", "fp8") and not args.no_prefill:
-        run_fp8(args, A, W, dev, world, flush, peaks, peak_kind, line)
+        run_fp8(ctx)
     if args.workload in ("all", "window") and not args.no_prefill:
-        run_window(args, A, W, dev, world, flush, peaks, peak_kind, line)
+        run_window(ctx)
     if args.workload in ("all", "append"):
-        run_append(args, A, W, dev, world, flush, peaks, peak_kind, line)
+        run_append(ctx)
     if args.workload in ("all", "backward") and not args.no_prefill:
-        run_backward(args, A, W, dev, world, flush, peaks, peak_kind, line)
+        run_backward(ctx)
     if args.workload in ("all", "only_qv") and not args.no_prefill:
-        run_only_qv(args, A, W, dev, world, flush, peaks, peak_kind, line)
+        run_only_qv(ctx)
     if args.workload in ("all", "patch") and not args.no_prefill:
-        run_patch_and_small(args, A, W, dev, world, flush, peaks, peak_kind, line)
+        run_patch_and_small(ctx)
+    line["peaks"] = {"hbm_gbs": peaks["hbm_gbs"], "bf16_tflops": peaks["bf16_tflops"],
+                     "fp8_tflops": round(peaks["fp8_tflops"], 1), "kind": peak_kind,
+                     "fp8_kind": fp8_kind, "spec": SPEC_PEAKS}
     if args.workload in ("all", "decode") and rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
     if rank == 0:
-        print(json.dumps(line), flush=True)
+        print(json.dumps(line, separators=(",", ":")), flush=True)
 
 
-def run_decode(args, A, W, dev, world, flush, peaks, peak_kind, line):
+def run_decode(c):
     # ---------------- decode (primary)
+    args, A, W, dev, world, flush = c["args"], c["A"], c["W"], c["dev"], c["world"], c["flush"]
+    peaks, line = c["peaks"], c["line"]
     w = W.paged_decode(seed=args.seed)
     t = w.tensors
     P = w.params
@@ -409,10 +466,13 @@ def run_decode(args, A, W, dev, world, flush, peaks, peak_kind, line):
     ns = 1 if A.attn_decode_workspace_size(P["B"], P["Hq"], P["Hkv"], P["D"],
                                            P["max_blocks_per_seq"]) <= 16 else 2
 
-    # end to end through the binding with host buffers: q, block_table, seqused_k in
-    # (pinned), O and LSE out; the paged cache is resident device state.  The inputs
-    # travel packed in one pinned buffer (one copy in) and O | LSE come back in one
-    # buffer (one copy out), as a serving loop would stage a step's metadata.
+    # End to end through the binding with host buffers: every step copies its q,
+    # block_table and seqused_k in from pinned host memory (one packed buffer) and
+    # its O and LSE out (one buffer); the paged cache is resident device state.  As
+    # in a serving loop, the copies run on a second stream: step i+1's inputs go in
+    # while step i's kernels run, and step i's outputs come back while step i+1's
+    # run (two buffers each way).  The K steps are one timed region (device events);
+    # the 574 MB of K/V read per step is larger than L2.
     def views_of(buf, like):
         out, off = [], 0
         for x in like:
@@ -426,23 +486,56 @@ def run_decode(args, A, W, dev, world, flush, peaks, peak_kind, line):
     hin = torch.empty(n_in, dtype=torch.uint8).pin_memory()
     for v, x in zip(views_of(hin, ins), ins):
         v.copy_(x)
-    din = torch.empty(n_in, dtype=torch.uint8, device=dev)
-    qd, btd, sud = views_of(din, ins)
-    dout = torch.empty(o.numel() * o.element_size() + lse.numel() * lse.element_size(),
-                       dtype=torch.uint8, device=dev)
-    od, ld = views_of(dout, [o, lse])
-    hout = torch.empty(dout.numel(), dtype=torch.uint8).pin_memory()
+    n_out = o.numel() * o.element_size() + lse.numel() * lse.element_size()
+    din = [torch.empty(n_in, dtype=torch.uint8, device=dev) for _ in range(2)]
+    dout = [torch.empty(n_out, dtype=torch.uint8, device=dev) for _ in range(2)]
+    hout = [torch.empty(n_out, dtype=torch.uint8).pin_memory() for _ in range(2)]
+    vin = [views_of(b, ins) for b in din]
+    vout = [views_of(b, [o, lse]) for b in dout]
+    ks = torch.cuda.current_stream()
+    cs = torch.cuda.Stream(device=dev)
 
-    def e2e_step():
-        din.copy_(hin, non_blocking=True)
-        A.attn_decode_paged(qd, d["k_cache"], d["v_cache"], btd, sud, scale=P["scale"], out=od,
-                            lse=ld, workspace=ws)
-        hout.copy_(dout, non_blocking=True)
+    def e2e_run(n):
+        ev_in = [torch.cuda.Event() for _ in range(2)]
+        ev_k = [torch.cuda.Event() for _ in range(2)]
+        ev_out = [torch.cuda.Event() for _ in range(2)]
+        with torch.cuda.stream(cs):
+            din[0].copy_(hin, non_blocking=True)
+            ev_in[0].record(cs)
+        for i in range(n):
+            j = i % 2
+            ks.wait_event(ev_in[j])
+            if i >= 2:
+                ks.wait_event(ev_out[j])            # step i-2's outputs have left buffer j
+            qd, btd, sud = vin[j]
+            od, ld = vout[j]
+            A.attn_decode_paged(qd, d["k_cache"], d["v_cache"], btd, sud, scale=P["scale"],
+                                out=od, lse=ld, workspace=ws, stream=ks)
+            ev_k[j].record(ks)
+            with torch.cuda.stream(cs):
+                if i + 1 < n:
+                    jn = (i + 1) % 2
+                    if i >= 1:
+                        cs.wait_event(ev_k[jn])     # step i-1 has consumed buffer jn
+                    din[jn].copy_(hin, non_blocking=True)
+                    ev_in[jn].record(cs)
+                cs.wait_event(ev_k[j])
+                hout[j].copy_(dout[j], non_blocking=True)
+                ev_out[j].record(cs)
+        ks.wait_event(ev_out[(n - 1) % 2])
+        if n >= 2:
+            ks.wait_event(ev_out[(n - 2) % 2])
 
-    e2e_times = time_steps(e2e_step, args.steps, args.warmup, world, flush)
-    e2e_ms = max_over_ranks(sum(e2e_times), world) / args.steps
-    h2d = hin.numel()
-    d2h = hout.numel()
+    e2e_run(args.warmup)
+    barrier(world)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(ks)
+    cs.wait_event(t0)
+    e2e_run(args.steps)
+    t1.record(ks)
+    barrier(world)
+    e2e_ms = max_over_ranks(t0.elapsed_time(t1), world) / args.steps
+    c["launches"] += args.steps * ns * 2          # device-timed and end-to-end legs
 
     line.update({
         "value": round(value, 2), "ms_per_step": round(ms_max, 5),
@@ -452,29 +545,27 @@ def run_decode(args, A, W, dev, world, flush, peaks, peak_kind, line):
                                "20000-page pool" % (args.seed, int(t["seqused_k"].sum())),
                    "global_batch": P["B"] * world, "seq_len": int(t["seqused_k"].max()),
                    "parallelism": "replicas" if world > 1 else "single",
-                   "l2": "L2 flushed between timed steps by a read sweep of a 512 MiB buffer "
-                         "(and %.0f MB of K/V per step, larger than L2)" % (nbytes / 1e6),
+                   "l2": "flushed between timed steps (read sweep of 512 MiB); 574 MB of K/V "
+                         "per step, larger than L2",
                    "bytes_per_step": nbytes},
-        "roofline": {"bound": "hbm", "achieved": round(kernel_gbs, 1),
-                     "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": round(kernel_gbs / peaks["hbm_gbs"], 4),
-                     "traffic": measured_traffic("decode"),
-                     "kernel": "decode_pages_kernel<128> + decode_pages_combine_kernel<128> (one call)",
-                     "peak_kind": peak_kind},
+        "roofline": roofline(kernel_gbs, "GB/s", "hbm", peaks, c["peak_kind"],
+                             measured_traffic("decode"),
+                             "decode_pages_kernel<128> + decode_pages_combine_kernel<128>"),
         "e2e": {"value": round(nbytes * world / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "h2d_bytes_per_step": n_in, "d2h_bytes_per_step": n_out,
                 "ms_per_step": round(e2e_ms, 5),
-                "note": "paged K/V cache resident on the device; q, block_table, seqused_k "
-                        "copied in (one packed pinned buffer) and O, LSE copied out (one "
-                        "buffer) every step"},
-        "gpu_launches": args.steps * ns,
+                "note": "K steps in one timed region; each step copies q, block_table, "
+                        "seqused_k in and O, LSE out (pinned host), on a copy stream "
+                        "overlapping the neighbouring steps' kernels"},
         "clocks": clocks,
     })
+    line["gpu_launches"] = c["launches"]
     return w
 
 
-def run_prefill(args, A, W, dev, world, flush, peaks, peak_kind, line):
-    # ---------------- prefill (carried in the same line)
+def run_prefill(c):
+    args, A, W, dev, world, flush = c["args"], c["A"], c["W"], c["dev"], c["world"], c["flush"]
+    peaks = c["peaks"]
     wp = W.varlen_paged_prefill(seed=args.seed)
     tp, Pp = wp.tensors, wp.params
     dp = {k: v.to(dev) for k, v in tp.items()}
@@ -487,25 +578,23 @@ def run_prefill(args, A, W, dev, world, flush, peaks, peak_kind, line):
                                 block_table=dp["block_table"], seqused_k=dp["seqused_k"],
                                 mask=A.MASK_CAUSAL, scale=Pp["scale"], out=op, lse=lp)
 
-    pt = time_steps(pf_step, args.steps, args.warmup, world, flush)
-    pms = statistics.mean(pt)
+    pms = statistics.mean(time_steps(pf_step, args.steps, args.warmup, world, flush))
     flops = causal_flops(tp["seqused_k"].numpy(), Pp["Hq"], Pp["D"])
     tf = flops / (pms * 1e-3) / 1e12
-    line["prefill"] = {
-        "workload": "varlen_paged_gqa_prefill_causal_bf16: 16 seqs, q len = kv len ~ "
-                    "U[64,4096] (seed %d: %d tokens), Hq=32, Hkv=8, D=128, 16-token pages"
-                    % (args.seed, Pp["total_q"]),
-        "value": round(tf, 2), "unit": "TFLOP/s", "ms_per_step": round(pms, 5),
-        "flops_per_step": flops,
-        "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": peaks["bf16_tflops"],
-                     "unit": "TFLOP/s", "frac": round(tf / peaks["bf16_tflops"], 4),
-                     "traffic": measured_traffic("prefill"), "kernel": "prefill_kernel<128,bf16>",
-                     "peak_kind": peak_kind},
-    }
+    e = entry(tf, "TFLOP/s", pms, "tensor", peaks)
+    e["workload"] = "varlen paged GQA causal, %d tokens" % Pp["total_q"]
+    e["flops_per_step"] = flops
+    e["roofline"] = roofline(tf, "TFLOP/s", "tensor", peaks, c["peak_kind"],
+                             measured_traffic("prefill"), "prefill_kernel<128,bf16>")
+    c["line"]["prefill"] = e
+    c["launches"] += args.steps
+    c["line"]["gpu_launches"] = c["launches"]
     del dp
 
 
-def run_fp8(args, A, W, dev, world, flush, peaks, peak_kind, line):
+def run_fp8(c):
+    args, A, W, dev, world, flush = c["args"], c["A"], c["W"], c["dev"], c["world"], c["flush"]
+    peaks = c["peaks"]
     w8 = W.fp8_dense_causal(seed=args.seed)
     t8 = w8.tensors
     d8 = {k: v.to(dev) for k, v in t8.items()}
@@ -524,28 +613,27 @@ def run_fp8(args, A, W, dev, world, flush, peaks, peak_kind, line):
     f8ms = statistics.mean(time_steps(f8_step, args.steps, args.warmup, world, flush))
     b16ms = statistics.mean(time_steps(b16_step, args.steps, args.warmup, world, flush))
     fl8 = causal_flops([4096] * 4, 16, 128)
-    fp8_peak = 2.0 * peaks["bf16_tflops"]
-    line["prefill_fp8"] = {
-        "workload": "fp8_e4m3_dense_causal: B=4, H=16, L=4096, D=128, per-tensor descale",
-        "value": round(fl8 / (f8ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
-        "ms_per_step": round(f8ms, 5),
-        "bf16_same_data": {"value": round(fl8 / (b16ms * 1e-3) / 1e12, 2),
-                           "ms_per_step": round(b16ms, 5),
-                           "fp8_time_over_bf16_time": round(f8ms / b16ms, 4)},
-        "roofline": {"bound": "tensor", "achieved": round(fl8 / (f8ms * 1e-3) / 1e12, 1),
-                     "peak": fp8_peak, "unit": "TFLOP/s",
-                     "frac": round(fl8 / (f8ms * 1e-3) / 1e12 / fp8_peak, 4), "traffic": None,
-                     "kernel": "prefill_kernel<128,fp8>",
-                     "peak_kind": peak_kind + " bf16 x 2 (nominal fp8/bf16 ratio)"},
-    }
+    tf8, tf16 = fl8 / (f8ms * 1e-3) / 1e12, fl8 / (b16ms * 1e-3) / 1e12
+    e = entry(tf8, "TFLOP/s", f8ms, "tensor", peaks, dtype="fp8")
+    e["workload"] = "fp8 e4m3 dense causal B=4 H=16 L=4096 D=128"
+    e["bf16_same_data"] = entry(tf16, "TFLOP/s", b16ms, "tensor", peaks)
+    e["fp8_time_over_bf16_time"] = round(f8ms / b16ms, 4)
+    e["roofline"] = roofline(tf8, "TFLOP/s", "tensor", peaks, c["fp8_kind"],
+                             measured_traffic("prefill_fp8"), "prefill_kernel<128,fp8>",
+                             dtype="fp8")
+    c["line"]["prefill_fp8"] = e
+    c["launches"] += 2 * args.steps
+    c["line"]["gpu_launches"] = c["launches"]
     del d8
 
 
 WINDOW, SOFTCAP = 1024, 50.0
 
 
-def run_window(args, A, W, dev, world, flush, peaks, peak_kind, line):
+def run_window(c):
     """Decode and varlen prefill with a sliding window, a softcap, and both."""
+    args, A, W, dev, world, flush = c["args"], c["A"], c["W"], c["dev"], c["world"], c["flush"]
+    peaks = c["peaks"]
     w = W.paged_decode(seed=args.seed)
     t, P = w.tensors, w.params
     d = {k: v.to(dev) for k, v in t.items()}
@@ -565,13 +653,8 @@ def run_window(args, A, W, dev, world, flush, peaks, peak_kind, line):
         dms = statistics.mean(time_steps(dec_step, args.steps, args.warmup, world, flush))
         nb = (window_decode_bytes(t, P["Hq"], P["Hkv"], P["D"], wl) if wl >= 0
               else decode_bytes(t, P["Hq"], P["Hkv"], P["D"]))
-        gbs = nb / (dms * 1e-3) / 1e9
-        out[name] = {"value": round(gbs, 2), "unit": "GB/s", "ms_per_step": round(dms, 5),
-                     "bytes_per_step": nb,
-                     "roofline": {"bound": "hbm", "achieved": round(gbs, 1),
-                                  "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                                  "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": None,
-                                  "peak_kind": peak_kind}}
+        out[name] = entry(nb / (dms * 1e-3) / 1e9, "GB/s", dms, "hbm", peaks)
+        c["launches"] += 2 * args.steps
     del d
 
     wp = W.varlen_paged_prefill(seed=args.seed)
@@ -593,23 +676,18 @@ def run_window(args, A, W, dev, world, flush, peaks, peak_kind, line):
         pms = statistics.mean(time_steps(pf_step, args.steps, args.warmup, world, flush))
         fl = (window_causal_flops(lens, Pp["Hq"], Pp["D"], wl) if wl >= 0
               else causal_flops(lens, Pp["Hq"], Pp["D"]))
-        tf = fl / (pms * 1e-3) / 1e12
-        out[name] = {"value": round(tf, 2), "unit": "TFLOP/s", "ms_per_step": round(pms, 5),
-                     "flops_per_step": fl,
-                     "roofline": {"bound": "tensor", "achieved": round(tf, 1),
-                                  "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                                  "frac": round(tf / peaks["bf16_tflops"], 4), "traffic": None,
-                                  "peak_kind": peak_kind}}
+        out[name] = entry(fl / (pms * 1e-3) / 1e12, "TFLOP/s", pms, "tensor", peaks)
+        c["launches"] += args.steps
     del dp
-    out["workloads"] = ("the paged GQA decode and varlen paged GQA prefill workloads above, "
-                        "with window_left %d (decode: keys L-1-%d .. L-1) and/or softcap %g; "
-                        "work counted over the keys inside each window only" % (WINDOW, WINDOW,
-                                                                                 SOFTCAP))
-    line["window_softcap"] = out
+    out["note"] = "decode and varlen prefill workloads; work counted inside each window only"
+    c["line"]["window_softcap"] = out
+    c["line"]["gpu_launches"] = c["launches"]
 
 
-def run_append(args, A, W, dev, world, flush, peaks, peak_kind, line):
+def run_append(c):
     """Paged KV append at prefill size, and a decode step with its append."""
+    args, A, W, dev, world, flush = c["args"], c["A"], c["W"], c["dev"], c["world"], c["flush"]
+    peaks = c["peaks"]
     wp = W.varlen_paged_prefill(seed=args.seed)
     tp, Pp = wp.tensors, wp.params
     lens = tp["seqused_k"]
@@ -628,12 +706,10 @@ def run_append(args, A, W, dev, world, flush, peaks, peak_kind, line):
 
     ams = statistics.mean(time_steps(app_step, args.steps, args.warmup, world, flush))
     nbytes = 2 * 2 * total * Hkv * D * 2 + int(lens.numel()) * 4 * 3 + 4 * (lens.numel() + 1)
-    gbs = nbytes / (ams * 1e-3) / 1e9
     del k_new, v_new, kc, vc
 
     w = W.paged_decode(seed=args.seed)
     t, P = w.tensors, w.params
-    # one more page-table slot of room per sequence is already there (L <= 8192 < 512 pages)
     d = {k: v.to(dev) for k, v in t.items()}
     g = torch.Generator().manual_seed(args.seed + 99)
     kn = torch.randn(P["B"], P["Hkv"], P["D"], generator=g).to(torch.bfloat16).to(dev)
@@ -656,30 +732,20 @@ def run_append(args, A, W, dev, world, flush, peaks, peak_kind, line):
     lens_after = (t["seqused_k"] - 1).clamp(min=0) + 1
     nb_dec = decode_bytes({"seqused_k": lens_after}, P["Hq"], P["Hkv"], P["D"]) + \
         2 * 2 * P["B"] * P["Hkv"] * P["D"] * 2
-    dgbs = nb_dec / (dms * 1e-3) / 1e9
     del d
-    line["kv_append"] = {
-        "prefill_size": {
-            "workload": "every token of the varlen paged prefill workload (%d tokens, Hkv=8, "
-                        "D=128, bf16) appended to empty sequences" % total,
-            "value": round(gbs, 2), "unit": "GB/s", "ms_per_step": round(ams, 5),
-            "bytes_per_step": nbytes,
-            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"],
-                         "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4),
-                         "traffic": None, "kernel": "kv_append_kernel", "peak_kind": peak_kind}},
-        "decode_step": {
-            "workload": "the paged GQA decode workload, each sequence appending its newest "
-                        "token in the same call (append + decode)",
-            "value": round(dgbs, 2), "unit": "GB/s", "ms_per_step": round(dms, 5),
-            "bytes_per_step": nb_dec,
-            "roofline": {"bound": "hbm", "achieved": round(dgbs, 1), "peak": peaks["hbm_gbs"],
-                         "unit": "GB/s", "frac": round(dgbs / peaks["hbm_gbs"], 4),
-                         "traffic": None, "peak_kind": peak_kind}},
-    }
+    e1 = entry(nbytes / (ams * 1e-3) / 1e9, "GB/s", ams, "hbm", peaks)
+    e1["workload"] = "all %d prefill tokens into empty sequences" % total
+    e2 = entry(nb_dec / (dms * 1e-3) / 1e9, "GB/s", dms, "hbm", peaks)
+    e2["workload"] = "decode step with its one-token append (PDL chain)"
+    c["line"]["kv_append"] = {"prefill_size": e1, "decode_step": e2}
+    c["launches"] += 4 * args.steps
+    c["line"]["gpu_launches"] = c["launches"]
 
 
-def run_backward(args, A, W, dev, world, flush, peaks, peak_kind, line):
+def run_backward(c):
     """dQ, dK, dV of the varlen causal GQA workload (packed K/V)."""
+    args, A, W, dev, world, flush = c["args"], c["A"], c["W"], c["dev"], c["world"], c["flush"]
+    peaks = c["peaks"]
     wp = W.varlen_paged_prefill(seed=args.seed)
     Pp = wp.params
     lens = wp.tensors["seqused_k"]
@@ -702,25 +768,20 @@ def run_backward(args, A, W, dev, world, flush, peaks, peak_kind, line):
 
     bms = statistics.mean(time_steps(bwd_step, args.steps, args.warmup, world, flush))
     flops = 2.5 * causal_flops(lens.numpy(), Hq, D)
-    tf = flops / (bms * 1e-3) / 1e12
-    line["backward"] = {
-        "workload": "varlen causal GQA backward: 16 seqs, L ~ U[64,4096] (seed %d: %d tokens), "
-                    "Hq=32, Hkv=8, D=128, packed K/V, bf16" % (args.seed, total),
-        "value": round(tf, 2), "unit": "TFLOP/s", "ms_per_step": round(bms, 5),
-        "flops_per_step": flops,
-        "flops_convention": "10*D per allowed (q,k) pair per query head (five GEMMs; the "
-                            "kernels run seven, recomputing S and dP for dQ)",
-        "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": peaks["bf16_tflops"],
-                     "unit": "TFLOP/s", "frac": round(tf / peaks["bf16_tflops"], 4),
-                     "traffic": None, "kernel": "bwd_dkdv_kernel<128> + bwd_dq_kernel<128> "
-                                                "(+ bwd_delta_kernel)", "peak_kind": peak_kind},
-    }
+    e = entry(flops / (bms * 1e-3) / 1e12, "TFLOP/s", bms, "tensor", peaks)
+    e["workload"] = "varlen causal GQA backward, %d tokens, packed K/V" % total
+    e["flops_convention"] = "10*D per allowed pair per query head (5 GEMMs; 7 run)"
+    c["line"]["backward"] = e
+    c["launches"] += 3 * args.steps
+    c["line"]["gpu_launches"] = c["launches"]
     del q, k, v, do, o, dq, dk, dv
 
 
-def run_only_qv(args, A, W, dev, world, flush, peaks, peak_kind, line):
+def run_only_qv(c):
     """The only_qv score path (score = scale * qv . v) on the decode and prefill workloads:
     the query tensor serves as qv and the value cache as the only KV store."""
+    args, A, W, dev, world, flush = c["args"], c["A"], c["W"], c["dev"], c["world"], c["flush"]
+    peaks = c["peaks"]
     w = W.paged_decode(seed=args.seed)
     t, P = w.tensors, w.params
     d = {k: v.to(dev) for k, v in t.items() if k != "k_cache"}
@@ -738,13 +799,7 @@ def run_only_qv(args, A, W, dev, world, flush, peaks, peak_kind, line):
     # algorithmic bytes: decode_bytes with the V half of the K/V stream only
     lens = t["seqused_k"].numpy().astype(np.int64)
     nb = decode_bytes(t, P["Hq"], P["Hkv"], P["D"]) - int(lens.sum()) * P["Hkv"] * P["D"] * 2
-    gbs = nb / (dms * 1e-3) / 1e9
-    out = {"decode": {"value": round(gbs, 2), "unit": "GB/s", "ms_per_step": round(dms, 5),
-                      "bytes_per_step": nb,
-                      "roofline": {"bound": "hbm", "achieved": round(gbs, 1),
-                                   "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                                   "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": None,
-                                   "peak_kind": peak_kind}}}
+    out = {"decode": entry(nb / (dms * 1e-3) / 1e9, "GB/s", dms, "hbm", peaks)}
     del d
 
     wp = W.varlen_paged_prefill(seed=args.seed)
@@ -761,23 +816,19 @@ def run_only_qv(args, A, W, dev, world, flush, peaks, peak_kind, line):
 
     pms = statistics.mean(time_steps(pf_step, args.steps, args.warmup, world, flush))
     fl = causal_flops(tp["seqused_k"].numpy(), Pp["Hq"], Pp["D"])
-    tf = fl / (pms * 1e-3) / 1e12
-    out["prefill"] = {"value": round(tf, 2), "unit": "TFLOP/s", "ms_per_step": round(pms, 5),
-                      "flops_per_step": fl,
-                      "roofline": {"bound": "tensor", "achieved": round(tf, 1),
-                                   "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                                   "frac": round(tf / peaks["bf16_tflops"], 4), "traffic": None,
-                                   "peak_kind": peak_kind}}
+    out["prefill"] = entry(fl / (pms * 1e-3) / 1e12, "TFLOP/s", pms, "tensor", peaks)
     del dp
-    out["workloads"] = ("the paged GQA decode and varlen paged GQA causal prefill workloads "
-                        "above with the query tensor as qv and the value cache as the only "
-                        "KV store; decode bytes count V once (no K stream)")
-    line["only_qv"] = out
+    out["note"] = "q as qv, the value cache as the only store; decode bytes count V once"
+    c["line"]["only_qv"] = out
+    c["launches"] += 3 * args.steps
+    c["line"]["gpu_launches"] = c["launches"]
 
 
-def run_patch_and_small(args, A, W, dev, world, flush, peaks, peak_kind, line):
+def run_patch_and_small(c):
     """The two remaining configurations: patch cross-attention (memory-bound: GB/s against
     HBM) and the small dense causal case (launch-latency bound: microseconds per call)."""
+    args, A, W, dev, world, flush = c["args"], c["A"], c["W"], c["dev"], c["world"], c["flush"]
+    peaks = c["peaks"]
     w = W.patch_cross(seed=args.seed)
     t, P = w.tensors, w.params
     d = {k: v.to(dev) for k, v in t.items()}
@@ -798,25 +849,12 @@ def run_patch_and_small(args, A, W, dev, world, flush, peaks, peak_kind, line):
 
     pms = statistics.mean(time_steps(patch_step, args.steps, args.warmup, world, flush))
     tms = statistics.mean(time_steps(patch_tiled_step, args.steps, args.warmup, world, flush))
-    # algorithmic bytes: every key and value row once (each belongs to one patch), Q and O,
-    # LSE, the per-query ranges and the cumulative lengths
-    nb = (2 * P["total_k"] * P["Hkv"] * P["D"] * 2 + 2 * P["total_q"] * P["Hq"] * P["D"] * 2
-          + P["total_q"] * P["Hq"] * 4 + P["total_q"] * 8 + 2 * (P["B"] + 1) * 4)
-    gbs = nb / (pms * 1e-3) / 1e9
-    out = {"patch": {"workload": "patch cross-attention bf16: B=4 x 8192 byte keys, Geometric(0.22) "
-                                 "patches clipped to [1,16] (seed %d: %d queries), H=16, D=64, "
-                                 "packed K/V" % (args.seed, P["total_q"]),
-                     "value": round(gbs, 2), "unit": "GB/s", "ms_per_step": round(pms, 5),
-                     "bytes_per_step": nb,
-                     "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"],
-                                  "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4),
-                                  "traffic": None, "kernel": "patch_query_kernel<64, 16> (attn_fwd_patch, "
-                                                              "max_interval 16)",
-                                  "peak_kind": peak_kind},
-                     "tiled_kernel": {"value": round(nb / (tms * 1e-3) / 1e9, 2), "unit": "GB/s",
-                                      "ms_per_step": round(tms, 5),
-                                      "note": "the same call through attn_fwd_varlen_paged "
-                                              "(tensor-core tiles with the patch mask)"}}}
+    nb = patch_bytes(P)
+    e = entry(nb / (pms * 1e-3) / 1e9, "GB/s", pms, "hbm", peaks)
+    e["workload"] = "B=4 x 8192 bytes, %d patch queries, H=16, D=64" % P["total_q"]
+    e["kernel"] = "patch_query_kernel<64,16> (attn_fwd_patch)"
+    e["tiled_kernel"] = entry(nb / (tms * 1e-3) / 1e9, "GB/s", tms, "hbm", peaks)
+    out = {"patch": e}
     del d
     w1 = W.dense(seed=args.seed)
     t1 = {k: v.to(dev) for k, v in w1.tensors.items()}
@@ -827,15 +865,94 @@ def run_patch_and_small(args, A, W, dev, world, flush, peaks, peak_kind, line):
         A.attn_fwd_dense(t1["q"], t1["k"], t1["v"], causal=True, scale=w1.params["scale"], out=o1, lse=l1)
 
     sms = statistics.mean(time_steps(small_step, args.steps, args.warmup, world, flush))
-    out["dense_small"] = {"workload": "dense causal bf16: B=2, Hq=Hkv=2, L=128, D=64",
-                          "value": round(sms * 1e3, 2), "unit": "us per call",
+    out["dense_small"] = {"value": round(sms * 1e3, 2), "unit": "us per call",
                           "higher_is_better": False,
-                          "note": "8.45 MFLOP: launch- and latency-bound, no roofline"}
-    line["other_configs"] = out
+                          "note": "B=2 L=128 H=2 D=64 causal: 8.45 MFLOP, latency-bound"}
+    c["line"]["other_configs"] = out
+    c["launches"] += 3 * args.steps
+    c["line"]["gpu_launches"] = c["launches"]
+
+
+def patch_bytes(P):
+    """Every key and value row once (each belongs to one patch), Q and O, LSE, the
+    per-query ranges and the cumulative lengths."""
+    return (2 * P["total_k"] * P["Hkv"] * P["D"] * 2 + 2 * P["total_q"] * P["Hq"] * P["D"] * 2
+            + P["total_q"] * P["Hq"] * 4 + P["total_q"] * 8 + 2 * (P["B"] + 1) * 4)
+
+
+def oracle_config_samples():
+    """Wall seconds of the fp64 oracle, as it stands, on a bounded sample of each
+    configuration (the small dense one whole), with the sample named and its work
+    rate in the configuration's unit."""
+    import oracle
+    from attention_paged_kv_gqa_b200 import workloads as W
+    n = os.cpu_count() or 1
+    out = {}
+    w = W.dense(seed=0)
+    t = w.tensors
+    t0 = time.perf_counter()
+    oracle.attn_dense(t["q"], t["k"], t["v"], scale=w.params["scale"], causal=True, nthreads=n)
+    out["dense_causal_small"] = {"seconds": round(time.perf_counter() - t0, 4),
+                                 "sample": "whole (B=2, L=128, H=2, D=64)"}
+    wp = W.varlen_paged_prefill(seed=0)
+    tp = wp.tensors
+    lens = tp["seqused_k"].numpy()
+    b = int(np.argmax(lens))
+    L = int(lens[b])
+    cu = tp["cu_seqlens_q"].numpy()
+    rows = 128
+    q = tp["q"][cu[b + 1] - rows:cu[b + 1]]
+    npg = (L + 15) // 16
+    kc, vc = tp["k_cache"][tp["block_table"][b, :npg].long()], tp["v_cache"][tp["block_table"][b, :npg].long()]
+    t0 = time.perf_counter()
+    oracle.attn_varlen(q, kc, vc, cu_seqlens_q=np.array([0, rows], np.int32),
+                       seqused_k=np.array([L], np.int32),
+                       block_table=np.arange(npg, dtype=np.int32)[None], num_heads_kv=8,
+                       scale=wp.params["scale"], mask=1, nthreads=n)
+    dt = time.perf_counter() - t0
+    pairs = sum(L - rows + i + 1 for i in range(rows))
+    out["varlen_paged_prefill"] = {"seconds": round(dt, 3),
+                                   "value": round(4 * 128 * 32 * pairs / dt / 1e9, 3),
+                                   "unit": "GFLOP/s",
+                                   "sample": "last %d rows of the %d-token sequence, 32 heads"
+                                             % (rows, L)}
+    wc = W.patch_cross(seed=0)
+    tc = wc.tensors
+    nq = 256
+    r = tc["patch_kv_range"][:nq]
+    t0 = time.perf_counter()
+    oracle.attn_varlen(tc["q"][:nq], tc["k"][:8192], tc["v"][:8192],
+                       cu_seqlens_q=np.array([0, nq], np.int32),
+                       cu_seqlens_k=np.array([0, 8192], np.int32), num_heads_kv=16,
+                       scale=wc.params["scale"], mask=2, patch_kv_range=r, nthreads=n)
+    dt = time.perf_counter() - t0
+    keys = int((r[:, 1] - r[:, 0]).sum())
+    nbytes = 2 * keys * 16 * 64 * 2 + 2 * nq * 16 * 64 * 2 + nq * 16 * 4 + nq * 8
+    out["patch_cross"] = {"seconds": round(dt, 3), "value": round(nbytes / dt / 1e9, 5),
+                          "unit": "GB/s",
+                          "sample": "first %d patch queries of sequence 0 (8192-key rows)" % nq}
+    w8 = W.fp8_dense_causal(seed=0)
+    t8 = w8.tensors
+    rows = 128
+    qd = oracle.dequant_e4m3(t8["q_fp8"][0:1, -rows:], t8["descale_q"])
+    kd = oracle.dequant_e4m3(t8["k_fp8"][0:1], t8["descale_k"])
+    vd = oracle.dequant_e4m3(t8["v_fp8"][0:1], t8["descale_v"])
+    t0 = time.perf_counter()
+    oracle.attn_varlen(qd[0], kd[0], vd[0], cu_seqlens_q=np.array([0, rows], np.int32),
+                       cu_seqlens_k=np.array([0, 4096], np.int32), num_heads_kv=16,
+                       scale=w8.params["scale"], mask=1, nthreads=n)
+    dt = time.perf_counter() - t0
+    pairs = sum(4096 - rows + i + 1 for i in range(rows))
+    out["fp8_dense_causal"] = {"seconds": round(dt, 3),
+                               "value": round(4 * 128 * 16 * pairs / dt / 1e9, 3),
+                               "unit": "GFLOP/s",
+                               "sample": "last %d rows of batch element 0, 16 heads" % rows}
+    return out
 
 
 def cpu_baseline(w):
-    """The oracle on rank 0 at N=1, a bounded sample (about 10 s) of the decode batch."""
+    """The oracle on rank 0 at N=1: a bounded sample (about 10 s) of the decode batch, in
+    the primary metric's unit, and its wall seconds on samples of every configuration."""
     secs, nb, nseq, tok = 0.0, 0, 0, 0
     t_start = time.perf_counter()
     i = 0
@@ -850,7 +967,7 @@ def cpu_baseline(w):
             "cores": os.cpu_count() or 1, "kind": "oracle",
             "sample": "%d oracle calls over %d whole sequences (%d keys, all "
                       "32 heads) of the decode batch" % (i, nseq, tok),
-            "cpu": cpu_model()}
+            "cpu": cpu_model(), "per_config": oracle_config_samples()}
 
 
 def main():

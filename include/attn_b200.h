@@ -122,15 +122,6 @@ attn_status_t attn_device_error(int *code_out, attn_stream_t stream);
  */
 attn_status_t attn_selftest_wait_expiry(long long limit_ns, attn_stream_t stream);
 
-/*
- * Evaluates, on the device, the polynomial exp2 that the prefill softmax runs
- * on the FMA pipe for part of its exponentials: y[i] ~ 2^x[i] (x <= 127;
- * x below -125, including -inf, gives exactly 0).  degree 3 (bf16 path, max
- * relative error 7.5e-5) or 2 (fp8 path, 1.7e-3).  x and y are device arrays
- * of n fp32.  A test hook for the accuracy of that building block; it has no
- * counterpart on the pages (their kernels call the hardware exp2 only).
- */
-attn_status_t attn_selftest_exp2(const float *x, float *y, int n, int degree, attn_stream_t stream);
 
 /*
  * Dense attention forward.

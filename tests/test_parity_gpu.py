@@ -269,9 +269,7 @@ def test_config_paged_decode_full():
     torch.cuda.synchronize()
     _no_device_error()
     lens = t["seqused_k"].numpy()
-    sample = sorted(set([int(np.argmax(lens)), int(np.argmin(lens))] +
-                        list(np.random.default_rng(0).choice(len(lens), 6, replace=False))))
-    for b in sample:
+    for b in range(len(lens)):                       # every sequence, element by element
         kc, vc, bt = _compact_pages(t["k_cache"], t["v_cache"], t["block_table"][b], lens[b])
         o_ref, lse_ref = oracle.attn_decode(t["q"][b:b + 1], kc, vc, bt, t["seqused_k"][b:b + 1],
                                             scale=w.params["scale"])
@@ -279,7 +277,8 @@ def test_config_paged_decode_full():
 
 
 def test_config_varlen_paged_prefill_full():
-    """Varlen paged GQA prefill, causal, 16 seqs, L ~ U[64,4096], Hq=32, Hkv=8, D=128 (sampled rows)."""
+    """Varlen paged GQA prefill, causal, 16 seqs, L ~ U[64,4096], Hq=32, Hkv=8, D=128: the
+    longest sequence whole (every row, all 32 heads) and sampled rows of the others."""
     w = W.FULL_SIZE["varlen_paged_gqa_prefill_causal_bf16"]()
     t = w.tensors
     o, lse = _run_varlen(w, A.MASK_CAUSAL)
@@ -288,8 +287,21 @@ def test_config_varlen_paged_prefill_full():
     o = o.float().cpu().numpy()
     lse = lse.cpu().numpy()
     cu = t["cu_seqlens_q"].numpy()
+    lens = t["seqused_k"].numpy()
+    bl = int(np.argmax(lens))
+    L = int(lens[bl])
+    kc, vc, bt = _compact_pages(t["k_cache"], t["v_cache"], t["block_table"][bl], L)
+    o_ref, lse_ref = oracle.attn_varlen(t["q"][cu[bl]:cu[bl + 1]], kc, vc,
+                                        cu_seqlens_q=np.array([0, L], np.int32),
+                                        seqused_k=np.array([L], np.int32), block_table=bt,
+                                        num_heads_kv=8, scale=w.params["scale"], mask=1)
+    _cmp(torch.from_numpy(o[cu[bl]:cu[bl + 1]]), torch.from_numpy(lse[:, cu[bl]:cu[bl + 1]]),
+         o_ref, lse_ref, TOL_O_BF16, TOL_LSE_BF16,
+         "varlen prefill, whole sequence %d (%d rows)" % (bl, L))
     rng = np.random.default_rng(1)
     for b in range(16):
+        if b == bl:
+            continue
         L = cu[b + 1] - cu[b]
         for i in sorted(set([0, L - 1, int(rng.integers(0, L)), min(127, L - 1), min(128, L - 1)])):
             r = cu[b] + i
@@ -299,13 +311,31 @@ def test_config_varlen_paged_prefill_full():
             assert np.max(np.abs(lse[:, r] - lse_ref)) <= TOL_LSE_BF16, (b, i)
 
 
+def _patch_every_query_ref(t, scale):
+    """The oracle for every query of the patch workload: query q attends exactly the bytes
+    start_q <= j < end_q of its sequence, so with the keys of each patch as a sequence of
+    its own (patches partition the bytes in order) it is unmasked attention over them."""
+    cq = t["cu_seqlens_q"].numpy()
+    r = t["patch_kv_range"].numpy().astype(np.int64)
+    seq = np.repeat(np.arange(len(cq) - 1), np.diff(cq))
+    starts = seq * 8192 + r[:, 0]
+    ck = np.concatenate([starts, [starts[-1] + (r[-1, 1] - r[-1, 0])]]).astype(np.int32)
+    assert np.all(np.diff(ck) == r[:, 1] - r[:, 0])
+    return oracle.attn_varlen(t["q"], t["k"], t["v"],
+                              cu_seqlens_q=np.arange(len(r) + 1, dtype=np.int32),
+                              cu_seqlens_k=ck, num_heads_kv=16, scale=scale, mask=0)
+
+
 def test_config_patch_cross_attention_full():
-    """Patch cross-attention, B=4 x 8192 bytes, Geom(0.22) patches, H=16, D=64 (sampled queries)."""
+    """Patch cross-attention, B=4 x 8192 bytes, Geom(0.22) patches, H=16, D=64: every query
+    (tiled kernel), and sampled queries against the oracle's patch mask itself."""
     w = W.FULL_SIZE["patch_cross_attention_bf16"]()
     t = w.tensors
     o, lse = _run_varlen(w, A.MASK_PATCH, paged=False, patch=t["patch_kv_range"])
     torch.cuda.synchronize()
     _no_device_error()
+    o_all, lse_all = _patch_every_query_ref(t, w.params["scale"])
+    _cmp(o, lse, o_all, lse_all, TOL_O_BF16, TOL_LSE_BF16, "patch, every query")
     cq = t["cu_seqlens_q"].numpy()
     rng = np.random.default_rng(2)
     for b in range(4):
@@ -339,7 +369,16 @@ def test_config_fp8_dense_causal_full():
     rng = np.random.default_rng(3)
     o8, o16 = o8.float().cpu().numpy(), o16.float().cpu().numpy()
     lse8, lse16 = lse8.cpu().numpy(), lse16.cpu().numpy()
-    for b in range(4):
+    # batch element 0 whole (4096 rows x 16 heads), in fp8 and in bf16
+    for name, (qq, kk, vv), oo, ll, tol_o, tol_l in (
+            ("fp8", (qd, kd, vd), o8, lse8, TOL_O_FP8, None),
+            ("bf16", (t["q"], t["k"], t["v"]), o16, lse16, TOL_O_BF16, TOL_LSE_BF16)):
+        ref_o, ref_l = oracle.attn_dense(qq[0:1], kk[0:1], vv[0:1], scale=w.params["scale"],
+                                         causal=True)
+        assert np.max(np.abs(oo[0] - ref_o[0])) <= tol_o, (name, "whole batch element 0")
+        if tol_l is not None:
+            assert np.max(np.abs(ll[0] - ref_l[0])) <= tol_l, (name, "whole batch element 0")
+    for b in range(1, 4):
         for i in sorted(set([0, 1, 2, 127, 128, 4095, int(rng.integers(0, 4096))])):
             for name, (qq, kk, vv), oo, ll, tol_o, tol_l in (
                     ("fp8", (qd, kd, vd), o8, lse8, TOL_O_FP8, None),
@@ -374,21 +413,6 @@ def test_dense_fp8_small(L, causal, Hq, Hkv):
                                        oracle.dequant_e4m3(vf, dv), scale=w.params["scale"],
                                        causal=causal)
     _cmp(o, lse, o_ref, lse_ref, TOL_O_FP8, None, "fp8 dense L%d" % L)
-
-
-# ---------------------------------------------------------------------------- building blocks
-@pytest.mark.parametrize("degree,bound", [(3, 1.0e-4), (2, 2.0e-3)])
-def test_fma_pipe_exp2_error_bound(degree, bound):
-    """The softmax's polynomial exp2 stays within its fitted relative-error bound of 2^x."""
-    x = torch.linspace(-60.0, 8.0, 1 << 20, dtype=torch.float32)
-    y = A.attn_selftest_exp2(x.to(DEV), degree=degree).cpu().double()
-    ref = torch.exp2(x.double())
-    rel = ((y - ref).abs() / ref).max().item()
-    assert rel <= bound, rel
-    tiny = A.attn_selftest_exp2(torch.tensor([-float("inf"), -500.0, -125.5, -125.0], device=DEV),
-                                degree).cpu()
-    assert tiny[0] == 0 and tiny[1] == 0 and tiny[2] == 0     # masked scores contribute nothing
-    assert 0 < tiny[3] < 2.0 ** -124
 
 
 @pytest.mark.parametrize("Hq,Hkv", [(32, 8), (8, 4), (4, 1), (16, 8)])
