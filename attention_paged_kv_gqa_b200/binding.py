@@ -130,7 +130,7 @@ def attn_check_device(device: int = 0) -> int:
 def attn_device_error(stream=None) -> int:
     code = ctypes.c_int(0)
     st = lib().attn_device_error(ctypes.byref(code), _stream(stream))
-    if st not in (0, 7):
+    if st not in (0, 7, 9):
         _check(st, "attn_device_error")
     return code.value
 

@@ -58,12 +58,12 @@ __global__ void __launch_bounds__(kAppendThreads) kv_append_kernel(const AppendA
         const int p = __ldg(&a.seqused_k[b]) + (t - first);
         const int slot = p >= 0 ? p / kPageRows : -1;
         if (slot < 0 || slot >= a.max_blocks) {
-            if (lane == 0) record_error(kErrAppendSlot);
+            if (lane == 0) record_data_error(kErrAppendSlot);
             continue;
         }
         const int page = __ldg(&a.block_table[(long long)b * a.max_blocks + slot]);
         if (page < 0 || page >= a.num_blocks) {
-            if (lane == 0) record_error(kErrAppendPage);
+            if (lane == 0) record_data_error(kErrAppendPage);
             continue;
         }
         const uint4* __restrict__ ks = a.k_new + (long long)t * P;

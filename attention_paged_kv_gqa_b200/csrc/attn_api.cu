@@ -474,6 +474,7 @@ const char* attn_status_string(attn_status_t s) {
     case ATTN_ERR_CUDA: return "CUDA runtime error";
     case ATTN_ERR_DEVICE_TIMEOUT: return "a kernel gave up on a bounded wait";
     case ATTN_ERR_SCRATCH_LIMIT: return "request needs more than the library's fixed scratch (8 MiB)";
+    case ATTN_ERR_DEVICE_RANGE: return "a kernel met an index outside its buffers (block table entry or append position)";
     default: return "unknown status";
     }
 }
@@ -493,18 +494,26 @@ attn_status_t attn_device_error(int* code_out, attn_stream_t stream) {
     const attn_status_t dv = current_device_ok(nullptr);
     if (dv != ATTN_OK) return dv;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    int host = 0;
+    int wait_code = 0, data_code = 0;
     const int zero = 0;
-    if (cudaMemcpyFromSymbolAsync(&host, g_device_error, sizeof(int), 0, cudaMemcpyDeviceToHost, st) !=
-            cudaSuccess ||
+    if (cudaMemcpyFromSymbolAsync(&wait_code, g_device_error, sizeof(int), 0, cudaMemcpyDeviceToHost,
+                                  st) != cudaSuccess ||
+        cudaMemcpyFromSymbolAsync(&data_code, g_data_error, sizeof(int), 0, cudaMemcpyDeviceToHost,
+                                  st) != cudaSuccess ||
         cudaMemcpyToSymbolAsync(g_device_error, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, st) !=
+            cudaSuccess ||
+        cudaMemcpyToSymbolAsync(g_data_error, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, st) !=
             cudaSuccess ||
         cudaStreamSynchronize(st) != cudaSuccess) {
         cudaGetLastError();
         return ATTN_ERR_CUDA;
     }
-    *code_out = host;
-    return host == 0 ? ATTN_OK : ATTN_ERR_DEVICE_TIMEOUT;
+    if (wait_code != 0) {
+        *code_out = wait_code;
+        return ATTN_ERR_DEVICE_TIMEOUT;
+    }
+    *code_out = data_code;
+    return data_code == 0 ? ATTN_OK : ATTN_ERR_DEVICE_RANGE;
 }
 
 attn_status_t attn_selftest_wait_expiry(long long limit_ns, attn_stream_t stream) {
@@ -677,6 +686,7 @@ static attn_status_t fwd_varlen_paged_impl(
     a.seqused_k = seqused_k;
     a.block_table = block_table;
     a.max_blocks = max_blocks_per_seq;
+    a.num_blocks = num_blocks;
     a.patch = patch_kv_range;
     a.scale = resolve_scale(softmax_scale, D);
     a.descale_q = dq;
@@ -925,6 +935,7 @@ static attn_status_t decode_paged_impl(const void* q, const void* k_cache, const
         pa.q = static_cast<const __nv_bfloat16*>(q);
         pa.block_table = block_table;
         pa.max_blocks = max_blocks_per_seq;
+        pa.num_blocks = num_blocks;
         pa.seqused_k = seqused_k;
         pa.scale = resolve_scale(softmax_scale, D);
         pa.window = window;
@@ -958,6 +969,7 @@ static attn_status_t decode_paged_impl(const void* q, const void* k_cache, const
     a.q = static_cast<const __nv_bfloat16*>(q);
     a.block_table = block_table;
     a.max_blocks = max_blocks_per_seq;
+    a.num_blocks = num_blocks;
     a.seqused_k = seqused_k;
     a.tokens_per_split = tps;
     a.num_splits = ns;

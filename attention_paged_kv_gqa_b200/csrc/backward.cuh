@@ -52,6 +52,36 @@ enum : int {
     kErrBwdLoad = 601, kErrBwdMma = 602, kErrBwdCompute = 603, kErrBwdDrain = 604,
 };
 
+#ifndef ATTN_BWD_SEQ_MAJOR
+#define ATTN_BWD_SEQ_MAJOR 1
+#endif
+
+// Sequence-major unit order for a varlen batch of at most 32 sequences: the
+// sequences longest first (ties by index), each owning `my_units` consecutive
+// units (lane s of every warp describes sequence s: its length and unit count;
+// lanes >= B pass length -1 and 0 units).  The CTAs that run together then
+// work on one sequence, whose operand tiles they share in L2.  Gives the
+// sequence of unit `lin` and the unit's index inside it; false past the last
+// unit.  Every warp computes the same answer.
+__device__ __forceinline__ bool seq_major_unit(int lin, int B, int my_len, int my_units,
+                                               int* seq_out, int* local_out) {
+    const int lane = threadIdx.x & 31;
+    int start = 0;
+#pragma unroll 1
+    for (int o = 0; o < B; ++o) {
+        const int lo = __shfl_sync(0xffffffffu, my_len, o);
+        const int no = __shfl_sync(0xffffffffu, my_units, o);
+        start += (lo > my_len || (lo == my_len && o < lane)) ? no : 0;
+    }
+    const bool mine = lane < B && lin >= start && lin < start + my_units;
+    const unsigned hit = __ballot_sync(0xffffffffu, mine);
+    if (hit == 0u) return false;
+    const int src = __ffs(hit) - 1;
+    *seq_out = src;
+    *local_out = lin - __shfl_sync(0xffffffffu, start, src);
+    return true;
+}
+
 struct BwdArgs {
     int B, Hq, Hkv, group;
     int mask, window;          // window: causal only, < 0 none
@@ -148,11 +178,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    // unit: the query tile slowest and descending (causal units with more key tiles first)
-    const int bh = a.B * a.Hq;
-    const int qt = a.nqt - 1 - (int)(blockIdx.x / bh);
-    const int b = (int)(blockIdx.x % bh) / a.Hq;
-    const int h = (int)(blockIdx.x % bh) % a.Hq;
+    int qt, b, h;
+    if (ATTN_BWD_SEQ_MAJOR && a.B <= 32) {
+        // sequences longest first; in each, the query tile descending (causal tiles
+        // with more key tiles first), all heads of a tile side by side
+        const int len = lane < a.B ? a.cu_q[lane + 1] - a.cu_q[lane] : -1;
+        const int nqb = lane < a.B ? (max(len, 0) + 127) / 128 : 0;
+        int local;
+        if (!seq_major_unit((int)blockIdx.x, a.B, len, nqb * a.Hq, &b, &local)) return;
+        qt = __shfl_sync(0xffffffffu, nqb, b) - 1 - local / a.Hq;
+        h = local % a.Hq;
+    } else {
+        // the query tile slowest and descending (causal units with more key tiles first)
+        const int bh = a.B * a.Hq;
+        qt = a.nqt - 1 - (int)(blockIdx.x / bh);
+        b = (int)(blockIdx.x % bh) / a.Hq;
+        h = (int)(blockIdx.x % bh) % a.Hq;
+    }
     const int g = h / a.group;
     const int q_off = a.cu_q[b], Lq = a.cu_q[b + 1] - q_off;
     const int k_off = a.cu_k[b], Lk = max(a.cu_k[b + 1] - k_off, 0);
@@ -220,10 +262,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 }
             }
             // every copy started must land before the CTA can exit
-            mbar_wait(q_full, 0, kErrBwdDrain);
+            mbar_wait_drain(q_full, 0, kErrBwdDrain);
             for (int st = 0; st < NS && st < issued; ++st) {
                 const int last = st + ((issued - 1 - st) / NS) * NS;
-                mbar_wait(&kv_full[st], (last / NS) & 1, kErrBwdDrain);
+                mbar_wait_drain(&kv_full[st], (last / NS) & 1, kErrBwdDrain);
             }
         }
     } else if (warp == kBwdMmaWarp) {
@@ -282,7 +324,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 mma_commit(&kv_empty[st]);
             }
             mma_commit(mma_done);
-            mbar_wait(mma_done, 0, kErrBwdMma);
+            mbar_wait_drain(mma_done, 0, kErrBwdMma);
         }
     } else {
         // ---------------------------------------------------- compute warpgroups: dS, then dQ out
@@ -410,11 +452,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     auto stDl = [&](int st) { return stL(st) + 128; };
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    // unit: key tile slowest (ascending: causal key tiles near the start see the most queries)
-    const int bg = a.B * a.Hkv;
-    const int kt = (int)(blockIdx.x / bg);
-    const int b = (int)(blockIdx.x % bg) / a.Hkv;
-    const int g = (int)(blockIdx.x % bg) % a.Hkv;
+    int kt, b, g;
+    if (ATTN_BWD_SEQ_MAJOR && a.B <= 32) {
+        // sequences longest first; in each, the key tile ascending (causal key tiles
+        // near the start see the most queries), all KV heads of a tile side by side
+        const int len = lane < a.B ? a.cu_k[lane + 1] - a.cu_k[lane] : -1;
+        const int nkb = lane < a.B ? (max(len, 0) + 127) / 128 : 0;
+        int local;
+        if (!seq_major_unit((int)blockIdx.x, a.B, len, nkb * a.Hkv, &b, &local)) return;
+        kt = local / a.Hkv;
+        g = local % a.Hkv;
+    } else {
+        // key tile slowest (ascending: causal key tiles near the start see the most queries)
+        const int bg = a.B * a.Hkv;
+        kt = (int)(blockIdx.x / bg);
+        b = (int)(blockIdx.x % bg) / a.Hkv;
+        g = (int)(blockIdx.x % bg) % a.Hkv;
+    }
     const int q_off = a.cu_q[b], Lq = a.cu_q[b + 1] - q_off;
     const int k_off = a.cu_k[b], Lk = max(a.cu_k[b + 1] - k_off, 0);
     const int k0 = kt * 128;
@@ -505,10 +559,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 }
             }
             if (lane == 0) {
-                mbar_wait(kv_full, 0, kErrBwdDrain);
+                mbar_wait_drain(kv_full, 0, kErrBwdDrain);
                 for (int st = 0; st < NS && st < issued; ++st) {
                     const int last = st + ((issued - 1 - st) / NS) * NS;
-                    mbar_wait(&st_full[st], (last / NS) & 1, kErrBwdDrain);
+                    mbar_wait_drain(&st_full[st], (last / NS) & 1, kErrBwdDrain);
                 }
             }
         }
@@ -548,7 +602,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 mma_commit(&st_empty[st]);
             }
             mma_commit(mma_done);
-            mbar_wait(mma_done, 0, kErrBwdMma);
+            mbar_wait_drain(mma_done, 0, kErrBwdMma);
         }
     } else {
         // ---------------------------------------------------- compute warpgroups (thread = key)
@@ -589,7 +643,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 tmem_ld32(tST + lane_off + c4 * 32, us);
                 tmem_ld32(tdPT + lane_off + c4 * 32, ud);
                 tmem_wait_ld();
-                uint32_t pp[16], dd[16];
+                uint32_t pp[8], dd[8];   // one half (8 words = 16 columns) of the block's results
                 float4 lv, dv;   // 4 rows of LSE (base 2) and Delta, broadcast from shared memory
 #pragma unroll
                 for (int c = 0; c < 16; ++c) {
@@ -617,12 +671,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     }
                     const float2 dp = fadd2(make_float2(__uint_as_float(ud[2 * c]), __uint_as_float(ud[2 * c + 1])), nd);
                     const float2 ds = fmul2(p, fmul2(dp, make_float2(a.scale, a.scale)));
-                    pp[c] = pack_bf16(p.x, p.y);
-                    dd[c] = pack_bf16(ds.x, ds.y);
+                    pp[c & 7] = pack_bf16(p.x, p.y);
+                    dd[c & 7] = pack_bf16(ds.x, ds.y);
+                    if ((c & 7) == 7) {
+                        // block c4, half c / 8 -> columns this warpgroup has already read
+                        tmem_st8(tST + lane_off + bwd_out_col(c4) + (c & 8), pp);
+                        tmem_st8(tdPT + lane_off + bwd_out_col(c4) + (c & 8), dd);
+                    }
                 }
-                // block c4 -> columns this warpgroup has already read
-                tmem_st16(tST + lane_off + bwd_out_col(c4), pp);
-                tmem_st16(tdPT + lane_off + bwd_out_col(c4), dd);
             }
             tmem_wait_st();
             tc_fence_before();

@@ -34,6 +34,7 @@ struct DecodeArgs {
     const __nv_bfloat16* q;   // [B][Hq][D]
     const int* block_table;
     int max_blocks;
+    int num_blocks;           // pages in the cache: entries outside [0, num_blocks) are errors
     const int* seqused_k;
     int tokens_per_split;     // multiple of kDecStageTok
     int num_splits;
@@ -217,6 +218,10 @@ __global__ void __launch_bounds__(kDecThreads, 2)
                     const int slot = slot0 + w * 32 + lane;
                     pg = (slot * kPageRows < it.t_end && slot < a.max_blocks)
                              ? a.block_table[(long long)it.b * a.max_blocks + slot] : 0;
+                    if (pg < 0 || pg >= a.num_blocks) {
+                        record_data_error(kErrDecPageRange);   // outside the cache: reported, page 0 read
+                        pg = 0;
+                    }
                 }
                 int pages[4];
 #pragma unroll
@@ -251,7 +256,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
         if (lane == 0) {
             for (int st = 0; st < NS && st < ctr; ++st) {
                 const int last = st + ((ctr - 1 - st) / NS) * NS;
-                mbar_wait(&full[st], (last / NS) & 1, kErrDecFull);
+                mbar_wait_drain(&full[st], (last / NS) & 1, kErrDecFull);
             }
         }
     } else {
@@ -467,6 +472,7 @@ struct DecodePagesArgs {
     const __nv_bfloat16* q;   // [B][Hq][D]
     const int* block_table;
     int max_blocks;
+    int num_blocks;           // pages in the cache: entries outside [0, num_blocks) are errors
     const int* seqused_k;
     float scale;
     int window;               // sliding window: keys L-1-window .. L-1; < 0: none
@@ -577,6 +583,10 @@ __global__ void __launch_bounds__(32 * (kPgMaxWarps + 1), 1)
                 const int b = seq_of(g);
                 const int slot = g - prefix[b] + win_first_page_key(lenv[b], a.window) / kPageRows;
                 phys = a.block_table[(long long)b * a.max_blocks + slot];
+                if (phys < 0 || phys >= a.num_blocks) {
+                    record_data_error(kErrDecPageRange);   // outside the cache: reported, page 0 read
+                    phys = 0;
+                }
             }
             const int cnt = min(32, npages - base);
             bool ok = true;
@@ -603,7 +613,7 @@ __global__ void __launch_bounds__(32 * (kPgMaxWarps + 1), 1)
         if (lane == 0) {
             for (int st = 0; st < NS && st < issued; ++st) {
                 const int last = st + ((issued - 1 - st) / NS) * NS;
-                mbar_wait(&full[st], (last / NS) & 1, kErrDecFull);
+                mbar_wait_drain(&full[st], (last / NS) & 1, kErrDecFull);
             }
         }
     } else if (warp < Hkv) {

@@ -48,6 +48,7 @@ enum : int {
     kErrSmS = 301, kErrSmV = 302, kErrSmO = 303,
     kErrDecFull = 401, kErrDecEmpty = 402,
     kErrSelftestWait = 901,
+    kErrPageRange = 111, kErrDecPageRange = 411,   // a block_table entry outside the cache
 };
 
 struct PrefillArgs {
@@ -64,6 +65,7 @@ struct PrefillArgs {
     const int* seqused_k;
     const int* block_table;
     int max_blocks;
+    int num_blocks;      // pages in the cache (paged): entries outside [0, num_blocks) are errors
     const int* patch;    // [total_q][2] sequence-local [start, end)
     float scale;         // softmax scale (natural units)
     const float* descale_q;
@@ -193,7 +195,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         // Block-sparse tile range of each sub-tile from its rows' key intervals.
         const int t = warp >> 2;
         const int r = (warp & 3) * 32 + lane;
-        const int qi = q0[t] + r;
+        const int qi = (t ? q0[1] : q0[0]) + r;   // (a select: no dynamically indexed array)
         int s = 0x7fffffff, e = -0x7fffffff;
         if (qi < Lq) {
             const int rs = max(a.patch[2LL * (q_off + qi)], 0);
@@ -306,8 +308,14 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                 constexpr int PPT = kBN / kPageRows;   // pages per tile
                 if (a.paged && lane < PPT) {
                     const int slot = j * PPT + lane;
-                    if (slot * kPageRows < Lk && slot < a.max_blocks)
+                    if (slot * kPageRows < Lk && slot < a.max_blocks) {
                         page = a.block_table[(long long)b * a.max_blocks + slot];
+                        if (page < 0 || page >= a.num_blocks) {
+                            // outside the cache: reported, and a page inside it read instead
+                            record_data_error(kErrPageRange);
+                            page = 0;
+                        }
+                    }
                 }
                 int npv = 0;
 #pragma unroll
@@ -366,8 +374,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                 for (int st = 0; st < vring && st < issued; ++st) {
                     const int last = st + ((issued - 1 - st) / vring) * vring;
                     const uint32_t ph = (last / vring) & 1;
-                    if (!OQ) mbar_wait(&k_full[st], ph, kErrProdDrain);
-                    mbar_wait(vslot_full(st), ph, kErrProdDrain);
+                    if (!OQ) mbar_wait_drain(&k_full[st], ph, kErrProdDrain);
+                    mbar_wait_drain(vslot_full(st), ph, kErrProdDrain);
                 }
             }
         }
@@ -457,7 +465,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             }
             // All MMAs this thread issued must finish before TMEM is released.
             mma_commit(mma_done);
-            mbar_wait(mma_done, 0, kErrMmaDone);
+            mbar_wait_drain(mma_done, 0, kErrMmaDone);
         }
     } else {
         // -------------------------------------------------------- softmax warpgroups (a5, a7)
@@ -467,9 +475,13 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
         const uint32_t tS = tbase + lane_off + t * 128;
         const uint32_t tO = tbase + lane_off + 256 + t * D;
-        const int qi = q0[t] + r;
+        // This sub-tile's values as scalars (selects, so that the small per-sub-tile
+        // arrays stay in registers instead of on the stack).
+        const int lo_mine = t ? lo_t[1] : lo_t[0];
+        const int hi_mine = t ? hi_t[1] : hi_t[0];
+        const int qi = (t ? q0[1] : q0[0]) + r;
         const bool row_ok = (t == 0 ? valid0 : valid1) && qi < Lq;
-        const int head_t = head[t];
+        const int head_t = t ? head[1] : head[0];
         float sl2 = a.scale * kLog2e;
         float eff = a.scale;                 // logit = eff * (raw dot product)
         float out_scale = 1.0f;
@@ -496,10 +508,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         if (!row_ok) { klo = 0; khi = Lk; }
 
         float m_run = -INFINITY, l_run = 0.0f;
-        const int n_t = hi_t[t] - lo_t[t];
+        const int n_t = hi_mine - lo_mine;
         bool ok = true;
         for (int jj = 0; jj < n_t; ++jj) {
-            const int j = lo_t[t] + jj;
+            const int j = lo_mine + jj;
             ok = mbar_wait(&s_full[t], jj & 1, kErrSmS);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;

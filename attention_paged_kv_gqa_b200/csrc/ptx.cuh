@@ -19,9 +19,14 @@
 
 namespace attn {
 
-// Device error word: 0 = fine, otherwise the code of the first wait that gave up.
-// (The library is one translation unit, so the definition lives here.)
+// Device error words (the library is one translation unit, so the definitions
+// live here).  g_device_error: 0 = fine, otherwise the code of the first wait
+// that gave up; while it is set, the other waits give up early.
+// g_data_error: the code of the first out-of-range index a kernel met (a block
+// table entry outside the cache, an append position past the block table); the
+// kernel carries on with a safe substitute and nothing else stops.
 __device__ int g_device_error = 0;
+__device__ int g_data_error = 0;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -35,6 +40,10 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 
 __device__ __forceinline__ void record_error(int code) {
     atomicCAS(&g_device_error, 0, code);
+}
+
+__device__ __forceinline__ void record_data_error(int code) {
+    atomicCAS(&g_data_error, 0, code);
 }
 
 __device__ __forceinline__ bool error_flagged() {
@@ -99,6 +108,24 @@ __device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity, in
 // The kernels' wait: bounded by ATTN_WAIT_LIMIT_NS.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int code) {
     return mbar_wait_for(bar, parity, code, ATTN_WAIT_LIMIT_NS);
+}
+
+// The wait for this CTA's own asynchronous work (TMA copies, tensor-core ops)
+// before it leaves: bounded by ATTN_WAIT_LIMIT_NS only -- it does not give up
+// early when another CTA has recorded an error, since that work completes on
+// its own and must land before the CTA's shared memory and TMEM are released.
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, int code) {
+    const uint32_t a = smem_u32(bar);
+    if (mbar_try_wait(a, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    uint32_t spins = 0;
+    while (true) {
+        if (mbar_try_wait(a, parity)) return true;
+        if ((++spins & 63u) == 0 && globaltimer_ns() - t0 > ATTN_WAIT_LIMIT_NS) {
+            record_error(code);
+            return false;
+        }
+    }
 }
 
 // Makes generic-proxy shared-memory writes visible to the async proxy (TMA, tcgen05).

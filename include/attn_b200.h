@@ -80,7 +80,8 @@ typedef enum {
     ATTN_ERR_WORKSPACE_TOO_SMALL = 5,
     ATTN_ERR_CUDA = 6,               /* a CUDA runtime call or a launch failed */
     ATTN_ERR_DEVICE_TIMEOUT = 7,     /* a kernel gave up on a bounded wait (see attn_device_error) */
-    ATTN_ERR_SCRATCH_LIMIT = 8       /* attn_decode_paged_noalloc: needs more than its fixed scratch */
+    ATTN_ERR_SCRATCH_LIMIT = 8,      /* attn_decode_paged_noalloc: needs more than its fixed scratch */
+    ATTN_ERR_DEVICE_RANGE = 9        /* a kernel met an out-of-range index (see attn_device_error) */
 } attn_status_t;
 
 typedef enum { ATTN_MASK_NONE = 0, ATTN_MASK_CAUSAL = 1, ATTN_MASK_PATCH = 2 } attn_mask_t;
@@ -102,9 +103,18 @@ attn_status_t attn_check_device(int device);
 const char *attn_status_string(attn_status_t status);
 
 /*
- * Reads and clears the device-side error word of the current device: 0 when
- * no kernel gave up on a bounded wait since the last read, otherwise a code
- * naming the wait.  Synchronises `stream` (a debugging aid, not for hot loops).
+ * Reads and clears the two device-side error words of the current device and
+ * synchronises `stream` (a debugging aid, not for hot loops).
+ *   - A kernel gave up on a bounded wait since the last read: returns
+ *     ATTN_ERR_DEVICE_TIMEOUT, *code_out names the wait (101..303 forward,
+ *     401..402 decode, 601..604 backward, 901 the test hook below).  While that
+ *     word is set, the other kernels' waits give up early.
+ *   - Otherwise, a kernel met an index outside its buffers: returns
+ *     ATTN_ERR_DEVICE_RANGE, *code_out names it (111 forward and 411 decode: a
+ *     block_table entry outside [0, num_blocks), page 0 read in its place;
+ *     501/502 KV append: a position past the block table / a page outside the
+ *     cache, that token not written).  Nothing else stops on these.
+ *   - Neither: ATTN_OK and *code_out = 0.
  */
 attn_status_t attn_device_error(int *code_out, attn_stream_t stream);
 
@@ -155,8 +165,9 @@ attn_status_t attn_fwd_dense(
  *   patch_kv_range int32 [total_q, 2], PATCH only: per-query [start, end).
  *   o            [total_q, Hq, D] bf16.   lse [Hq, total_q] fp32 or NULL.
  *   workspace    unused by this version; may be NULL with workspace_bytes 0.
- * Page indices outside [0, num_blocks) read zeros (TMA bounds fill); the
- * caller must keep block_table entries for the used pages valid.
+ * A used block_table entry outside [0, num_blocks) is a caller error: the
+ * kernel reads page 0 in its place and records code 111 for attn_device_error
+ * (ATTN_ERR_DEVICE_RANGE); the decode calls do the same with code 411.
  */
 attn_status_t attn_fwd_varlen_paged(
     const void *q, const void *k_cache, const void *v_cache,
@@ -280,7 +291,8 @@ attn_status_t attn_decode_paged_only_qv(
  * different sequences must map to different cache rows.  A position past a
  * sequence's block table, or a page index outside [0, num_blocks), is not
  * written: the kernel records code 501 (position) or 502 (page) in the device
- * error word (attn_device_error) and copies the remaining tokens.
+ * data-error word (attn_device_error reports ATTN_ERR_DEVICE_RANGE) and copies
+ * the remaining tokens.
  */
 attn_status_t attn_kv_append_paged(
     const void *k_new, const void *v_new, void *k_cache, void *v_cache,

@@ -40,7 +40,7 @@ def test_every_declared_symbol_is_exported(L):
 
 
 def test_status_strings(L):
-    for s in range(0, 8):
+    for s in range(0, 10):
         assert binding.status_string(s)
     assert binding.status_string(0) == "ok"
 
