@@ -95,3 +95,26 @@ def test_config_patch_cross_full_cuda_cores():
                                   t["patch_kv_range"], 16, 16, w.params["scale"],
                                   w.params["max_seqlen_q"])
     _cmp(o, lse, o_ref, lse_ref, "patch full")
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("Hq,Hkv", [(8, 2), (4, 4), (8, 8), (16, 16)])
+def test_patch_short_intervals_ragged(D, Hq, Hkv):
+    """Intervals of at most 16 keys through attn_fwd_patch: GQA; empty, one-key and clipped
+    intervals; starts out of order and overlapping; sequences with no queries or no keys."""
+    rng = np.random.default_rng(100 + D + Hq)
+    lens_q, lens_k = [0, 37, 5, 120, 1, 64, 9], [10, 100, 0, 700, 16, 90, 40]
+    cq, ck = W.cu_from_lens(lens_q), W.cu_from_lens(lens_k)
+    rows = []
+    for b in range(len(lens_q)):
+        for i in range(lens_q[b]):
+            s0 = int(rng.integers(-3, lens_k[b] + 3))
+            n = int(rng.choice([0, 1, 2, 7, 15, 16]))
+            rows.append((s0, s0 + n))
+    ranges = torch.tensor(rows, dtype=torch.int32).reshape(-1, 2)
+    q = W.randn_bf16((int(cq[-1]), Hq, D), 5, 1)
+    k = W.randn_bf16((int(ck[-1]), Hkv, D), 5, 2)
+    v = W.randn_bf16((int(ck[-1]), Hkv, D), 5, 3)
+    o, lse, o_ref, lse_ref = _run(q, k, v, cq, ck, ranges, Hkv, 16, 0.15, max(lens_q))
+    _cmp(o, lse, o_ref, lse_ref, "patch short D%d Hq%d Hkv%d" % (D, Hq, Hkv))
+
