@@ -251,12 +251,15 @@ def attn_decode_workspace_size(B, num_heads_q, num_heads_kv, head_dim, max_block
 
 
 def attn_decode_paged(q, k_cache, v_cache, block_table, seqused_k, *, scale=None, num_splits=0,
-                      window_left=-1, softcap=0.0, out=None, lse=None, workspace=None,
-                      return_lse=True, stream=None):
+                      window_left=-1, softcap=0.0, descale_q=None, descale_k=None,
+                      descale_v=None, out=None, lse=None, workspace=None, return_lse=True,
+                      stream=None):
     """q [B, Hq, D] against a paged cache -> (o [B, Hq, D] bf16, lse [B, Hq] fp32).
 
     The query is the newest cached token; window_left >= 0 keeps the keys
     L-1-window_left .. L-1; softcap > 0 caps the logits as in the prefill calls.
+    With q and the cache in float8_e4m3fn, descale_q/k/v ([Hkv] fp32 each) are
+    required (head_dim 128, automatic split).
     """
     B, Hq, D = q.shape
     num_blocks, block_size, Hkv = k_cache.shape[0], k_cache.shape[1], k_cache.shape[2]
@@ -271,7 +274,7 @@ def attn_decode_paged(q, k_cache, v_cache, block_table, seqused_k, *, scale=None
     st = lib().attn_decode_paged(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), mbps,
                                  num_blocks, block_size, _ptr(seqused_k), B, Hq, Hkv, D,
                                  _scale(scale), int(window_left), float(softcap), int(num_splits),
-                                 _dtype_code(q), None, None, None,
+                                 _dtype_code(q), _ptr(descale_q), _ptr(descale_k), _ptr(descale_v),
                                  _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(),
                                  _stream(stream))
     _check(st, "attn_decode_paged")

@@ -386,7 +386,7 @@ void* noalloc_scratch_address(int dev) {
     return p;
 }
 
-template <int D>
+template <int D, bool FP8>
 attn_status_t launch_decode_pages(const CUtensorMap& mk, const CUtensorMap& mv, const DecodePagesArgs& a,
                                   int grid, cudaStream_t st, __nv_bfloat16* o, float* lse,
                                   bool pdl = false) {
@@ -395,12 +395,12 @@ attn_status_t launch_decode_pages(const CUtensorMap& mk, const CUtensorMap& mv, 
     cudaGetDevice(&dev);
     const uint64_t bit = 1ull << (dev & 63);
     if (!(attr_mask.load() & bit)) {
-        const attn_status_t s = set_smem(decode_pages_kernel<D>, 227 * 1024);
+        const attn_status_t s = set_smem(decode_pages_kernel<D, FP8>, 227 * 1024);
         if (s != ATTN_OK) return s;
         attr_mask.fetch_or(bit);
     }
-    const int smem = DecodePagesCfg<D>::smem_bytes(a.Hkv, a.B, a.nstages, a.only_qv != 0);
-    attn_status_t s = launch_maybe_pdl(decode_pages_kernel<D>, dim3(grid), dim3(32 * (a.Hkv + 1)),
+    const int smem = DecodePagesCfg<D, FP8>::smem_bytes(a.Hkv, a.B, a.nstages, a.only_qv != 0);
+    attn_status_t s = launch_maybe_pdl(decode_pages_kernel<D, FP8>, dim3(grid), dim3(32 * (a.Hkv + 1)),
                                        smem, st, pdl, mk, mv, a);
     if (s != ATTN_OK) return s;
     cudaLaunchConfig_t cfg;
@@ -819,11 +819,13 @@ static void decode_splits(int B, int Hkv, int max_tokens, int requested, int* nu
     *num_splits = (max_tokens + t - 1) / t;
 }
 
-static int decode_pages_stages(int D, int Hkv, int B, bool vonly = false) {
+static int decode_pages_stages(int D, int Hkv, int B, bool vonly = false, bool fp8 = false) {
     const int cap = 227 * 1024;
-    const int max_ns = vonly ? 16 : 8;      // V-only stages are half as large: twice as many
+    const int max_ns = (vonly || fp8) ? 16 : 8;   // V-only or e4m3 stages are half as large
     int ns = 0;
-    if (D == 128)
+    if (fp8)
+        while (ns < max_ns && DecodePagesCfg<128, true>::smem_bytes(Hkv, B, ns + 1, vonly) <= cap) ++ns;
+    else if (D == 128)
         while (ns < max_ns && DecodePagesCfg<128>::smem_bytes(Hkv, B, ns + 1, vonly) <= cap) ++ns;
     else
         while (ns < max_ns && DecodePagesCfg<64>::smem_bytes(Hkv, B, ns + 1, vonly) <= cap) ++ns;
@@ -873,9 +875,6 @@ static attn_status_t decode_paged_impl(const void* q, const void* k_cache, const
                                        const float* dq, const float* dk, const float* dv, void* o,
                                        float* lse, void* workspace, size_t workspace_bytes,
                                        attn_stream_t stream, bool pdl, int only_qv = 0) {
-    (void)dq;
-    (void)dk;
-    (void)dv;
     if (!q || !k_cache || !v_cache || !block_table || !seqused_k || !o) return ATTN_ERR_INVALID_ARG;
     {
         // the query is the newest token: the window is a causal one by construction
@@ -886,13 +885,20 @@ static attn_status_t decode_paged_impl(const void* q, const void* k_cache, const
     if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
     if (num_blocks <= 0 || max_blocks_per_seq <= 0) return ATTN_ERR_INVALID_ARG;
     if (!dtype_ok(dtype)) return ATTN_ERR_INVALID_ARG;
-    if (dtype != ATTN_BF16) return ATTN_ERR_UNSUPPORTED;
+    const bool fp8 = dtype == ATTN_FP8_E4M3;
+    if (fp8) {
+        // e4m3 q and cache: the page-stream decode (automatic split), head_dim 128
+        if (only_qv) return ATTN_ERR_UNSUPPORTED;
+        if (!dq || !dk || !dv) return ATTN_ERR_INVALID_ARG;
+        if (D != 128 || num_splits > 0) return ATTN_ERR_UNSUPPORTED;
+    }
     if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
     if (block_size != kPageRows) return ATTN_ERR_UNSUPPORTED;
     if (Hq / Hkv > kDecRows) return ATTN_ERR_UNSUPPORTED;
     if (B > kDecMaxSeqs) return ATTN_ERR_UNSUPPORTED;
     if ((long long)num_blocks * block_size >= (1LL << 31)) return ATTN_ERR_UNSUPPORTED;
     if ((long long)max_blocks_per_seq * block_size >= (1LL << 30)) return ATTN_ERR_UNSUPPORTED;
+    if (fp8 && !use_page_stream(B, Hq, Hkv, D, num_splits)) return ATTN_ERR_UNSUPPORTED;
     if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o))
         return ATTN_ERR_INVALID_ARG;
     int ns, tps;
@@ -913,14 +919,15 @@ static attn_status_t decode_paged_impl(const void* q, const void* k_cache, const
     if (use_page_stream(B, Hq, Hkv, D, num_splits)) {
         // {d, token, head, page} view: one box = a whole page's 128-byte column
         CUtensorMap pk, pv;
-        const uint64_t rowk = (uint64_t)Hkv * D * 2;
+        const int E = elem_bytes(dtype);
+        const uint64_t rowk = (uint64_t)Hkv * D * E;
         const uint64_t pd[4] = {(uint64_t)D, (uint64_t)kPageRows, (uint64_t)Hkv, (uint64_t)num_blocks};
-        const uint64_t ps[3] = {rowk, (uint64_t)D * 2, rowk * kPageRows};
-        const uint32_t pbox[4] = {64, (uint32_t)kPageRows, (uint32_t)Hkv, 1};
+        const uint64_t ps[3] = {rowk, (uint64_t)D * E, rowk * kPageRows};
+        const uint32_t pbox[4] = {(uint32_t)(128 / E), (uint32_t)kPageRows, (uint32_t)Hkv, 1};
         attn_status_t s;
-        if ((s = get_map(&pv, v_cache, ATTN_BF16, pd, ps, pbox)) != ATTN_OK) return s;
+        if ((s = get_map(&pv, v_cache, dtype, pd, ps, pbox)) != ATTN_OK) return s;
         if (only_qv) pk = pv;   // no key store: its map is never used
-        else if ((s = get_map(&pk, k_cache, ATTN_BF16, pd, ps, pbox)) != ATTN_OK) return s;
+        else if ((s = get_map(&pk, k_cache, dtype, pd, ps, pbox)) != ATTN_OK) return s;
         const int grid = sm_count(dev);
         const size_t slots = (size_t)grid + B;
         const size_t need_pg = slots * Hq * (D + 1) * sizeof(float) + (size_t)(B + 2) * sizeof(int);
@@ -932,7 +939,10 @@ static attn_status_t decode_paged_impl(const void* q, const void* k_cache, const
         pa.Hq = Hq;
         pa.Hkv = Hkv;
         pa.group = Hq / Hkv;
-        pa.q = static_cast<const __nv_bfloat16*>(q);
+        pa.q = q;
+        pa.descale_q = dq;
+        pa.descale_k = dk;
+        pa.descale_v = dv;
         pa.block_table = block_table;
         pa.max_blocks = max_blocks_per_seq;
         pa.num_blocks = num_blocks;
@@ -943,11 +953,13 @@ static attn_status_t decode_paged_impl(const void* q, const void* k_cache, const
         pa.o_part = static_cast<float*>(workspace);
         pa.lse_part = pa.o_part + slots * Hq * D;
         pa.meta = reinterpret_cast<int*>(pa.lse_part + slots * Hq);
-        pa.nstages = decode_pages_stages(D, Hkv, B, only_qv != 0);
+        pa.nstages = decode_pages_stages(D, Hkv, B, only_qv != 0, fp8);
         pa.only_qv = only_qv ? 1 : 0;
+        if (fp8)
+            return launch_decode_pages<128, true>(pk, pv, pa, grid, stp, static_cast<__nv_bfloat16*>(o), lse, pdl);
         if (D == 128)
-            return launch_decode_pages<128>(pk, pv, pa, grid, stp, static_cast<__nv_bfloat16*>(o), lse, pdl);
-        return launch_decode_pages<64>(pk, pv, pa, grid, stp, static_cast<__nv_bfloat16*>(o), lse, pdl);
+            return launch_decode_pages<128, false>(pk, pv, pa, grid, stp, static_cast<__nv_bfloat16*>(o), lse, pdl);
+        return launch_decode_pages<64, false>(pk, pv, pa, grid, stp, static_cast<__nv_bfloat16*>(o), lse, pdl);
     }
 
     const uint64_t rowk = (uint64_t)Hkv * D * 2;

@@ -469,7 +469,10 @@ constexpr int kPgMaxWarps = 8;         // consumer warps (KV heads) of the page-
 
 struct DecodePagesArgs {
     int B, Hq, Hkv, group;
-    const __nv_bfloat16* q;   // [B][Hq][D]
+    const void* q;            // [B][Hq][D] bf16, or e4m3 (the FP8 instance)
+    const float* descale_q;   // FP8: device fp32 scalars (real value = code x descale)
+    const float* descale_k;
+    const float* descale_v;
     const int* block_table;
     int max_blocks;
     int num_blocks;           // pages in the cache: entries outside [0, num_blocks) are errors
@@ -484,10 +487,12 @@ struct DecodePagesArgs {
     int only_qv;              // 1: score = q . v (no K loads; the score reads the V rows)
 };
 
-template <int D>
+template <int D, bool FP8 = false>
 struct DecodePagesCfg {
-    static constexpr int ROWB = D * 2;
-    static constexpr int NCHUNK = ROWB / 128;
+    static constexpr int E = FP8 ? 1 : 2;               // bytes per element
+    static constexpr int ROWB = D * E;
+    static constexpr int NCHUNK = ROWB / 128;           // 128-byte swizzle columns per row
+    static constexpr int CHUNK_E = 128 / E;             // elements per swizzle column
     // stage = one page of K and V for all heads: 2 * 16 * Hkv * D * 2 bytes (half: V alone,
     // for the only_qv score)
     __host__ __device__ static constexpr int stage_bytes(int Hkv, bool vonly = false) {
@@ -499,11 +504,19 @@ struct DecodePagesCfg {
     }
 };
 
-template <int D>
+// FP8: the cache (and q) hold e4m3 codes with per-tensor descales.  Pages
+// arrive half as large; the consumers turn the codes into f16 in registers
+// (exact) and contract with the f16 warp MMA, the descales folded into the score
+// scale and the output.  For Q.K^T the contraction index is permuted alike in
+// q and k, so that each lane's non-transposed ldmatrix word (4 consecutive key
+// bytes) is its B fragment; for P.V a transposed ldmatrix word holds 2 keys x 2
+// columns, split by a byte permute into the fragments of two 8-column tiles
+// (even and odd columns of a 16-column block).
+template <int D, bool FP8>
 __global__ void __launch_bounds__(32 * (kPgMaxWarps + 1), 1)
     decode_pages_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                         const DecodePagesArgs a) {
-    using C = DecodePagesCfg<D>;
+    using C = DecodePagesCfg<D, FP8>;
     const int NS = a.nstages;
     const int Hkv = a.Hkv, G = a.group;
     const int SB = C::stage_bytes(Hkv, a.only_qv);          // K and V of a page, or V alone
@@ -603,8 +616,10 @@ __global__ void __launch_bounds__(32 * (kPgMaxWarps + 1), 1)
 #pragma unroll
                     for (int c = 0; c < C::NCHUNK; ++c) {
                         if (!a.only_qv)
-                            tma_load_4d_hint(&tmK, &full[st], dk + c * rows * 128, c * 64, 0, 0, page, pol);
-                        tma_load_4d_hint(&tmV, &full[st], dv + c * rows * 128, c * 64, 0, 0, page, pol);
+                            tma_load_4d_hint(&tmK, &full[st], dk + c * rows * 128, c * C::CHUNK_E, 0, 0,
+                                             page, pol);
+                        tma_load_4d_hint(&tmV, &full[st], dv + c * rows * 128, c * C::CHUNK_E, 0, 0, page,
+                                         pol);
                     }
                 }
             }
@@ -620,27 +635,50 @@ __global__ void __launch_bounds__(32 * (kPgMaxWarps + 1), 1)
         // ------------------------------------------------------------ consumer warp = KV head
         const int h = warp;
         const int gid = lane >> 2, t4 = lane & 3;
-        const float sl2 = a.scale * kLog2e;
+        // logit = eff * (raw dot product); FP8: the raw dot product is of the codes
+        float eff = a.scale, out_scale = 1.0f;
+        if constexpr (FP8) {
+            eff *= __ldg(a.descale_q) * __ldg(a.descale_k);
+            out_scale = __ldg(a.descale_v);
+        }
+        const float sl2 = eff * kLog2e;
         const bool capped = a.softcap > 0.0f;
-        const float cap_in = capped ? a.scale / a.softcap : 0.0f;
-        const float cap_out = capped ? a.softcap / a.scale : 0.0f;
+        const float cap_in = capped ? eff / a.softcap : 0.0f;
+        const float cap_out = capped ? a.softcap / eff : 0.0f;
         uint32_t qa[D / 16][4];
         float o[D / 8][4];
         float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.0f, l1 = 0.0f;
         int b = -1, b_end = 0, L = 0, kb = 0, kf = 0;
         auto load_q = [&](int bb) {
-            const __nv_bfloat16* qb = a.q + ((long long)bb * a.Hq + (long long)h * G) * D;
+            if constexpr (FP8) {
+                // A fragment of 16-column block s: the contraction index permuted so that
+                // logical k = 2 t4 + j is column 16 s + 4 t4 + j and k = 2 t4 + 8 + j is
+                // column 16 s + 4 t4 + 2 + j (matching the K words below)
+                const uint8_t* qb = static_cast<const uint8_t*>(a.q) + ((long long)bb * a.Hq + (long long)h * G) * D;
 #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-                const int c0 = kk * 16 + 2 * t4;
-                auto ld = [&](int row, int col) -> uint32_t {
-                    if (row >= G) return 0u;
-                    return __ldg(reinterpret_cast<const unsigned int*>(qb + (long long)row * D + col));
-                };
-                qa[kk][0] = ld(gid, c0);
-                qa[kk][1] = ld(gid + 8, c0);
-                qa[kk][2] = ld(gid, c0 + 8);
-                qa[kk][3] = ld(gid + 8, c0 + 8);
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const int c0 = kk * 16 + 4 * t4;
+                    const uint32_t w0 = gid < G ? __ldg(reinterpret_cast<const unsigned int*>(qb + (long long)gid * D + c0)) : 0u;
+                    const uint32_t w1 = gid + 8 < G ? __ldg(reinterpret_cast<const unsigned int*>(qb + (long long)(gid + 8) * D + c0)) : 0u;
+                    qa[kk][0] = e4m3x2_to_f16x2(w0);
+                    qa[kk][1] = e4m3x2_to_f16x2(w1);
+                    qa[kk][2] = e4m3x2_to_f16x2(w0 >> 16);
+                    qa[kk][3] = e4m3x2_to_f16x2(w1 >> 16);
+                }
+            } else {
+                const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(a.q) + ((long long)bb * a.Hq + (long long)h * G) * D;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const int c0 = kk * 16 + 2 * t4;
+                    auto ld = [&](int row, int col) -> uint32_t {
+                        if (row >= G) return 0u;
+                        return __ldg(reinterpret_cast<const unsigned int*>(qb + (long long)row * D + col));
+                    };
+                    qa[kk][0] = ld(gid, c0);
+                    qa[kk][1] = ld(gid + 8, c0);
+                    qa[kk][2] = ld(gid, c0 + 8);
+                    qa[kk][3] = ld(gid + 8, c0 + 8);
+                }
             }
         };
         auto reset = [&]() {
@@ -657,16 +695,33 @@ __global__ void __launch_bounds__(32 * (kPgMaxWarps + 1), 1)
             s1 += __shfl_xor_sync(0xffffffffu, s1, 1);
             s1 += __shfl_xor_sync(0xffffffffu, s1, 2);
             const long long slot = (long long)blockIdx.x + b;
-            const float i0 = s0 > 0.0f ? 1.0f / s0 : 0.0f, i1 = s1 > 0.0f ? 1.0f / s1 : 0.0f;
+            const float i0 = s0 > 0.0f ? out_scale / s0 : 0.0f, i1 = s1 > 0.0f ? out_scale / s1 : 0.0f;
+            float* r0p = &a.o_part[(slot * a.Hq + h * G + gid) * D];
+            float* r1p = &a.o_part[(slot * a.Hq + h * G + gid + 8) * D];
+            if constexpr (FP8) {
+                // tiles 2s (even columns) and 2s + 1 (odd columns) of 16-column block s:
+                // element e of either is column 16 s + 4 t4 + 2 e (+ 1 for the odd tile)
 #pragma unroll
-            for (int i = 0; i < D / 8; ++i) {
-                const int col = i * 8 + 2 * t4;
-                if (gid < G)
-                    *reinterpret_cast<float2*>(&a.o_part[(slot * a.Hq + h * G + gid) * D + col]) =
-                        make_float2(o[i][0] * i0, o[i][1] * i0);
-                if (gid + 8 < G)
-                    *reinterpret_cast<float2*>(&a.o_part[(slot * a.Hq + h * G + gid + 8) * D + col]) =
-                        make_float2(o[i][2] * i1, o[i][3] * i1);
+                for (int sb = 0; sb < D / 16; ++sb) {
+                    const float* ev = o[2 * sb];
+                    const float* od = o[2 * sb + 1];
+                    const int col = sb * 16 + 4 * t4;
+                    if (gid < G) {
+                        *reinterpret_cast<float2*>(r0p + col) = make_float2(ev[0] * i0, od[0] * i0);
+                        *reinterpret_cast<float2*>(r0p + col + 2) = make_float2(ev[1] * i0, od[1] * i0);
+                    }
+                    if (gid + 8 < G) {
+                        *reinterpret_cast<float2*>(r1p + col) = make_float2(ev[2] * i1, od[2] * i1);
+                        *reinterpret_cast<float2*>(r1p + col + 2) = make_float2(ev[3] * i1, od[3] * i1);
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < D / 8; ++i) {
+                    const int col = i * 8 + 2 * t4;
+                    if (gid < G) *reinterpret_cast<float2*>(r0p + col) = make_float2(o[i][0] * i0, o[i][1] * i0);
+                    if (gid + 8 < G) *reinterpret_cast<float2*>(r1p + col) = make_float2(o[i][2] * i1, o[i][3] * i1);
+                }
             }
             if (t4 == 0) {
                 if (gid < G) a.lse_part[slot * a.Hq + h * G + gid] = s0 > 0.0f ? (m0 + log2f(s0)) * kLn2 : -INFINITY;
@@ -698,25 +753,48 @@ __global__ void __launch_bounds__(32 * (kPgMaxWarps + 1), 1)
             const int r0 = h * kPageRows;                      // this head's first row in the stage
             if (ok) {
                 if (tok0 + kPageRows > L) {
-                    // zero this head's V rows past the sequence end (not data of it)
-                    for (int e = lane; e < kPageRows * (D / 8); e += 32) {
-                        const int rr = e / (D / 8), cc = (e % (D / 8)) * 8;
+                    // zero this head's V rows past the sequence end (not data of it): every
+                    // 16-byte piece of those rows, in each 128-byte column of the stage
+                    constexpr int PPR = C::ROWB / 16;             // pieces per row
+                    for (int e = lane; e < kPageRows * PPR; e += 32) {
+                        const int rr = e / PPR, pc = e % PPR;
                         if (tok0 + rr >= L)
-                            *reinterpret_cast<uint4*>(sv + swz_off<D>(r0 + rr, cc, rows)) = make_uint4(0, 0, 0, 0);
+                            *reinterpret_cast<uint4*>(sv + (pc >> 3) * rows * 128 + (r0 + rr) * 128 + (pc & 7) * 16) =
+                                make_uint4(0, 0, 0, 0);
                     }
                     __syncwarp();
                 }
                 float sc[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}};
                 const uint32_t skb = smem_u32(sk);
+                if constexpr (FP8) {
+                    // one ldmatrix.x4 = key blocks 0 / 1 of 16-column blocks kk and kk + 1; a
+                    // lane's word is 4 consecutive codes k[key][16 kk + 4 t4 ..]: its low pair
+                    // is the B fragment's first register, its high pair the second
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const int mi = lane >> 3, ri = lane & 7;
-                    const int row = r0 + (mi >> 1) * 8 + ri;
-                    const int col = kk * 16 + (mi & 1) * 8;
-                    uint32_t b0, b1, b2, b3;
-                    ldmatrix_x4(skb + swz_off<D>(row, col, rows), b0, b1, b2, b3);
-                    mma_bf16_16816(sc[0], qa[kk], b0, b1);
-                    mma_bf16_16816(sc[1], qa[kk], b2, b3);
+                    for (int kk = 0; kk < D / 16; kk += 2) {
+                        const int mi = lane >> 3, ri = lane & 7;
+                        const int row = r0 + (mi & 1) * 8 + ri;
+                        const int byte = (kk + (mi >> 1)) * 16;
+                        uint32_t w[4];
+                        ldmatrix_x4(skb + row * 128 + (((byte >> 4) ^ (row & 7)) << 4), w[0], w[1], w[2], w[3]);
+#pragma unroll
+                        for (int u = 0; u < 2; ++u)
+#pragma unroll
+                            for (int nt = 0; nt < 2; ++nt)
+                                mma_f16_16816(sc[nt], qa[kk + u], e4m3x2_to_f16x2(w[2 * u + nt]),
+                                              e4m3x2_to_f16x2(w[2 * u + nt] >> 16));
+                    }
+                } else {
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const int mi = lane >> 3, ri = lane & 7;
+                        const int row = r0 + (mi >> 1) * 8 + ri;
+                        const int col = kk * 16 + (mi & 1) * 8;
+                        uint32_t b0, b1, b2, b3;
+                        ldmatrix_x4(skb + swz_off<D>(row, col, rows), b0, b1, b2, b3);
+                        mma_bf16_16816(sc[0], qa[kk], b0, b1);
+                        mma_bf16_16816(sc[1], qa[kk], b2, b3);
+                    }
                 }
                 if (capped) {
 #pragma unroll
@@ -765,20 +843,47 @@ __global__ void __launch_bounds__(32 * (kPgMaxWarps + 1), 1)
                     l1 += pp[nt][2] + pp[nt][3];
                 }
                 uint32_t pa[4];
-                pa[0] = pack_bf16(pp[0][0], pp[0][1]);
-                pa[1] = pack_bf16(pp[0][2], pp[0][3]);
-                pa[2] = pack_bf16(pp[1][0], pp[1][1]);
-                pa[3] = pack_bf16(pp[1][2], pp[1][3]);
                 const uint32_t svb = smem_u32(sv);
+                if constexpr (FP8) {
+                    pa[0] = pack_f16(pp[0][0], pp[0][1]);
+                    pa[1] = pack_f16(pp[0][2], pp[0][3]);
+                    pa[2] = pack_f16(pp[1][0], pp[1][1]);
+                    pa[3] = pack_f16(pp[1][2], pp[1][3]);
+                    // one ldmatrix.x4.trans = key blocks 0 / 1 of 16-column blocks sb and sb + 1;
+                    // a lane's word holds v[2 t4][2 g], v[2 t4][2 g + 1], v[2 t4 + 1][2 g],
+                    // v[2 t4 + 1][2 g + 1] (g = lane / 4): the byte permute pairs the keys of
+                    // column 2 g (low half: the even tile) and of column 2 g + 1 (the odd tile)
 #pragma unroll
-                for (int nd = 0; nd < D / 8; nd += 2) {
-                    const int mi = lane >> 3, ri = lane & 7;
-                    const int row = r0 + (mi & 1) * 8 + ri;
-                    const int col = nd * 8 + (mi >> 1) * 8;
-                    uint32_t b0, b1, b2, b3;
-                    ldmatrix_x4_trans(svb + swz_off<D>(row, col, rows), b0, b1, b2, b3);
-                    mma_bf16_16816(o[nd], pa, b0, b1);
-                    mma_bf16_16816(o[nd + 1], pa, b2, b3);
+                    for (int sb = 0; sb < D / 16; sb += 2) {
+                        const int mi = lane >> 3, ri = lane & 7;
+                        const int row = r0 + (mi & 1) * 8 + ri;
+                        const int byte = (sb + (mi >> 1)) * 16;
+                        uint32_t w[4];
+                        ldmatrix_x4_trans(svb + row * 128 + (((byte >> 4) ^ (row & 7)) << 4), w[0], w[1], w[2], w[3]);
+#pragma unroll
+                        for (int u = 0; u < 2; ++u) {
+                            const uint32_t lo = __byte_perm(w[2 * u], 0u, 0x3120u);       // keys 0..7
+                            const uint32_t hi = __byte_perm(w[2 * u + 1], 0u, 0x3120u);   // keys 8..15
+                            mma_f16_16816(o[2 * (sb + u)], pa, e4m3x2_to_f16x2(lo), e4m3x2_to_f16x2(hi));
+                            mma_f16_16816(o[2 * (sb + u) + 1], pa, e4m3x2_to_f16x2(lo >> 16),
+                                          e4m3x2_to_f16x2(hi >> 16));
+                        }
+                    }
+                } else {
+                    pa[0] = pack_bf16(pp[0][0], pp[0][1]);
+                    pa[1] = pack_bf16(pp[0][2], pp[0][3]);
+                    pa[2] = pack_bf16(pp[1][0], pp[1][1]);
+                    pa[3] = pack_bf16(pp[1][2], pp[1][3]);
+#pragma unroll
+                    for (int nd = 0; nd < D / 8; nd += 2) {
+                        const int mi = lane >> 3, ri = lane & 7;
+                        const int row = r0 + (mi & 1) * 8 + ri;
+                        const int col = nd * 8 + (mi >> 1) * 8;
+                        uint32_t b0, b1, b2, b3;
+                        ldmatrix_x4_trans(svb + swz_off<D>(row, col, rows), b0, b1, b2, b3);
+                        mma_bf16_16816(o[nd], pa, b0, b1);
+                        mma_bf16_16816(o[nd + 1], pa, b2, b3);
+                    }
                 }
             }
             __syncwarp();

@@ -285,6 +285,15 @@ def decode_bytes(t, Hq, Hkv, D):
     return kv + B * Hq * D * 2 * 2 + B * Hq * 4 + pages + B * 4
 
 
+def decode_bytes_fp8(t, Hq, Hkv, D):
+    """decode_bytes with one-byte K, V and q (O stays bf16)."""
+    lens = t["seqused_k"].numpy().astype(np.int64)
+    B = len(lens)
+    kv = int(lens.sum()) * Hkv * D * 2
+    pages = int(((lens + 15) // 16).sum()) * 4
+    return kv + B * Hq * D * (1 + 2) + B * Hq * 4 + pages + B * 4
+
+
 def causal_flops(lens, Hq, D):
     lens = np.asarray(lens, np.int64)
     return float(4 * D * Hq * (lens * (lens + 1) // 2).sum())
@@ -625,6 +634,37 @@ def run_fp8(c):
     c["launches"] += 2 * args.steps
     c["line"]["gpu_launches"] = c["launches"]
     del d8
+
+    # the paged decode workload with q and the cache in e4m3 (per-tensor descales)
+    w = W.paged_decode(seed=args.seed)
+    t, P = w.tensors, w.params
+    d = {k: t[k].to(dev) for k in ("block_table", "seqused_k")}
+    for name in ("q", "k_cache", "v_cache"):
+        d[name], d["descale_" + name] = W.quantize_e4m3(t[name].to(dev))
+        d["descale_" + name] = d["descale_" + name].to(dev)
+    ws = torch.empty(max(A.attn_decode_workspace_size(P["B"], P["Hq"], P["Hkv"], P["D"],
+                                                      P["max_blocks_per_seq"]), 16),
+                     dtype=torch.uint8, device=dev)
+    o = torch.empty(P["B"], P["Hq"], P["D"], dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(P["B"], P["Hq"], dtype=torch.float32, device=dev)
+
+    def dec_step():
+        A.attn_decode_paged(d["q"], d["k_cache"], d["v_cache"], d["block_table"], d["seqused_k"],
+                            scale=P["scale"], descale_q=d["descale_q"],
+                            descale_k=d["descale_k_cache"], descale_v=d["descale_v_cache"],
+                            out=o, lse=lse, workspace=ws)
+
+    dms = statistics.mean(time_steps(dec_step, args.steps, args.warmup, world, flush))
+    nb = decode_bytes_fp8(t, P["Hq"], P["Hkv"], P["D"])
+    e = entry(nb / (dms * 1e-3) / 1e9, "GB/s", dms, "hbm", peaks, dtype="fp8")
+    e["workload"] = ("paged_gqa_decode with q and the cache in e4m3: B=32, Hq=32, Hkv=8, D=128, "
+                     "kv len ~ U[1,8192]")
+    e["bytes_per_step"] = nb
+    e["keys_per_us"] = round(int(t["seqused_k"].sum()) / (dms * 1e3), 1)
+    c["line"]["decode_fp8"] = e
+    c["launches"] += 2 * args.steps
+    c["line"]["gpu_launches"] = c["launches"]
+    del d
 
 
 WINDOW, SOFTCAP = 1024, 50.0

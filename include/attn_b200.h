@@ -238,14 +238,17 @@ size_t attn_decode_workspace_size(int B, int num_heads_q, int num_heads_kv, int 
  * combine.  The query is the newest of the sequence's cached keys and sees
  * all of them, or with window_left >= 0 only keys L-1-window_left .. L-1
  * (L = seqused_k[b]); softcap as above.
- *   q            [B, Hq, D] bf16, contiguous.
+ *   q            [B, Hq, D] bf16 (or e4m3), contiguous.
  *   k_cache/v_cache, block_table, block_size: as in attn_fwd_varlen_paged.
  *   seqused_k    int32 [B], keys cached per sequence (0 gives O = 0, LSE = -inf).
  *   num_splits   key-range splits per sequence; <= 0 chooses automatically.
+ *   dtype        ATTN_BF16, or ATTN_FP8_E4M3 for an e4m3 q and cache with
+ *                descale_q/k/v (device fp32 scalars, all three required):
+ *                head_dim 128, num_splits <= 0, at most 8 KV heads.
  *   o            [B, Hq, D] bf16.   lse [B, Hq] fp32 or NULL.
  *   workspace    >= attn_decode_workspace_size(...) bytes of device memory,
  *                16-byte aligned; its contents on entry do not matter.
- * Supported: bf16, head_dim in {64, 128}, Hq/Hkv <= 16.
+ * Supported: bf16, head_dim in {64, 128}, Hq/Hkv <= 16; e4m3 as above.
  */
 attn_status_t attn_decode_paged(
     const void *q, const void *k_cache, const void *v_cache, const int32_t *block_table,

@@ -180,7 +180,7 @@ def test_noalloc_decode_reports_bad_arguments_like_the_workspace_decode(L):
         "null q, B 0": {0: None, 8: 0}, "null o, B 0": {13: None, 8: 0},
         "negative B": {8: -1}, "Hq not a multiple": {9: 6, 10: 4}, "Hkv 0": {10: 0},
         "max_blocks 0": {4: 0}, "num_blocks 0": {5: 0}, "dtype 7": {12: 7},
-        "fp8": {12: 1}, "head_dim 96": {11: 96}, "head_dim 96, B 0": {11: 96, 8: 0},
+        "head_dim 96": {11: 96}, "head_dim 96, B 0": {11: 96, 8: 0},
         "block_size 32": {6: 32}, "group 32": {9: 32, 10: 1}, "B 5000": {8: 5000},
         "misaligned q": {0: odd}, "misaligned o": {13: odd},
     }
@@ -195,3 +195,23 @@ def test_noalloc_decode_reports_bad_arguments_like_the_workspace_decode(L):
                                                 dt, o, None, None)
         assert ws_status != 0, name
         assert na_status == ws_status, name
+
+
+def test_fp8_decode_argument_checks(L):
+    """e4m3 decode: descales required (invalid without); head_dim 128, automatic split and
+    the key store only (unsupported otherwise); the noalloc call takes bf16 only."""
+    p = ctypes.c_void_p(1 << 20)
+
+    def dec(D=128, splits=0, dq=p, dk=p, dv=p, Hq=8, Hkv=2, B=2):
+        return L.attn_decode_paged(p, p, p, p, 4, 100, 16, p, B, Hq, Hkv, D, 0.0, -1, 0.0, splits,
+                                   1, dq, dk, dv, p, None, p, 1 << 24, None)
+
+    assert dec(dq=None) == 1 and dec(dk=None) == 1 and dec(dv=None) == 1
+    assert dec(D=64) == 2
+    assert dec(splits=3) == 2
+    assert dec(Hq=32, Hkv=16) == 2          # more KV heads than consumer warps
+    st = L.attn_decode_paged_only_qv(p, p, p, 4, 100, 16, p, 2, 8, 2, 128, 0.0, -1, 0.0, 0, 1,
+                                     p, None, p, 1 << 24, None)
+    assert st == 2
+    st = L.attn_decode_paged_noalloc(p, p, p, p, 4, 100, 16, p, 2, 8, 2, 128, 0.0, 1, p, None, None)
+    assert st == 2
