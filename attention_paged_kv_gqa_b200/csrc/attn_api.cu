@@ -386,7 +386,7 @@ void* noalloc_scratch_address(int dev) {
     return p;
 }
 
-template <int D, bool FP8>
+template <int D, bool FP8, int NT>
 attn_status_t launch_decode_pages(const CUtensorMap& mk, const CUtensorMap& mv, const DecodePagesArgs& a,
                                   int grid, cudaStream_t st, __nv_bfloat16* o, float* lse,
                                   bool pdl = false) {
@@ -395,12 +395,12 @@ attn_status_t launch_decode_pages(const CUtensorMap& mk, const CUtensorMap& mv, 
     cudaGetDevice(&dev);
     const uint64_t bit = 1ull << (dev & 63);
     if (!(attr_mask.load() & bit)) {
-        const attn_status_t s = set_smem(decode_pages_kernel<D, FP8>, 227 * 1024);
+        const attn_status_t s = set_smem(decode_pages_kernel<D, FP8, NT>, 227 * 1024);
         if (s != ATTN_OK) return s;
         attr_mask.fetch_or(bit);
     }
     const int smem = DecodePagesCfg<D, FP8>::smem_bytes(a.Hkv, a.B, a.nstages, a.only_qv != 0);
-    attn_status_t s = launch_maybe_pdl(decode_pages_kernel<D, FP8>, dim3(grid), dim3(32 * (a.Hkv + 1)),
+    attn_status_t s = launch_maybe_pdl(decode_pages_kernel<D, FP8, NT>, dim3(grid), dim3(32 * (a.Hkv + 1)),
                                        smem, st, pdl, mk, mv, a);
     if (s != ATTN_OK) return s;
     cudaLaunchConfig_t cfg;
@@ -955,11 +955,16 @@ static attn_status_t decode_paged_impl(const void* q, const void* k_cache, const
         pa.meta = reinterpret_cast<int*>(pa.lse_part + slots * Hq);
         pa.nstages = decode_pages_stages(D, Hkv, B, only_qv != 0, fp8);
         pa.only_qv = only_qv ? 1 : 0;
+        __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(o);
+        const bool wide = pa.group > 8;          // two n-tiles of 8 query heads
         if (fp8)
-            return launch_decode_pages<128, true>(pk, pv, pa, grid, stp, static_cast<__nv_bfloat16*>(o), lse, pdl);
+            return wide ? launch_decode_pages<128, true, 2>(pk, pv, pa, grid, stp, ob, lse, pdl)
+                        : launch_decode_pages<128, true, 1>(pk, pv, pa, grid, stp, ob, lse, pdl);
         if (D == 128)
-            return launch_decode_pages<128, false>(pk, pv, pa, grid, stp, static_cast<__nv_bfloat16*>(o), lse, pdl);
-        return launch_decode_pages<64, false>(pk, pv, pa, grid, stp, static_cast<__nv_bfloat16*>(o), lse, pdl);
+            return wide ? launch_decode_pages<128, false, 2>(pk, pv, pa, grid, stp, ob, lse, pdl)
+                        : launch_decode_pages<128, false, 1>(pk, pv, pa, grid, stp, ob, lse, pdl);
+        return wide ? launch_decode_pages<64, false, 2>(pk, pv, pa, grid, stp, ob, lse, pdl)
+                    : launch_decode_pages<64, false, 1>(pk, pv, pa, grid, stp, ob, lse, pdl);
     }
 
     const uint64_t rowk = (uint64_t)Hkv * D * 2;

@@ -512,7 +512,7 @@ struct DecodePagesCfg {
 // bytes) is its B fragment; for P.V a transposed ldmatrix word holds 2 keys x 2
 // columns, split by a byte permute into the fragments of two 8-column tiles
 // (even and odd columns of a 16-column block).
-template <int D, bool FP8>
+template <int D, bool FP8, int NT>
 __global__ void __launch_bounds__(32 * (kPgMaxWarps + 1), 1)
     decode_pages_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                         const DecodePagesArgs a) {
@@ -633,6 +633,10 @@ __global__ void __launch_bounds__(32 * (kPgMaxWarps + 1), 1)
         }
     } else if (warp < Hkv) {
         // ------------------------------------------------------------ consumer warp = KV head
+        // The page's 16 keys are the M side of both warp MMAs: S^T = K Q^T (16 keys x 8
+        // query heads per n-tile; NT n-tiles cover the group), then O^T += V^T P^T (16
+        // output columns x 8 heads).  Of n-tile nt a lane holds heads 8 nt + 2 t4 and
+        // 8 nt + 2 t4 + 1 (t4 = lane % 4), for keys gid and gid + 8 (gid = lane / 4).
         const int h = warp;
         const int gid = lane >> 2, t4 = lane & 3;
         // logit = eff * (raw dot product); FP8: the raw dot product is of the codes
@@ -645,89 +649,78 @@ __global__ void __launch_bounds__(32 * (kPgMaxWarps + 1), 1)
         const bool capped = a.softcap > 0.0f;
         const float cap_in = capped ? eff / a.softcap : 0.0f;
         const float cap_out = capped ? a.softcap / eff : 0.0f;
-        uint32_t qa[D / 16][4];
-        float o[D / 8][4];
-        float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.0f, l1 = 0.0f;
+        constexpr int QW = FP8 ? D / 32 : D / 16;          // k-steps of the score MMA
+        uint32_t qb[NT][QW][2];                             // B fragments of Q^T
+        float o[D / 16][NT][4];                             // O^T, one 16-column tile each
+        float m[NT][2], l[NT][2];                           // l: this lane's keys only
         int b = -1, b_end = 0, L = 0, kb = 0, kf = 0;
         auto load_q = [&](int bb) {
-            if constexpr (FP8) {
-                // A fragment of 16-column block s: the contraction index permuted so that
-                // logical k = 2 t4 + j is column 16 s + 4 t4 + j and k = 2 t4 + 8 + j is
-                // column 16 s + 4 t4 + 2 + j (matching the K words below)
-                const uint8_t* qb = static_cast<const uint8_t*>(a.q) + ((long long)bb * a.Hq + (long long)h * G) * D;
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const int c0 = kk * 16 + 4 * t4;
-                    const uint32_t w0 = gid < G ? __ldg(reinterpret_cast<const unsigned int*>(qb + (long long)gid * D + c0)) : 0u;
-                    const uint32_t w1 = gid + 8 < G ? __ldg(reinterpret_cast<const unsigned int*>(qb + (long long)(gid + 8) * D + c0)) : 0u;
-                    qa[kk][0] = e4m3x2_to_f16x2(w0);
-                    qa[kk][1] = e4m3x2_to_f16x2(w1);
-                    qa[kk][2] = e4m3x2_to_f16x2(w0 >> 16);
-                    qa[kk][3] = e4m3x2_to_f16x2(w1 >> 16);
-                }
-            } else {
-                const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(a.q) + ((long long)bb * a.Hq + (long long)h * G) * D;
+            for (int nt = 0; nt < NT; ++nt) {
+                const int head = nt * 8 + gid;
+                const bool live = head < G;
+                const long long row = (long long)bb * a.Hq + (long long)h * G + (live ? head : 0);
+                if constexpr (FP8) {
+                    // B (32 x 8 e4m3): word 0 = q[head][32 j + 4 t4 ..], word 1 = 16 columns on
+                    const uint8_t* qr = static_cast<const uint8_t*>(a.q) + row * D;
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const int c0 = kk * 16 + 2 * t4;
-                    auto ld = [&](int row, int col) -> uint32_t {
-                        if (row >= G) return 0u;
-                        return __ldg(reinterpret_cast<const unsigned int*>(qb + (long long)row * D + col));
-                    };
-                    qa[kk][0] = ld(gid, c0);
-                    qa[kk][1] = ld(gid + 8, c0);
-                    qa[kk][2] = ld(gid, c0 + 8);
-                    qa[kk][3] = ld(gid + 8, c0 + 8);
+                    for (int j = 0; j < QW; ++j) {
+                        qb[nt][j][0] = live ? __ldg(reinterpret_cast<const unsigned int*>(qr + 32 * j + 4 * t4)) : 0u;
+                        qb[nt][j][1] = live ? __ldg(reinterpret_cast<const unsigned int*>(qr + 32 * j + 16 + 4 * t4)) : 0u;
+                    }
+                } else {
+                    // B (16 x 8 bf16): word 0 = q[head][16 kk + 2 t4 ..], word 1 = 8 columns on
+                    const __nv_bfloat16* qr = static_cast<const __nv_bfloat16*>(a.q) + row * D;
+#pragma unroll
+                    for (int kk = 0; kk < QW; ++kk) {
+                        qb[nt][kk][0] = live ? __ldg(reinterpret_cast<const unsigned int*>(qr + 16 * kk + 2 * t4)) : 0u;
+                        qb[nt][kk][1] = live ? __ldg(reinterpret_cast<const unsigned int*>(qr + 16 * kk + 8 + 2 * t4)) : 0u;
+                    }
                 }
             }
         };
         auto reset = [&]() {
 #pragma unroll
-            for (int i = 0; i < D / 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.0f;
-            m0 = m1 = -INFINITY;
-            l0 = l1 = 0.0f;
+            for (int c = 0; c < D / 16; ++c)
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) o[c][nt][0] = o[c][nt][1] = o[c][nt][2] = o[c][nt][3] = 0.0f;
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                m[nt][0] = m[nt][1] = -INFINITY;
+                l[nt][0] = l[nt][1] = 0.0f;
+            }
         };
         // write the partial of (this CTA, sequence b) for this head's G query heads
         auto flush_partial = [&]() {
-            float s0 = l0, s1 = l1;
-            s0 += __shfl_xor_sync(0xffffffffu, s0, 1);
-            s0 += __shfl_xor_sync(0xffffffffu, s0, 2);
-            s1 += __shfl_xor_sync(0xffffffffu, s1, 1);
-            s1 += __shfl_xor_sync(0xffffffffu, s1, 2);
             const long long slot = (long long)blockIdx.x + b;
-            const float i0 = s0 > 0.0f ? out_scale / s0 : 0.0f, i1 = s1 > 0.0f ? out_scale / s1 : 0.0f;
-            float* r0p = &a.o_part[(slot * a.Hq + h * G + gid) * D];
-            float* r1p = &a.o_part[(slot * a.Hq + h * G + gid + 8) * D];
-            if constexpr (FP8) {
-                // tiles 2s (even columns) and 2s + 1 (odd columns) of 16-column block s:
-                // element e of either is column 16 s + 4 t4 + 2 e (+ 1 for the odd tile)
 #pragma unroll
-                for (int sb = 0; sb < D / 16; ++sb) {
-                    const float* ev = o[2 * sb];
-                    const float* od = o[2 * sb + 1];
-                    const int col = sb * 16 + 4 * t4;
-                    if (gid < G) {
-                        *reinterpret_cast<float2*>(r0p + col) = make_float2(ev[0] * i0, od[0] * i0);
-                        *reinterpret_cast<float2*>(r0p + col + 2) = make_float2(ev[1] * i0, od[1] * i0);
-                    }
-                    if (gid + 8 < G) {
-                        *reinterpret_cast<float2*>(r1p + col) = make_float2(ev[2] * i1, od[2] * i1);
-                        *reinterpret_cast<float2*>(r1p + col + 2) = make_float2(ev[3] * i1, od[3] * i1);
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    float s = l[nt][e];
+                    s += __shfl_xor_sync(0xffffffffu, s, 4);
+                    s += __shfl_xor_sync(0xffffffffu, s, 8);
+                    s += __shfl_xor_sync(0xffffffffu, s, 16);
+                    const int head = nt * 8 + 2 * t4 + e;
+                    if (head < G) {
+                        const float inv = s > 0.0f ? out_scale / s : 0.0f;
+                        float* rp = &a.o_part[(slot * a.Hq + h * G + head) * D];
+#pragma unroll
+                        for (int c = 0; c < D / 16; ++c) {
+                            if constexpr (FP8) {
+                                // tile rows gid / gid + 8 are columns 16 c + 2 gid and + 1
+                                *reinterpret_cast<float2*>(rp + 16 * c + 2 * gid) =
+                                    make_float2(o[c][nt][e] * inv, o[c][nt][2 + e] * inv);
+                            } else {
+                                rp[16 * c + gid] = o[c][nt][e] * inv;
+                                rp[16 * c + 8 + gid] = o[c][nt][2 + e] * inv;
+                            }
+                        }
+                        if (gid == 0)
+                            a.lse_part[slot * a.Hq + h * G + head] =
+                                s > 0.0f ? (m[nt][e] + log2f(s)) * kLn2 : -INFINITY;
                     }
                 }
-            } else {
-#pragma unroll
-                for (int i = 0; i < D / 8; ++i) {
-                    const int col = i * 8 + 2 * t4;
-                    if (gid < G) *reinterpret_cast<float2*>(r0p + col) = make_float2(o[i][0] * i0, o[i][1] * i0);
-                    if (gid + 8 < G) *reinterpret_cast<float2*>(r1p + col) = make_float2(o[i][2] * i1, o[i][3] * i1);
-                }
-            }
-            if (t4 == 0) {
-                if (gid < G) a.lse_part[slot * a.Hq + h * G + gid] = s0 > 0.0f ? (m0 + log2f(s0)) * kLn2 : -INFINITY;
-                if (gid + 8 < G)
-                    a.lse_part[slot * a.Hq + h * G + gid + 8] = s1 > 0.0f ? (m1 + log2f(s1)) * kLn2 : -INFINITY;
-            }
         };
         bool ok = true;
         for (int i = 0; i < npages; ++i) {
@@ -764,125 +757,109 @@ __global__ void __launch_bounds__(32 * (kPgMaxWarps + 1), 1)
                     }
                     __syncwarp();
                 }
-                float sc[2][4] = {{0, 0, 0, 0}, {0, 0, 0, 0}};
+                const int mi = lane >> 3, ri = lane & 7;
+                float sc[NT][4];
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.0f;
                 const uint32_t skb = smem_u32(sk);
                 if constexpr (FP8) {
-                    // one ldmatrix.x4 = key blocks 0 / 1 of 16-column blocks kk and kk + 1; a
-                    // lane's word is 4 consecutive codes k[key][16 kk + 4 t4 ..]: its low pair
-                    // is the B fragment's first register, its high pair the second
+                    // A (16 keys x 32 e4m3): one ldmatrix.x4 = keys 0-7 / 8-15 of the 16-byte
+                    // pieces 2 j and 2 j + 1, which is the fragment as it stands
 #pragma unroll
-                    for (int kk = 0; kk < D / 16; kk += 2) {
-                        const int mi = lane >> 3, ri = lane & 7;
+                    for (int j = 0; j < QW; ++j) {
                         const int row = r0 + (mi & 1) * 8 + ri;
-                        const int byte = (kk + (mi >> 1)) * 16;
-                        uint32_t w[4];
-                        ldmatrix_x4(skb + row * 128 + (((byte >> 4) ^ (row & 7)) << 4), w[0], w[1], w[2], w[3]);
+                        const int piece = 2 * j + (mi >> 1);
+                        uint32_t ka[4];
+                        ldmatrix_x4(skb + row * 128 + ((piece ^ (row & 7)) << 4), ka[0], ka[1], ka[2], ka[3]);
 #pragma unroll
-                        for (int u = 0; u < 2; ++u)
-#pragma unroll
-                            for (int nt = 0; nt < 2; ++nt)
-                                mma_f16_16816(sc[nt], qa[kk + u], e4m3x2_to_f16x2(w[2 * u + nt]),
-                                              e4m3x2_to_f16x2(w[2 * u + nt] >> 16));
+                        for (int nt = 0; nt < NT; ++nt) mma_e4m3_16832(sc[nt], ka, qb[nt][j][0], qb[nt][j][1]);
                     }
                 } else {
 #pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const int mi = lane >> 3, ri = lane & 7;
-                        const int row = r0 + (mi >> 1) * 8 + ri;
-                        const int col = kk * 16 + (mi & 1) * 8;
-                        uint32_t b0, b1, b2, b3;
-                        ldmatrix_x4(skb + swz_off<D>(row, col, rows), b0, b1, b2, b3);
-                        mma_bf16_16816(sc[0], qa[kk], b0, b1);
-                        mma_bf16_16816(sc[1], qa[kk], b2, b3);
+                    for (int kk = 0; kk < QW; ++kk) {
+                        const int row = r0 + (mi & 1) * 8 + ri;
+                        const int col = kk * 16 + (mi >> 1) * 8;
+                        uint32_t ka[4];
+                        ldmatrix_x4(skb + swz_off<D>(row, col, rows), ka[0], ka[1], ka[2], ka[3]);
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(sc[nt], ka, qb[nt][kk][0], qb[nt][kk][1]);
                     }
                 }
                 if (capped) {
 #pragma unroll
-                    for (int nt = 0; nt < 2; ++nt)
+                    for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                         for (int e = 0; e < 4; ++e) sc[nt][e] = softcap_raw(sc[nt][e], cap_in, cap_out);
                 }
-                float mx0 = -INFINITY, mx1 = -INFINITY;
+                const int key0 = tok0 + gid, key1 = key0 + 8;
+                const bool dead0 = key0 >= L || key0 < kf, dead1 = key1 >= L || key1 < kf;
+                uint32_t pb[NT][2];
 #pragma unroll
-                for (int nt = 0; nt < 2; ++nt)
+                for (int nt = 0; nt < NT; ++nt) {
+                    if (dead0) sc[nt][0] = sc[nt][1] = -INFINITY;
+                    if (dead1) sc[nt][2] = sc[nt][3] = -INFINITY;
+                    float p[4];
 #pragma unroll
                     for (int e = 0; e < 2; ++e) {
-                        const int kv = tok0 + nt * 8 + 2 * t4 + e;
-                        if (kv >= L || kv < kf) { sc[nt][e] = -INFINITY; sc[nt][2 + e] = -INFINITY; }
-                        mx0 = fmaxf(mx0, sc[nt][e]);
-                        mx1 = fmaxf(mx1, sc[nt][2 + e]);
+                        // the max over the page's keys: this lane's two, then across gid
+                        float mx = fmaxf(sc[nt][e], sc[nt][2 + e]);
+                        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+                        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+                        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+                        const float mn = fmaxf(m[nt][e], mx * sl2);
+                        const float al = (mn == -INFINITY) ? 1.0f : ex2(m[nt][e] - mn);
+                        m[nt][e] = mn;
+#pragma unroll
+                        for (int c = 0; c < D / 16; ++c) {
+                            o[c][nt][e] *= al;
+                            o[c][nt][2 + e] *= al;
+                        }
+                        const float mu = (mn == -INFINITY) ? 0.0f : mn;
+                        p[e] = ex2(fmaf(sc[nt][e], sl2, -mu));
+                        p[2 + e] = ex2(fmaf(sc[nt][2 + e], sl2, -mu));
+                        l[nt][e] = l[nt][e] * al + p[e] + p[2 + e];
                     }
-                mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
-                mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
-                mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-                mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-                const float mn0 = fmaxf(m0, mx0 * sl2), mn1 = fmaxf(m1, mx1 * sl2);
-                const float al0 = (mn0 == -INFINITY) ? 1.0f : ex2(m0 - mn0);
-                const float al1 = (mn1 == -INFINITY) ? 1.0f : ex2(m1 - mn1);
-                m0 = mn0;
-                m1 = mn1;
-                l0 *= al0;
-                l1 *= al1;
-#pragma unroll
-                for (int k2 = 0; k2 < D / 8; ++k2) {
-                    o[k2][0] *= al0;
-                    o[k2][1] *= al0;
-                    o[k2][2] *= al1;
-                    o[k2][3] *= al1;
+                    // P (keys x heads, this lane: keys gid / gid + 8, heads 2 t4, 2 t4 + 1)
+                    // transposed in registers: B (16 keys x 8 heads) of the P.V MMA
+                    if constexpr (FP8) {
+                        pb[nt][0] = movmatrix_trans(pack_f16(p[0], p[1]));
+                        pb[nt][1] = movmatrix_trans(pack_f16(p[2], p[3]));
+                    } else {
+                        pb[nt][0] = movmatrix_trans(pack_bf16(p[0], p[1]));
+                        pb[nt][1] = movmatrix_trans(pack_bf16(p[2], p[3]));
+                    }
                 }
-                const float mu0 = (m0 == -INFINITY) ? 0.0f : m0;
-                const float mu1 = (m1 == -INFINITY) ? 0.0f : m1;
-                float pp[2][4];
-#pragma unroll
-                for (int nt = 0; nt < 2; ++nt) {
-                    pp[nt][0] = ex2(fmaf(sc[nt][0], sl2, -mu0));
-                    pp[nt][1] = ex2(fmaf(sc[nt][1], sl2, -mu0));
-                    pp[nt][2] = ex2(fmaf(sc[nt][2], sl2, -mu1));
-                    pp[nt][3] = ex2(fmaf(sc[nt][3], sl2, -mu1));
-                    l0 += pp[nt][0] + pp[nt][1];
-                    l1 += pp[nt][2] + pp[nt][3];
-                }
-                uint32_t pa[4];
                 const uint32_t svb = smem_u32(sv);
                 if constexpr (FP8) {
-                    pa[0] = pack_f16(pp[0][0], pp[0][1]);
-                    pa[1] = pack_f16(pp[0][2], pp[0][3]);
-                    pa[2] = pack_f16(pp[1][0], pp[1][1]);
-                    pa[3] = pack_f16(pp[1][2], pp[1][3]);
-                    // one ldmatrix.x4.trans = key blocks 0 / 1 of 16-column blocks sb and sb + 1;
-                    // a lane's word holds v[2 t4][2 g], v[2 t4][2 g + 1], v[2 t4 + 1][2 g],
-                    // v[2 t4 + 1][2 g + 1] (g = lane / 4): the byte permute pairs the keys of
-                    // column 2 g (low half: the even tile) and of column 2 g + 1 (the odd tile)
+                    // A (16 columns x 16 keys, f16): one ldmatrix.x4.trans = keys 0-7 / 8-15 of
+                    // pieces cc and cc + 1; a lane's word holds v[2 t4][2 gid], v[2 t4][2 gid + 1],
+                    // v[2 t4 + 1][2 gid], v[2 t4 + 1][2 gid + 1].  The byte permute pairs the
+                    // keys of column 2 gid (tile row gid) and of column 2 gid + 1 (row gid + 8).
 #pragma unroll
-                    for (int sb = 0; sb < D / 16; sb += 2) {
-                        const int mi = lane >> 3, ri = lane & 7;
+                    for (int cc = 0; cc < D / 16; cc += 2) {
                         const int row = r0 + (mi & 1) * 8 + ri;
-                        const int byte = (sb + (mi >> 1)) * 16;
+                        const int piece = cc + (mi >> 1);
                         uint32_t w[4];
-                        ldmatrix_x4_trans(svb + row * 128 + (((byte >> 4) ^ (row & 7)) << 4), w[0], w[1], w[2], w[3]);
+                        ldmatrix_x4_trans(svb + row * 128 + ((piece ^ (row & 7)) << 4), w[0], w[1], w[2], w[3]);
 #pragma unroll
                         for (int u = 0; u < 2; ++u) {
                             const uint32_t lo = __byte_perm(w[2 * u], 0u, 0x3120u);       // keys 0..7
                             const uint32_t hi = __byte_perm(w[2 * u + 1], 0u, 0x3120u);   // keys 8..15
-                            mma_f16_16816(o[2 * (sb + u)], pa, e4m3x2_to_f16x2(lo), e4m3x2_to_f16x2(hi));
-                            mma_f16_16816(o[2 * (sb + u) + 1], pa, e4m3x2_to_f16x2(lo >> 16),
-                                          e4m3x2_to_f16x2(hi >> 16));
+                            const uint32_t va[4] = {e4m3x2_to_f16x2(lo), e4m3x2_to_f16x2(lo >> 16),
+                                                    e4m3x2_to_f16x2(hi), e4m3x2_to_f16x2(hi >> 16)};
+#pragma unroll
+                            for (int nt = 0; nt < NT; ++nt) mma_f16_16816(o[cc + u][nt], va, pb[nt][0], pb[nt][1]);
                         }
                     }
                 } else {
-                    pa[0] = pack_bf16(pp[0][0], pp[0][1]);
-                    pa[1] = pack_bf16(pp[0][2], pp[0][3]);
-                    pa[2] = pack_bf16(pp[1][0], pp[1][1]);
-                    pa[3] = pack_bf16(pp[1][2], pp[1][3]);
 #pragma unroll
-                    for (int nd = 0; nd < D / 8; nd += 2) {
-                        const int mi = lane >> 3, ri = lane & 7;
-                        const int row = r0 + (mi & 1) * 8 + ri;
-                        const int col = nd * 8 + (mi >> 1) * 8;
-                        uint32_t b0, b1, b2, b3;
-                        ldmatrix_x4_trans(svb + swz_off<D>(row, col, rows), b0, b1, b2, b3);
-                        mma_bf16_16816(o[nd], pa, b0, b1);
-                        mma_bf16_16816(o[nd + 1], pa, b2, b3);
+                    for (int c = 0; c < D / 16; ++c) {
+                        const int row = r0 + (mi >> 1) * 8 + ri;
+                        const int col = c * 16 + (mi & 1) * 8;
+                        uint32_t va[4];
+                        ldmatrix_x4_trans(svb + swz_off<D>(row, col, rows), va[0], va[1], va[2], va[3]);
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(o[c][nt], va, pb[nt][0], pb[nt][1]);
                     }
                 }
             }
