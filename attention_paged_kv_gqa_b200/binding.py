@@ -68,6 +68,9 @@ def lib():
         L.attn_decode_paged.argtypes = [P, P, P, P, I, I, I, P, I, I, I, I, F, I, F, I, I, P, P,
                                         P, P, P, P, Z, P]
         L.attn_decode_paged.restype = I
+        L.attn_decode_paged_qv.argtypes = [P, P, P, P, P, I, I, I, P, I, I, I, I, F, I, F, I, I,
+                                           P, P, P, Z, P]
+        L.attn_decode_paged_qv.restype = I
         L.attn_decode_paged_noalloc.argtypes = [P, P, P, P, I, I, I, P, I, I, I, I, F, I, P, P, P]
         L.attn_decode_paged_noalloc.restype = I
         L.attn_kv_append_paged.argtypes = [P, P, P, P, P, I, I, I, P, P, P, I, I, I, I, I, P]
@@ -278,6 +281,34 @@ def attn_decode_paged(q, k_cache, v_cache, block_table, seqused_k, *, scale=None
                                  _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(),
                                  _stream(stream))
     _check(st, "attn_decode_paged")
+    return out, lse
+
+
+def attn_decode_paged_qv(q, qv, k_cache, v_cache, block_table, seqused_k, *, scale=None,
+                         num_splits=0, window_left=-1, softcap=0.0, out=None, lse=None,
+                         workspace=None, return_lse=True, stream=None):
+    """Paged decode whose logit adds the Qv term: scale * (q.k + qv.v).
+
+    q, qv [B, Hq, D] bf16 -> (o [B, Hq, D] bf16, lse [B, Hq] fp32); arguments as
+    attn_decode_paged.
+    """
+    B, Hq, D = q.shape
+    num_blocks, block_size, Hkv = k_cache.shape[0], k_cache.shape[1], k_cache.shape[2]
+    mbps = block_table.shape[1]
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=torch.bfloat16, device=q.device)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    ws_bytes = attn_decode_workspace_size(B, Hq, Hkv, D, mbps, block_size, num_splits)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=q.device)
+    st = lib().attn_decode_paged_qv(_ptr(q), _ptr(qv), _ptr(k_cache), _ptr(v_cache),
+                                    _ptr(block_table), mbps, num_blocks, block_size,
+                                    _ptr(seqused_k), B, Hq, Hkv, D, _scale(scale),
+                                    int(window_left), float(softcap), int(num_splits),
+                                    _dtype_code(q), _ptr(out), _ptr(lse), _ptr(workspace),
+                                    workspace.numel(), _stream(stream))
+    _check(st, "attn_decode_paged_qv")
     return out, lse
 
 

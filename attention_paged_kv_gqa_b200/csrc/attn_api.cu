@@ -386,7 +386,7 @@ void* noalloc_scratch_address(int dev) {
     return p;
 }
 
-template <int D, bool FP8, int NT>
+template <int D, bool FP8, int NT, bool HQ = false>
 attn_status_t launch_decode_pages(const CUtensorMap& mk, const CUtensorMap& mv, const DecodePagesArgs& a,
                                   int grid, cudaStream_t st, __nv_bfloat16* o, float* lse,
                                   bool pdl = false) {
@@ -395,12 +395,12 @@ attn_status_t launch_decode_pages(const CUtensorMap& mk, const CUtensorMap& mv, 
     cudaGetDevice(&dev);
     const uint64_t bit = 1ull << (dev & 63);
     if (!(attr_mask.load() & bit)) {
-        const attn_status_t s = set_smem(decode_pages_kernel<D, FP8, NT>, 227 * 1024);
+        const attn_status_t s = set_smem(decode_pages_kernel<D, FP8, NT, HQ>, 227 * 1024);
         if (s != ATTN_OK) return s;
         attr_mask.fetch_or(bit);
     }
     const int smem = DecodePagesCfg<D, FP8>::smem_bytes(a.Hkv, a.B, a.nstages, a.only_qv != 0);
-    attn_status_t s = launch_maybe_pdl(decode_pages_kernel<D, FP8, NT>, dim3(grid), dim3(32 * (a.Hkv + 1)),
+    attn_status_t s = launch_maybe_pdl(decode_pages_kernel<D, FP8, NT, HQ>, dim3(grid), dim3(32 * (a.Hkv + 1)),
                                        smem, st, pdl, mk, mv, a);
     if (s != ATTN_OK) return s;
     cudaLaunchConfig_t cfg;
@@ -874,7 +874,8 @@ static attn_status_t decode_paged_impl(const void* q, const void* k_cache, const
                                        int window_left, float softcap, int num_splits, int dtype,
                                        const float* dq, const float* dk, const float* dv, void* o,
                                        float* lse, void* workspace, size_t workspace_bytes,
-                                       attn_stream_t stream, bool pdl, int only_qv = 0) {
+                                       attn_stream_t stream, bool pdl, int only_qv = 0,
+                                       const void* qv = nullptr) {
     if (!q || !k_cache || !v_cache || !block_table || !seqused_k || !o) return ATTN_ERR_INVALID_ARG;
     {
         // the query is the newest token: the window is a causal one by construction
@@ -888,7 +889,7 @@ static attn_status_t decode_paged_impl(const void* q, const void* k_cache, const
     const bool fp8 = dtype == ATTN_FP8_E4M3;
     if (fp8) {
         // e4m3 q and cache: the page-stream decode (automatic split), head_dim 128
-        if (only_qv) return ATTN_ERR_UNSUPPORTED;
+        if (only_qv || qv) return ATTN_ERR_UNSUPPORTED;
         if (!dq || !dk || !dv) return ATTN_ERR_INVALID_ARG;
         if (D != 128 || num_splits > 0) return ATTN_ERR_UNSUPPORTED;
     }
@@ -899,6 +900,12 @@ static attn_status_t decode_paged_impl(const void* q, const void* k_cache, const
     if ((long long)num_blocks * block_size >= (1LL << 31)) return ATTN_ERR_UNSUPPORTED;
     if ((long long)max_blocks_per_seq * block_size >= (1LL << 30)) return ATTN_ERR_UNSUPPORTED;
     if (fp8 && !use_page_stream(B, Hq, Hkv, D, num_splits)) return ATTN_ERR_UNSUPPORTED;
+    if (qv) {
+        // the extra Qv score term: bf16, the page-stream decode (automatic split)
+        if (dtype != ATTN_BF16 || only_qv || !use_page_stream(B, Hq, Hkv, D, num_splits))
+            return ATTN_ERR_UNSUPPORTED;
+        if (!aligned16(qv)) return ATTN_ERR_INVALID_ARG;
+    }
     if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o))
         return ATTN_ERR_INVALID_ARG;
     int ns, tps;
@@ -940,6 +947,7 @@ static attn_status_t decode_paged_impl(const void* q, const void* k_cache, const
         pa.Hkv = Hkv;
         pa.group = Hq / Hkv;
         pa.q = q;
+        pa.qv = qv;
         pa.descale_q = dq;
         pa.descale_k = dk;
         pa.descale_v = dv;
@@ -957,6 +965,13 @@ static attn_status_t decode_paged_impl(const void* q, const void* k_cache, const
         pa.only_qv = only_qv ? 1 : 0;
         __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(o);
         const bool wide = pa.group > 8;          // two n-tiles of 8 query heads
+        if (qv) {
+            if (D == 128)
+                return wide ? launch_decode_pages<128, false, 2, true>(pk, pv, pa, grid, stp, ob, lse, pdl)
+                            : launch_decode_pages<128, false, 1, true>(pk, pv, pa, grid, stp, ob, lse, pdl);
+            return wide ? launch_decode_pages<64, false, 2, true>(pk, pv, pa, grid, stp, ob, lse, pdl)
+                        : launch_decode_pages<64, false, 1, true>(pk, pv, pa, grid, stp, ob, lse, pdl);
+        }
         if (fp8)
             return wide ? launch_decode_pages<128, true, 2>(pk, pv, pa, grid, stp, ob, lse, pdl)
                         : launch_decode_pages<128, true, 1>(pk, pv, pa, grid, stp, ob, lse, pdl);
@@ -1024,6 +1039,20 @@ attn_status_t attn_decode_paged(const void* q, const void* k_cache, const void* 
                              block_size, seqused_k, B, Hq, Hkv, D, softmax_scale, window_left,
                              softcap, num_splits, dtype, dq, dk, dv, o, lse, workspace,
                              workspace_bytes, stream, false);
+}
+
+attn_status_t attn_decode_paged_qv(const void* q, const void* qv, const void* k_cache,
+                                   const void* v_cache, const int32_t* block_table,
+                                   int max_blocks_per_seq, int num_blocks, int block_size,
+                                   const int32_t* seqused_k, int B, int Hq, int Hkv, int D,
+                                   float softmax_scale, int window_left, float softcap,
+                                   int num_splits, int dtype, void* o, float* lse, void* workspace,
+                                   size_t workspace_bytes, attn_stream_t stream) {
+    if (!qv) return ATTN_ERR_INVALID_ARG;
+    return decode_paged_impl(q, k_cache, v_cache, block_table, max_blocks_per_seq, num_blocks,
+                             block_size, seqused_k, B, Hq, Hkv, D, softmax_scale, window_left,
+                             softcap, num_splits, dtype, nullptr, nullptr, nullptr, o, lse,
+                             workspace, workspace_bytes, stream, false, 0, qv);
 }
 
 attn_status_t attn_decode_paged_only_qv(const void* qv, const void* v_cache,

@@ -470,6 +470,7 @@ constexpr int kPgMaxWarps = 8;         // consumer warps (KV heads) of the page-
 struct DecodePagesArgs {
     int B, Hq, Hkv, group;
     const void* q;            // [B][Hq][D] bf16, or e4m3 (the FP8 instance)
+    const void* qv;           // HQ instance: [B][Hq][D] bf16, the Qv operand of the score
     const float* descale_q;   // FP8: device fp32 scalars (real value = code x descale)
     const float* descale_k;
     const float* descale_v;
@@ -512,11 +513,15 @@ struct DecodePagesCfg {
 // bytes) is its B fragment; for P.V a transposed ldmatrix word holds 2 keys x 2
 // columns, split by a byte permute into the fragments of two 8-column tiles
 // (even and odd columns of a 16-column block).
-template <int D, bool FP8, int NT>
+// HQ: the score has the extra term q_v . v_j of the "Rope dim" forward (HasQv):
+// logit = scale (q . k_j + q_v . v_j), the page's V rows serving as a second A
+// operand of the score MMA (bf16 only).
+template <int D, bool FP8, int NT, bool HQ>
 __global__ void __launch_bounds__(32 * (kPgMaxWarps + 1), 1)
     decode_pages_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                         const DecodePagesArgs a) {
     using C = DecodePagesCfg<D, FP8>;
+    static_assert(!(FP8 && HQ), "the Qv score term is bf16 only");
     const int NS = a.nstages;
     const int Hkv = a.Hkv, G = a.group;
     const int SB = C::stage_bytes(Hkv, a.only_qv);          // K and V of a page, or V alone
@@ -651,6 +656,7 @@ __global__ void __launch_bounds__(32 * (kPgMaxWarps + 1), 1)
         const float cap_out = capped ? a.softcap / eff : 0.0f;
         constexpr int QW = FP8 ? D / 32 : D / 16;          // k-steps of the score MMA
         uint32_t qb[NT][QW][2];                             // B fragments of Q^T
+        uint32_t qvb[HQ ? NT : 1][HQ ? QW : 1][2];          // HQ: B fragments of Qv^T
         float o[D / 16][NT][4];                             // O^T, one 16-column tile each
         float m[NT][2], l[NT][2];                           // l: this lane's keys only
         int b = -1, b_end = 0, L = 0, kb = 0, kf = 0;
@@ -675,6 +681,14 @@ __global__ void __launch_bounds__(32 * (kPgMaxWarps + 1), 1)
                     for (int kk = 0; kk < QW; ++kk) {
                         qb[nt][kk][0] = live ? __ldg(reinterpret_cast<const unsigned int*>(qr + 16 * kk + 2 * t4)) : 0u;
                         qb[nt][kk][1] = live ? __ldg(reinterpret_cast<const unsigned int*>(qr + 16 * kk + 8 + 2 * t4)) : 0u;
+                    }
+                    if constexpr (HQ) {
+                        const __nv_bfloat16* qvr = static_cast<const __nv_bfloat16*>(a.qv) + row * D;
+#pragma unroll
+                        for (int kk = 0; kk < QW; ++kk) {
+                            qvb[nt][kk][0] = live ? __ldg(reinterpret_cast<const unsigned int*>(qvr + 16 * kk + 2 * t4)) : 0u;
+                            qvb[nt][kk][1] = live ? __ldg(reinterpret_cast<const unsigned int*>(qvr + 16 * kk + 8 + 2 * t4)) : 0u;
+                        }
                     }
                 }
             }
@@ -783,6 +797,19 @@ __global__ void __launch_bounds__(32 * (kPgMaxWarps + 1), 1)
                         ldmatrix_x4(skb + swz_off<D>(row, col, rows), ka[0], ka[1], ka[2], ka[3]);
 #pragma unroll
                         for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(sc[nt], ka, qb[nt][kk][0], qb[nt][kk][1]);
+                    }
+                    if constexpr (HQ) {
+                        // + V Qv^T: the V rows as the A operand, read like the K rows
+                        const uint32_t svs = smem_u32(sv);
+#pragma unroll
+                        for (int kk = 0; kk < QW; ++kk) {
+                            const int row = r0 + (mi & 1) * 8 + ri;
+                            const int col = kk * 16 + (mi >> 1) * 8;
+                            uint32_t va[4];
+                            ldmatrix_x4(svs + swz_off<D>(row, col, rows), va[0], va[1], va[2], va[3]);
+#pragma unroll
+                            for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(sc[nt], va, qvb[nt][kk][0], qvb[nt][kk][1]);
+                        }
                     }
                 }
                 if (capped) {

@@ -259,6 +259,27 @@ attn_status_t attn_decode_paged(
     void *o, float *lse, void *workspace, size_t workspace_bytes, attn_stream_t stream);
 
 /*
+ * Paged decode with the extra Qv score term of "Rope dim" (vllm-project
+ * flash-attention PR 172, overview: the Qv GEMM beside the QK GEMM, HasQv):
+ * the logit of key j is scale * (q . k_j + qv . v_j), then softcap, masks,
+ * softmax and P.V as in attn_decode_paged.
+ *   qv           [B, Hq, D] bf16, contiguous, 16-byte aligned; the value head
+ *                dimension equals the key one here.
+ *   other arguments as attn_decode_paged (workspace sized by
+ *                attn_decode_workspace_size with the same arguments).
+ * Supported: bf16, head_dim in {64, 128}, num_splits <= 0 (the automatic
+ * split), Hkv <= 8, Hq/Hkv <= 16, B <= 4096; otherwise ATTN_ERR_UNSUPPORTED.
+ * qv NULL gives ATTN_ERR_INVALID_ARG.  Each value row is read once per page
+ * and feeds both the score and the P.V product.
+ */
+attn_status_t attn_decode_paged_qv(
+    const void *q, const void *qv, const void *k_cache, const void *v_cache,
+    const int32_t *block_table, int max_blocks_per_seq, int num_blocks, int block_size,
+    const int32_t *seqused_k, int B, int num_heads_q, int num_heads_kv, int head_dim,
+    float softmax_scale, int window_left, float softcap, int num_splits, int dtype, void *o,
+    float *lse, void *workspace, size_t workspace_bytes, attn_stream_t stream);
+
+/*
  * Paged decode with the only_qv score (as attn_fwd_varlen_paged_only_qv): the
  * score of key j is scale * (qv . v_j), read from the one value store; each
  * page of V is fetched once.  Arguments as attn_decode_paged with qv in place

@@ -215,3 +215,21 @@ def test_fp8_decode_argument_checks(L):
     assert st == 2
     st = L.attn_decode_paged_noalloc(p, p, p, p, 4, 100, 16, p, 2, 8, 2, 128, 0.0, 1, p, None, None)
     assert st == 2
+
+
+def test_decode_qv_argument_checks(L):
+    """Decode with the Qv term: qv required (invalid without); bf16 and the automatic split
+    only (unsupported otherwise); a misaligned qv is invalid."""
+    p = ctypes.c_void_p(1 << 20)
+    odd = ctypes.c_void_p((1 << 20) + 8)
+
+    def dec(qv=p, D=128, splits=0, dtype=0, Hq=8, Hkv=2):
+        return L.attn_decode_paged_qv(p, qv, p, p, p, 4, 100, 16, p, 2, Hq, Hkv, D, 0.0, -1, 0.0,
+                                      splits, dtype, p, None, p, 1 << 24, None)
+
+    assert dec(qv=None) == 1
+    assert dec(qv=odd) == 1
+    assert dec(D=96) == 2
+    assert dec(splits=2) == 2
+    assert dec(dtype=1) == 2
+    assert dec(Hq=32, Hkv=16) == 2
