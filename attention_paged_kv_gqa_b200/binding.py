@@ -68,6 +68,9 @@ def lib():
         L.attn_decode_paged.argtypes = [P, P, P, P, I, I, I, P, I, I, I, I, F, I, F, I, I, P, P,
                                         P, P, P, P, Z, P]
         L.attn_decode_paged.restype = I
+        L.attn_fwd_varlen_paged_qv.argtypes = [P, P, P, P, P, I, I, I, P, P, P, I, I, I, I, I, I,
+                                               I, F, I, P, I, F, I, P, P, P]
+        L.attn_fwd_varlen_paged_qv.restype = I
         L.attn_decode_paged_qv.argtypes = [P, P, P, P, P, I, I, I, P, I, I, I, I, F, I, F, I, I,
                                            P, P, P, Z, P]
         L.attn_decode_paged_qv.restype = I
@@ -224,6 +227,34 @@ def attn_fwd_varlen_paged_only_qv(qv, v_cache, *, cu_seqlens_q, max_seqlen_q, bl
         int(window_left), float(softcap), _dtype_code(qv), _ptr(descale_qv), _ptr(descale_v),
         _ptr(out), _ptr(lse), _stream(stream))
     _check(st, "attn_fwd_varlen_paged_only_qv")
+    return out, lse
+
+
+def attn_fwd_varlen_paged_qv(q, qv, k_cache, v_cache, *, cu_seqlens_q, max_seqlen_q,
+                             block_table=None, cu_seqlens_k=None, seqused_k=None, mask=MASK_NONE,
+                             scale=None, patch_kv_range=None, window_left=-1, softcap=0.0,
+                             out=None, lse=None, return_lse=True, stream=None):
+    """The forward with the Qv score term, scale * (q.k + qv.v): q, qv [total_q, Hq, D] bf16;
+    K/V paged or packed as in attn_fwd_varlen_paged.
+    Returns (o [total_q, Hq, D] bf16, lse [Hq, total_q] fp32)."""
+    total_q, Hq, D = q.shape
+    B = cu_seqlens_q.numel() - 1
+    if block_table is not None:
+        num_blocks, block_size, Hkv = k_cache.shape[0], k_cache.shape[1], k_cache.shape[2]
+        mbps, total_k = block_table.shape[1], 0
+    else:
+        num_blocks, block_size, mbps = 0, 0, 0
+        total_k, Hkv = k_cache.shape[0], k_cache.shape[1]
+    if out is None:
+        out = torch.empty((total_q, Hq, D), dtype=torch.bfloat16, device=q.device)
+    if lse is None and return_lse:
+        lse = torch.empty((Hq, total_q), dtype=torch.float32, device=q.device)
+    st = lib().attn_fwd_varlen_paged_qv(
+        _ptr(q), _ptr(qv), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), mbps, num_blocks,
+        block_size, _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), _ptr(seqused_k), B, total_q, total_k,
+        int(max_seqlen_q), Hq, Hkv, D, _scale(scale), int(mask), _ptr(patch_kv_range),
+        int(window_left), float(softcap), _dtype_code(q), _ptr(out), _ptr(lse), _stream(stream))
+    _check(st, "attn_fwd_varlen_paged_qv")
     return out, lse
 
 

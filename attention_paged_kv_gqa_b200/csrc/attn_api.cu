@@ -44,7 +44,7 @@ attn_status_t check_device_uncached(int device) {
     cudaGetDevice(&prev);
     if (prev != device) cudaSetDevice(device);
     cudaFuncAttributes fa;
-    const cudaError_t e = cudaFuncGetAttributes(&fa, prefill_kernel<128, false, false, false>);
+    const cudaError_t e = cudaFuncGetAttributes(&fa, prefill_kernel<128, false, false, false, false>);
     if (prev != device && prev >= 0) cudaSetDevice(prev);
     if (e != cudaSuccess) {
         cudaGetLastError();
@@ -222,51 +222,62 @@ attn_status_t launch_maybe_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, 
 }
 
 // ------------------------------------------------------------------ prefill dispatch
-template <int D, bool FP8, bool CAP, bool OQ>
+template <int D, bool FP8, bool CAP, bool OQ, bool HQ = false>
 attn_status_t launch_prefill_t(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                               const PrefillArgs& a, long long grid, cudaStream_t stream) {
-    using Cfg = PrefillCfg<D, FP8>;
+                               const CUtensorMap& mqv, const PrefillArgs& a, long long grid,
+                               cudaStream_t stream) {
+    using Cfg = PrefillCfg<D, FP8, HQ>;
     static std::atomic<uint64_t> attr_mask{0};   // one bit per device
     int dev = 0;
     cudaGetDevice(&dev);
     const uint64_t bit = 1ull << (dev & 63);
     if (!(attr_mask.load() & bit)) {
-        const attn_status_t s = set_smem(prefill_kernel<D, FP8, CAP, OQ>, Cfg::SMEM_BYTES);
+        const attn_status_t s = set_smem(prefill_kernel<D, FP8, CAP, OQ, HQ>, Cfg::SMEM_BYTES);
         if (s != ATTN_OK) return s;
         attr_mask.fetch_or(bit);
     }
-    prefill_kernel<D, FP8, CAP, OQ><<<static_cast<unsigned>(grid), kPrefillThreads, Cfg::SMEM_BYTES, stream>>>(
-        mq, mk, mv, a);
+    prefill_kernel<D, FP8, CAP, OQ, HQ><<<static_cast<unsigned>(grid), kPrefillThreads, Cfg::SMEM_BYTES, stream>>>(
+        mq, mk, mv, mqv, a);
     return launch_status();
 }
 
 attn_status_t launch_prefill(int D, int dtype, const CUtensorMap& mq, const CUtensorMap& mk,
                              const CUtensorMap& mv, const PrefillArgs& a, long long grid,
-                             cudaStream_t stream) {
+                             cudaStream_t stream, const CUtensorMap* mqv = nullptr) {
     if (grid <= 0) return ATTN_OK;
     if (grid >= (1LL << 31)) return ATTN_ERR_UNSUPPORTED;
     const bool cap = a.softcap > 0.0f;
+    if (mqv) {
+        // the Qv score term (bf16)
+        if (dtype == ATTN_BF16 && D == 128)
+            return cap ? launch_prefill_t<128, false, true, false, true>(mq, mk, mv, *mqv, a, grid, stream)
+                       : launch_prefill_t<128, false, false, false, true>(mq, mk, mv, *mqv, a, grid, stream);
+        if (dtype == ATTN_BF16 && D == 64)
+            return cap ? launch_prefill_t<64, false, true, false, true>(mq, mk, mv, *mqv, a, grid, stream)
+                       : launch_prefill_t<64, false, false, false, true>(mq, mk, mv, *mqv, a, grid, stream);
+        return ATTN_ERR_UNSUPPORTED;
+    }
     if (a.only_qv) {
         if (dtype == ATTN_BF16 && D == 128)
-            return cap ? launch_prefill_t<128, false, true, true>(mq, mk, mv, a, grid, stream)
-                       : launch_prefill_t<128, false, false, true>(mq, mk, mv, a, grid, stream);
+            return cap ? launch_prefill_t<128, false, true, true>(mq, mk, mv, mq, a, grid, stream)
+                       : launch_prefill_t<128, false, false, true>(mq, mk, mv, mq, a, grid, stream);
         if (dtype == ATTN_BF16 && D == 64)
-            return cap ? launch_prefill_t<64, false, true, true>(mq, mk, mv, a, grid, stream)
-                       : launch_prefill_t<64, false, false, true>(mq, mk, mv, a, grid, stream);
+            return cap ? launch_prefill_t<64, false, true, true>(mq, mk, mv, mq, a, grid, stream)
+                       : launch_prefill_t<64, false, false, true>(mq, mk, mv, mq, a, grid, stream);
         if (dtype == ATTN_FP8_E4M3 && D == 128)
-            return cap ? launch_prefill_t<128, true, true, true>(mq, mk, mv, a, grid, stream)
-                       : launch_prefill_t<128, true, false, true>(mq, mk, mv, a, grid, stream);
+            return cap ? launch_prefill_t<128, true, true, true>(mq, mk, mv, mq, a, grid, stream)
+                       : launch_prefill_t<128, true, false, true>(mq, mk, mv, mq, a, grid, stream);
         return ATTN_ERR_UNSUPPORTED;
     }
     if (dtype == ATTN_BF16 && D == 128)
-        return cap ? launch_prefill_t<128, false, true, false>(mq, mk, mv, a, grid, stream)
-                   : launch_prefill_t<128, false, false, false>(mq, mk, mv, a, grid, stream);
+        return cap ? launch_prefill_t<128, false, true, false>(mq, mk, mv, mq, a, grid, stream)
+                   : launch_prefill_t<128, false, false, false>(mq, mk, mv, mq, a, grid, stream);
     if (dtype == ATTN_BF16 && D == 64)
-        return cap ? launch_prefill_t<64, false, true, false>(mq, mk, mv, a, grid, stream)
-                   : launch_prefill_t<64, false, false, false>(mq, mk, mv, a, grid, stream);
+        return cap ? launch_prefill_t<64, false, true, false>(mq, mk, mv, mq, a, grid, stream)
+                   : launch_prefill_t<64, false, false, false>(mq, mk, mv, mq, a, grid, stream);
     if (dtype == ATTN_FP8_E4M3 && D == 128)
-        return cap ? launch_prefill_t<128, true, true, false>(mq, mk, mv, a, grid, stream)
-                   : launch_prefill_t<128, true, false, false>(mq, mk, mv, a, grid, stream);
+        return cap ? launch_prefill_t<128, true, true, false>(mq, mk, mv, mq, a, grid, stream)
+                   : launch_prefill_t<128, true, false, false>(mq, mk, mv, mq, a, grid, stream);
     return ATTN_ERR_UNSUPPORTED;
 }
 
@@ -621,7 +632,8 @@ static attn_status_t fwd_varlen_paged_impl(
     const int32_t* cu_seqlens_k, const int32_t* seqused_k, int B, int total_q, int total_k,
     int max_seqlen_q, int Hq, int Hkv, int D, float softmax_scale, int mask,
     const int32_t* patch_kv_range, int window_left, float softcap, int dtype, const float* dq,
-    const float* dk, const float* dv, void* o, float* lse, attn_stream_t stream, int only_qv) {
+    const float* dk, const float* dv, void* o, float* lse, attn_stream_t stream, int only_qv,
+    const void* qv = nullptr) {
     if (!q || !k_cache || !v_cache || !o || !cu_seqlens_q) return ATTN_ERR_INVALID_ARG;
     if (B < 0 || total_q < 0 || max_seqlen_q < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0)
         return ATTN_ERR_INVALID_ARG;
@@ -634,6 +646,7 @@ static attn_status_t fwd_varlen_paged_impl(
     }
     if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
     if (dtype == ATTN_FP8_E4M3 && D != 128) return ATTN_ERR_UNSUPPORTED;
+    if (qv && (dtype != ATTN_BF16 || only_qv)) return ATTN_ERR_UNSUPPORTED;
     if (dtype == ATTN_FP8_E4M3 && (!dq || !dk || !dv)) return ATTN_ERR_INVALID_ARG;
     const bool paged = block_table != nullptr;
     if (paged) {
@@ -646,6 +659,7 @@ static attn_status_t fwd_varlen_paged_impl(
     }
     if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o))
         return ATTN_ERR_INVALID_ARG;
+    if (qv && !aligned16(qv)) return ATTN_ERR_INVALID_ARG;
     const int E = elem_bytes(dtype);
     if ((D * E) % 16) return ATTN_ERR_INVALID_ARG;
     const attn_status_t dvs = current_device_ok(nullptr);
@@ -665,6 +679,8 @@ static attn_status_t fwd_varlen_paged_impl(
     const uint32_t bkv[4] = {(uint32_t)chunk, 1, (uint32_t)(paged ? kPageRows : kBN), 1};
     attn_status_t s;
     if ((s = get_map(&mq, q, dtype, dq4, sq3, bq)) != ATTN_OK) return s;
+    CUtensorMap mqv;
+    if (qv && (s = get_map(&mqv, qv, dtype, dq4, sq3, bq)) != ATTN_OK) return s;
     if ((s = get_map(&mv, v_cache, dtype, dk4, sk3, bkv)) != ATTN_OK) return s;
     if (only_qv) mk = mv;   // no key store: its map is never used
     else if ((s = get_map(&mk, k_cache, dtype, dk4, sk3, bkv)) != ATTN_OK) return s;
@@ -700,7 +716,8 @@ static attn_status_t fwd_varlen_paged_impl(
     a.lse_stride_b = 0;
     long long grid;
     unit_grid(a, max_seqlen_q, &grid);
-    return launch_prefill(D, dtype, mq, mk, mv, a, grid, static_cast<cudaStream_t>(stream));
+    return launch_prefill(D, dtype, mq, mk, mv, a, grid, static_cast<cudaStream_t>(stream),
+                          qv ? &mqv : nullptr);
 }
 
 attn_status_t attn_fwd_varlen_paged(
@@ -718,6 +735,21 @@ attn_status_t attn_fwd_varlen_paged(
                                  total_k, max_seqlen_q, Hq, Hkv, D, softmax_scale, mask,
                                  patch_kv_range, window_left, softcap, dtype, dq, dk, dv, o, lse,
                                  stream, 0);
+}
+
+attn_status_t attn_fwd_varlen_paged_qv(
+    const void* q, const void* qv, const void* k_cache, const void* v_cache,
+    const int32_t* block_table, int max_blocks_per_seq, int num_blocks, int block_size,
+    const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, const int32_t* seqused_k, int B,
+    int total_q, int total_k, int max_seqlen_q, int Hq, int Hkv, int D, float softmax_scale,
+    int mask, const int32_t* patch_kv_range, int window_left, float softcap, int dtype, void* o,
+    float* lse, attn_stream_t stream) {
+    if (!qv) return ATTN_ERR_INVALID_ARG;
+    return fwd_varlen_paged_impl(q, k_cache, v_cache, block_table, max_blocks_per_seq, num_blocks,
+                                 block_size, cu_seqlens_q, cu_seqlens_k, seqused_k, B, total_q,
+                                 total_k, max_seqlen_q, Hq, Hkv, D, softmax_scale, mask,
+                                 patch_kv_range, window_left, softcap, dtype, nullptr, nullptr,
+                                 nullptr, o, lse, stream, 0, qv);
 }
 
 attn_status_t attn_fwd_varlen_paged_only_qv(

@@ -82,7 +82,7 @@ struct PrefillArgs {
     int NQ;              // query units per sequence (grid extent)
 };
 
-template <int D, bool FP8>
+template <int D, bool FP8, bool HQ = false>
 struct PrefillCfg {
     static constexpr int E = FP8 ? 1 : 2;              // bytes per element
     static constexpr int ROWB = D * E;                  // bytes per row
@@ -97,8 +97,20 @@ struct PrefillCfg {
     static constexpr int PV_STEPS = kBN / KSTEP;
     static constexpr uint32_t IDESC_QK = instr_desc(FP8 ? 0 : 1, FP8 ? 0 : 1, 0, 0, 128, kBN);
     static constexpr uint32_t IDESC_PV = instr_desc(FP8 ? 0 : 1, FP8 ? 0 : 1, 0, 1, 128, D);
+    // HQ (the Qv score term): the Qv sub-tiles beside the Q sub-tiles, and the rings
+    // as deep as the rest allows -- at D = 128 one key stage (a key tile is released
+    // by its score GEMM, long before the next one is due) and two value stages (the
+    // score GEMM of tile j + 1 reads V(j + 1) while P.V of tile j still reads V(j))
+    static constexpr int QBUF = (HQ ? 4 : 2) * QB;
+    static constexpr int NS_HQ = (4 * QB + 4 * 2 * KVB + 2048 <= 227 * 1024) ? 4
+                                 : (4 * QB + 3 * 2 * KVB + 2048 <= 227 * 1024) ? 3
+                                 : (4 * QB + 2 * 2 * KVB + 2048 <= 227 * 1024) ? 2 : 0;
+    static constexpr int NSK = HQ ? (NS_HQ ? NS_HQ : 1) : NS;   // key stages
+    static constexpr int NSV = HQ ? (NS_HQ ? NS_HQ : 2) : NS;   // value stages
     static constexpr int NBAR = 1 + 4 * NS + 2 + 2 + 2 + 1;
-    static constexpr int SMEM_BYTES = 1024 /*align slack*/ + 2 * QB + 2 * NS * KVB + 1024;
+    static constexpr int SMEM_BYTES = 1024 /*align slack*/ + QBUF + (NSK + NSV) * KVB + 1024;
+    static_assert(NSK <= NS && NSV <= NS, "barrier arrays are NS deep");
+    static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
     static_assert(ROWB % 128 == 0, "rows must be whole 128-byte swizzle columns");
     static_assert(NBAR * 8 + 64 <= 1024, "barrier area");
 };
@@ -108,24 +120,32 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 }
 
 // CAP: the score softcap is compiled in (a separate instance, so that the
-// uncapped kernel carries none of its code).  OQ: the only_qv score, Qv . V --
+// uncapped kernel carries none of its code).  HQ: the score adds the Qv term of
+// the "Rope dim" forward (HasQv), q . k + q_v . v: a second score GEMM of the
+// Qv sub-tile against the value tile (K-major, as the key tile), which must then
+// have landed before the score GEMM; bf16.  OQ: the only_qv score, Qv . V --
 // no key tiles are fetched, the value tile is the score GEMM's B operand, and
 // the key stages and barriers deepen the value ring to 2 NS slots.  Both are
 // template parameters because the single MMA-issuing thread's control path is
 // on the critical path: runtime switches there cost measurable throughput.
-template <int D, bool FP8, bool CAP, bool OQ>
+template <int D, bool FP8, bool CAP, bool OQ, bool HQ>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                   const __grid_constant__ CUtensorMap tmV, const PrefillArgs a) {
-    using C = PrefillCfg<D, FP8>;
-    constexpr int NS = C::NS;
+                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmQv,
+                   const PrefillArgs a) {
+    using C = PrefillCfg<D, FP8, HQ>;
+    static_assert(!(HQ && (OQ || FP8)), "the Qv score term is a bf16 instance of its own");
+    constexpr int NS = C::NS;       // barrier arrays
+    constexpr int NSK = C::NSK;     // key ring
+    constexpr int NSV = C::NSV;     // value stages
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
     uint8_t* sQ = smem;
-    uint8_t* sK = sQ + 2 * C::QB;
-    uint8_t* sV = sK + NS * C::KVB;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(sV + NS * C::KVB);
+    uint8_t* sQv = sQ + 2 * C::QB;          // HQ only
+    uint8_t* sK = sQ + C::QBUF;
+    uint8_t* sV = sK + NSK * C::KVB;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sV + NSV * C::KVB);
     uint64_t* q_full = bars;
     uint64_t* k_full = bars + 1;
     uint64_t* k_empty = k_full + NS;
@@ -138,10 +158,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
     // Value ring: the NS value stages, and with only_qv (no key tiles) the NS key
     // stages and their barriers too, so that 2 NS value tiles can be in flight.
-    constexpr int vring = OQ ? 2 * NS : NS;
-    auto vslot_buf = [&](int st) { return st < NS ? sV + st * C::KVB : sK + (st - NS) * C::KVB; };
-    auto vslot_full = [&](int st) { return st < NS ? &v_full[st] : &k_full[st - NS]; };
-    auto vslot_empty = [&](int st) { return st < NS ? &v_empty[st] : &k_empty[st - NS]; };
+    constexpr int vring = OQ ? 2 * NS : NSV;
+    auto vslot_buf = [&](int st) { return st < NSV ? sV + st * C::KVB : sK + (st - NSV) * C::KVB; };
+    auto vslot_full = [&](int st) { return st < NSV ? &v_full[st] : &k_full[st - NSV]; };
+    auto vslot_empty = [&](int st) { return st < NSV ? &v_empty[st] : &k_empty[st - NSV]; };
     int* sched = reinterpret_cast<int*>(tmem_slot + 2);   // [t][0]=min start, [t][1]=max end
 
     // ------------------------------------------------------------ work unit (a1)
@@ -277,6 +297,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             prefetch_tmap(&tmQ);
             prefetch_tmap(&tmK);
             prefetch_tmap(&tmV);
+            if constexpr (HQ) prefetch_tmap(&tmQv);
         }
         int issued = 0;
         if (any_tiles) {
@@ -285,21 +306,25 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
 #pragma unroll
                 for (int t = 0; t < 2; ++t)
                     if (hi_t[t] > lo_t[t]) qbytes += C::QB;
-                mbar_arrive_expect_tx(q_full, qbytes);
+                mbar_arrive_expect_tx(q_full, HQ ? 2 * qbytes : qbytes);
 #pragma unroll
                 for (int t = 0; t < 2; ++t) {
                     if (hi_t[t] <= lo_t[t]) continue;
 #pragma unroll
-                    for (int c = 0; c < C::NCHUNK; ++c)
+                    for (int c = 0; c < C::NCHUNK; ++c) {
                         tma_load_4d(&tmQ, q_full, sQ + t * C::QB + c * kBM * 128, c * C::CHUNK_E,
                                     head[t], q_off + q0[t], bcoord);
+                        if constexpr (HQ)
+                            tma_load_4d(&tmQv, q_full, sQv + t * C::QB + c * kBM * 128, c * C::CHUNK_E,
+                                        head[t], q_off + q0[t], bcoord);
+                    }
                 }
             }
             const uint64_t pol = policy_evict_last();
             for (int j = lo; j < hi; ++j, ++issued) {
                 const int it = j - lo;
-                const int st = it % NS;
-                const uint32_t ph = (it / NS) & 1;
+                const int st = it % NSK;
+                const uint32_t ph = (it / NSK) & 1;
                 const int vst = it % vring;                 // value ring (2 NS deep with only_qv)
                 const uint32_t vph = (it / vring) & 1;
                 uint64_t* vfull = vslot_full(vst);
@@ -371,11 +396,15 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             }
             // Let every copy this warp started land before the CTA can exit.
             if (lane == 0) {
+                if constexpr (!OQ) {
+                    for (int st = 0; st < NSK && st < issued; ++st) {
+                        const int last = st + ((issued - 1 - st) / NSK) * NSK;
+                        mbar_wait_drain(&k_full[st], (last / NSK) & 1, kErrProdDrain);
+                    }
+                }
                 for (int st = 0; st < vring && st < issued; ++st) {
                     const int last = st + ((issued - 1 - st) / vring) * vring;
-                    const uint32_t ph = (last / vring) & 1;
-                    if (!OQ) mbar_wait_drain(&k_full[st], ph, kErrProdDrain);
-                    mbar_wait_drain(vslot_full(st), ph, kErrProdDrain);
+                    mbar_wait_drain(vslot_full(st), (last / vring) & 1, kErrProdDrain);
                 }
             }
         }
@@ -388,7 +417,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             auto part = [&](int t, int j) { return lo_t[t] <= j && j < hi_t[t]; };
             // score GEMM: B operand at kb (the key tile; with only_qv the value tile, whose
             // slot is released by the P.V GEMM that reads it last)
-            auto issue_s = [&](int t, uint32_t kb) {
+            auto issue_s = [&](int t, uint32_t kb, uint32_t vb) {
 #pragma unroll
                 for (int kk = 0; kk < C::QK_STEPS; ++kk) {
                     const uint32_t cb = (kk * 32) / 128, off = (kk * 32) % 128;
@@ -398,6 +427,19 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                     const uint64_t db = smem_desc(ka, 16, 1024, 2);
                     if constexpr (FP8) mma_f8_ss(tS[t], da, db, C::IDESC_QK, kk > 0);
                     else mma_f16_ss(tS[t], da, db, C::IDESC_QK, kk > 0);
+                }
+                if constexpr (HQ) {
+                    // + Qv V^T: the value tile read K-major, exactly as the key tile
+                    const uint32_t sQva = smem_u32(sQv);
+#pragma unroll
+                    for (int kk = 0; kk < C::QK_STEPS; ++kk) {
+                        const uint32_t cb = (kk * 32) / 128, off = (kk * 32) % 128;
+                        const uint64_t da = smem_desc(sQva + t * C::QB + cb * kBM * 128 + off, 16, 1024, 2);
+                        const uint64_t db = smem_desc(vb + cb * kBN * 128 + off, 16, 1024, 2);
+                        mma_f16_ss(tS[t], da, db, C::IDESC_QK, 1u);
+                    }
+                } else {
+                    (void)vb;
                 }
             };
             auto issue_pv = [&](int t, uint32_t vb, bool acc) {
@@ -414,21 +456,22 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             bool started[2] = {false, false};
             int pcount[2] = {0, 0};
             if (ok) ok = mbar_wait(OQ ? vslot_full(0) : &k_full[0], 0, kErrMmaK);
+            if (HQ && ok) ok = mbar_wait(vslot_full(0), 0, kErrMmaV);
             if (ok) {
                 tc_fence_after();
                 const uint32_t kb0 = OQ ? smem_u32(vslot_buf(0)) : sKa;
 #pragma unroll
                 for (int t = 0; t < 2; ++t)
                     if (part(t, lo)) {
-                        issue_s(t, kb0);
+                        issue_s(t, kb0, smem_u32(vslot_buf(0)));
                         mma_commit(&s_full[t]);
                     }
                 if (!OQ) mma_commit(&k_empty[0]);
             }
             for (int j = lo; ok && j < hi; ++j) {
                 const int it = j - lo;
-                const int st1 = (it + 1) % NS;
-                const uint32_t ph1 = ((it + 1) / NS) & 1;
+                const int st1 = (it + 1) % NSK;
+                const uint32_t ph1 = ((it + 1) / NSK) & 1;
                 const int vst = it % vring, vst1 = (it + 1) % vring;
                 const uint32_t vph = (it / vring) & 1, vph1 = ((it + 1) / vring) & 1;
                 const bool next = j + 1 < hi;
@@ -448,11 +491,13 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                         if (!k1) {
                             ok = OQ ? mbar_wait(vslot_full(vst1), vph1, kErrMmaK)
                                            : mbar_wait(&k_full[st1], ph1, kErrMmaK);
+                            if (HQ && ok) ok = mbar_wait(vslot_full(vst1), vph1, kErrMmaV);
                             if (!ok) break;
                             tc_fence_after();
                             k1 = true;
                         }
-                        issue_s(t, OQ ? smem_u32(vslot_buf(vst1)) : sKa + st1 * C::KVB);
+                        issue_s(t, OQ ? smem_u32(vslot_buf(vst1)) : sKa + st1 * C::KVB,
+                                smem_u32(vslot_buf(vst1)));
                         mma_commit(&s_full[t]);
                     }
                 }

@@ -205,6 +205,26 @@ attn_status_t attn_fwd_patch(
     const float *descale_v, void *o, float *lse, attn_stream_t stream);
 
 /*
+ * The forward with the extra Qv score term of "Rope dim" (vllm-project
+ * flash-attention PR 172, overview: the Qv GEMM beside the QK GEMM, HasQv): the
+ * logit of query i and key j is scale * (q_i . k_j + qv_i . v_j), then softcap,
+ * masks, softmax and P.V as in attn_fwd_varlen_paged.
+ *   qv           [total_q, Hq, D] bf16, laid out as q, 16-byte aligned; the
+ *                value head dimension equals the key one here.
+ *   other arguments as attn_fwd_varlen_paged (no descales: bf16 only).
+ * Supported: bf16, head_dim in {64, 128}; fp8 gives ATTN_ERR_UNSUPPORTED and
+ * qv NULL ATTN_ERR_INVALID_ARG.  The value tile is read once per key tile and
+ * feeds both the second score GEMM and the P.V GEMM.
+ */
+attn_status_t attn_fwd_varlen_paged_qv(
+    const void *q, const void *qv, const void *k_cache, const void *v_cache,
+    const int32_t *block_table, int max_blocks_per_seq, int num_blocks, int block_size,
+    const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k, const int32_t *seqused_k, int B,
+    int total_q, int total_k, int max_seqlen_q, int num_heads_q, int num_heads_kv, int head_dim,
+    float softmax_scale, int mask, const int32_t *patch_kv_range, int window_left, float softcap,
+    int dtype, void *o, float *lse, attn_stream_t stream);
+
+/*
  * The only_qv score path of "Rope dim" (vllm-project flash-attention PR 172,
  * overview: the mode that skips the Q and K loads and the QK GEMM and
  * zero-initialises the score with the Qv GEMM).  The score of query i and key

@@ -233,3 +233,17 @@ def test_decode_qv_argument_checks(L):
     assert dec(splits=2) == 2
     assert dec(dtype=1) == 2
     assert dec(Hq=32, Hkv=16) == 2
+
+
+def test_fwd_qv_argument_checks(L):
+    """The forward with the Qv term: qv required; bf16 only; head_dim 64 / 128."""
+    p = ctypes.c_void_p(1 << 20)
+    cu = ctypes.c_void_p(1 << 21)
+
+    def fwd(qv=p, D=128, dtype=0):
+        return L.attn_fwd_varlen_paged_qv(p, qv, p, p, p, 4, 100, 16, cu, None, cu, 1, 16, 0, 16,
+                                          2, 2, D, 0.0, 1, None, -1, 0.0, dtype, p, None, None)
+
+    assert fwd(qv=None) == 1
+    assert fwd(D=96) == 2
+    assert fwd(dtype=1) == 2
