@@ -862,6 +862,56 @@ def run_only_qv(c):
     c["line"]["only_qv"] = out
     c["launches"] += 3 * args.steps
     c["line"]["gpu_launches"] = c["launches"]
+    run_qv(c)
+
+
+def run_qv(c):
+    """The score with the extra Qv term, scale * (q.k + qv.v), on the decode and varlen prefill
+    workloads (qv a second seeded bf16 tensor of q's shape)."""
+    args, A, W, dev, world, flush = c["args"], c["A"], c["W"], c["dev"], c["world"], c["flush"]
+    peaks = c["peaks"]
+    w = W.paged_decode(seed=args.seed)
+    t, P = w.tensors, w.params
+    d = {k: v.to(dev) for k, v in t.items()}
+    qv = W.randn_bf16(tuple(t["q"].shape), args.seed, 51).to(dev)
+    ws = torch.empty(max(A.attn_decode_workspace_size(P["B"], P["Hq"], P["Hkv"], P["D"],
+                                                      P["max_blocks_per_seq"]), 16),
+                     dtype=torch.uint8, device=dev)
+    o = torch.empty(P["B"], P["Hq"], P["D"], dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(P["B"], P["Hq"], dtype=torch.float32, device=dev)
+
+    def dec_step():
+        A.attn_decode_paged_qv(d["q"], qv, d["k_cache"], d["v_cache"], d["block_table"],
+                               d["seqused_k"], scale=P["scale"], out=o, lse=lse, workspace=ws)
+
+    dms = statistics.mean(time_steps(dec_step, args.steps, args.warmup, world, flush))
+    nb = decode_bytes(t, P["Hq"], P["Hkv"], P["D"]) + int(qv.numel()) * 2
+    out = {"decode": entry(nb / (dms * 1e-3) / 1e9, "GB/s", dms, "hbm", peaks)}
+    del d
+
+    wp = W.varlen_paged_prefill(seed=args.seed)
+    tp, Pp = wp.tensors, wp.params
+    dp = {k: v.to(dev) for k, v in tp.items()}
+    qvp = W.randn_bf16(tuple(tp["q"].shape), args.seed, 52).to(dev)
+    op = torch.empty(Pp["total_q"], Pp["Hq"], Pp["D"], dtype=torch.bfloat16, device=dev)
+    lp = torch.empty(Pp["Hq"], Pp["total_q"], dtype=torch.float32, device=dev)
+
+    def pf_step():
+        A.attn_fwd_varlen_paged_qv(dp["q"], qvp, dp["k_cache"], dp["v_cache"],
+                                   cu_seqlens_q=dp["cu_seqlens_q"], max_seqlen_q=Pp["max_seqlen_q"],
+                                   block_table=dp["block_table"], seqused_k=dp["seqused_k"],
+                                   mask=A.MASK_CAUSAL, scale=Pp["scale"], out=op, lse=lp)
+
+    pms = statistics.mean(time_steps(pf_step, args.steps, args.warmup, world, flush))
+    # three GEMMs per allowed pair (q.k, qv.v, P.V): 6 D flops per pair and query head
+    fl = causal_flops(tp["seqused_k"].numpy(), Pp["Hq"], Pp["D"]) * 1.5
+    out["prefill"] = entry(fl / (pms * 1e-3) / 1e12, "TFLOP/s", pms, "tensor", peaks)
+    del dp
+    out["note"] = ("score scale * (q.k + qv.v); decode bytes add qv, prefill flops count three "
+                   "GEMMs (6 D per allowed pair and query head)")
+    c["line"]["qv"] = out
+    c["launches"] += 3 * args.steps
+    c["line"]["gpu_launches"] = c["launches"]
 
 
 def run_patch_and_small(c):
