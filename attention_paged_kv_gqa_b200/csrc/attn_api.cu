@@ -150,13 +150,16 @@ attn_status_t get_map(CUtensorMap* out, const void* ptr, int dtype, const uint64
     if (!enc) return ATTN_ERR_TMA_ENCODE;
     CUtensorMap m;
     const cuuint32_t estride[4] = {1, 1, 1, 1};
+    // the swizzle span is the box's row: 128 bytes, or 64 (e4m3 rows of head_dim 64)
+    const uint32_t row_bytes = box[0] * (dtype == ATTN_FP8_E4M3 ? 1u : 2u);
+    const CUtensorMapSwizzle swz = row_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
     const CUresult r = enc(&m,
                            dtype == ATTN_FP8_E4M3 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
                                                   : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
                            4, const_cast<void*>(ptr), reinterpret_cast<const cuuint64_t*>(dims),
                            reinterpret_cast<const cuuint64_t*>(strides),
                            reinterpret_cast<const cuuint32_t*>(box), estride,
-                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return ATTN_ERR_TMA_ENCODE;
     MapEntry& e = g_maps[g_map_next];
@@ -267,6 +270,9 @@ attn_status_t launch_prefill(int D, int dtype, const CUtensorMap& mq, const CUte
         if (dtype == ATTN_FP8_E4M3 && D == 128)
             return cap ? launch_prefill_t<128, true, true, true>(mq, mk, mv, mq, a, grid, stream)
                        : launch_prefill_t<128, true, false, true>(mq, mk, mv, mq, a, grid, stream);
+        if (dtype == ATTN_FP8_E4M3 && D == 64)
+            return cap ? launch_prefill_t<64, true, true, true>(mq, mk, mv, mq, a, grid, stream)
+                       : launch_prefill_t<64, true, false, true>(mq, mk, mv, mq, a, grid, stream);
         return ATTN_ERR_UNSUPPORTED;
     }
     if (dtype == ATTN_BF16 && D == 128)
@@ -278,6 +284,9 @@ attn_status_t launch_prefill(int D, int dtype, const CUtensorMap& mq, const CUte
     if (dtype == ATTN_FP8_E4M3 && D == 128)
         return cap ? launch_prefill_t<128, true, true, false>(mq, mk, mv, mq, a, grid, stream)
                    : launch_prefill_t<128, true, false, false>(mq, mk, mv, mq, a, grid, stream);
+    if (dtype == ATTN_FP8_E4M3 && D == 64)
+        return cap ? launch_prefill_t<64, true, true, false>(mq, mk, mv, mq, a, grid, stream)
+                   : launch_prefill_t<64, true, false, false>(mq, mk, mv, mq, a, grid, stream);
     return ATTN_ERR_UNSUPPORTED;
 }
 
@@ -568,7 +577,6 @@ attn_status_t attn_fwd_dense(const void* q, const void* k, const void* v, void* 
         if (ms != ATTN_OK) return ms;
     }
     if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
-    if (dtype == ATTN_FP8_E4M3 && (D != 128)) return ATTN_ERR_UNSUPPORTED;
     if (dtype == ATTN_FP8_E4M3 && (!dq || !dk || !dv)) return ATTN_ERR_INVALID_ARG;
     const int E = elem_bytes(dtype);
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return ATTN_ERR_INVALID_ARG;
@@ -582,7 +590,7 @@ attn_status_t attn_fwd_dense(const void* q, const void* k, const void* v, void* 
     if (dvs != ATTN_OK) return dvs;
     if (B == 0 || Lq == 0) return ATTN_OK;
 
-    const int chunk = 128 / E;
+    const int chunk = std::min(128 / E, D);   // one swizzle column of a row
     CUtensorMap mq, mk, mv;
     const uint64_t dq4[4] = {(uint64_t)D, (uint64_t)Hq, (uint64_t)Lq, (uint64_t)B};
     const uint64_t sq3[3] = {(uint64_t)(sq[2] * E), (uint64_t)(sq[1] * E), (uint64_t)(sq[0] * E)};
@@ -645,7 +653,6 @@ static attn_status_t fwd_varlen_paged_impl(
         if (ms != ATTN_OK) return ms;
     }
     if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
-    if (dtype == ATTN_FP8_E4M3 && D != 128) return ATTN_ERR_UNSUPPORTED;
     if (qv && (dtype != ATTN_BF16 || only_qv)) return ATTN_ERR_UNSUPPORTED;
     if (dtype == ATTN_FP8_E4M3 && (!dq || !dk || !dv)) return ATTN_ERR_INVALID_ARG;
     const bool paged = block_table != nullptr;
@@ -666,7 +673,7 @@ static attn_status_t fwd_varlen_paged_impl(
     if (dvs != ATTN_OK) return dvs;
     if (B == 0 || total_q == 0 || max_seqlen_q == 0) return ATTN_OK;
 
-    const int chunk = 128 / E;
+    const int chunk = std::min(128 / E, D);   // one swizzle column of a row
     CUtensorMap mq, mk, mv;
     const uint64_t rowq = (uint64_t)Hq * D * E;
     const uint64_t dq4[4] = {(uint64_t)D, (uint64_t)Hq, (uint64_t)total_q, 1};

@@ -86,8 +86,11 @@ template <int D, bool FP8, bool HQ = false>
 struct PrefillCfg {
     static constexpr int E = FP8 ? 1 : 2;              // bytes per element
     static constexpr int ROWB = D * E;                  // bytes per row
-    static constexpr int NCHUNK = ROWB / 128;           // 128-byte swizzle columns per row
-    static constexpr int CHUNK_E = 128 / E;             // elements per swizzle column
+    // swizzle span: 128-byte columns, or one 64-byte column for 64-byte rows (fp8, D = 64)
+    static constexpr int SW = ROWB >= 128 ? 128 : 64;
+    static constexpr uint32_t SWZ = SW == 128 ? 2u : 4u;   // descriptor layout code
+    static constexpr int NCHUNK = ROWB / SW;            // swizzle columns per row
+    static constexpr int CHUNK_E = SW / E;              // elements per swizzle column
     static constexpr int QB = kBM * ROWB;
     static constexpr int KVB = kBN * ROWB;
     static constexpr int NS = (2 * QB + 4 * 2 * KVB + 2048 <= 227 * 1024) ? 4
@@ -111,7 +114,7 @@ struct PrefillCfg {
     static constexpr int SMEM_BYTES = 1024 /*align slack*/ + QBUF + (NSK + NSV) * KVB + 1024;
     static_assert(NSK <= NS && NSV <= NS, "barrier arrays are NS deep");
     static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
-    static_assert(ROWB % 128 == 0, "rows must be whole 128-byte swizzle columns");
+    static_assert(ROWB % SW == 0, "rows must be whole swizzle columns");
     static_assert(NBAR * 8 + 64 <= 1024, "barrier area");
 };
 
@@ -312,10 +315,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                     if (hi_t[t] <= lo_t[t]) continue;
 #pragma unroll
                     for (int c = 0; c < C::NCHUNK; ++c) {
-                        tma_load_4d(&tmQ, q_full, sQ + t * C::QB + c * kBM * 128, c * C::CHUNK_E,
+                        tma_load_4d(&tmQ, q_full, sQ + t * C::QB + c * kBM * C::SW, c * C::CHUNK_E,
                                     head[t], q_off + q0[t], bcoord);
                         if constexpr (HQ)
-                            tma_load_4d(&tmQv, q_full, sQv + t * C::QB + c * kBM * 128, c * C::CHUNK_E,
+                            tma_load_4d(&tmQv, q_full, sQv + t * C::QB + c * kBM * C::SW, c * C::CHUNK_E,
                                         head[t], q_off + q0[t], bcoord);
                     }
                 }
@@ -357,10 +360,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                         if (lane == 0) mbar_arrive_expect_tx(&k_full[st], bytes);
                         __syncwarp();
                         if (lane < PPT && j * kBN + lane * kPageRows < Lk) {
-                            uint8_t* dst = sK + st * C::KVB + lane * kPageRows * 128;
+                            uint8_t* dst = sK + st * C::KVB + lane * kPageRows * C::SW;
 #pragma unroll
                             for (int c = 0; c < C::NCHUNK; ++c)
-                                tma_load_4d_hint(&tmK, &k_full[st], dst + c * kBN * 128, c * C::CHUNK_E, g,
+                                tma_load_4d_hint(&tmK, &k_full[st], dst + c * kBN * C::SW, c * C::CHUNK_E, g,
                                                  page * kPageRows, 0, pol);
                         }
                     } else if (lane == 0) {
@@ -368,7 +371,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                         uint8_t* dst = sK + st * C::KVB;
 #pragma unroll
                         for (int c = 0; c < C::NCHUNK; ++c)
-                            tma_load_4d_hint(&tmK, &k_full[st], dst + c * kBN * 128,
+                            tma_load_4d_hint(&tmK, &k_full[st], dst + c * kBN * C::SW,
                                              c * C::CHUNK_E, g, k_off + j * kBN, bcoord, pol);
                     }
                 }
@@ -380,17 +383,17 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                     if (lane == 0) mbar_arrive_expect_tx(vfull, bytes);
                     __syncwarp();
                     if (lane < PPT && j * kBN + lane * kPageRows < Lk) {
-                        uint8_t* dst = vbuf + lane * kPageRows * 128;
+                        uint8_t* dst = vbuf + lane * kPageRows * C::SW;
 #pragma unroll
                         for (int c = 0; c < C::NCHUNK; ++c)
-                            tma_load_4d_hint(&tmV, vfull, dst + c * kBN * 128, c * C::CHUNK_E, g,
+                            tma_load_4d_hint(&tmV, vfull, dst + c * kBN * C::SW, c * C::CHUNK_E, g,
                                              page * kPageRows, 0, pol);
                     }
                 } else if (lane == 0) {
                     mbar_arrive_expect_tx(vfull, bytes);
 #pragma unroll
                     for (int c = 0; c < C::NCHUNK; ++c)
-                        tma_load_4d_hint(&tmV, vfull, vbuf + c * kBN * 128,
+                        tma_load_4d_hint(&tmV, vfull, vbuf + c * kBN * C::SW,
                                          c * C::CHUNK_E, g, k_off + j * kBN, bcoord, pol);
                 }
             }
@@ -420,11 +423,13 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             auto issue_s = [&](int t, uint32_t kb, uint32_t vb) {
 #pragma unroll
                 for (int kk = 0; kk < C::QK_STEPS; ++kk) {
-                    const uint32_t cb = (kk * 32) / 128, off = (kk * 32) % 128;
-                    const uint32_t qa = sQa + t * C::QB + cb * kBM * 128 + off;
-                    const uint32_t ka = kb + cb * kBN * 128 + off;
-                    const uint64_t da = smem_desc(qa, 16, 1024, 2);
-                    const uint64_t db = smem_desc(ka, 16, 1024, 2);
+                    // K-major, 8-row groups SW * 8 bytes apart; a K step of 32 bytes
+                    // moves the start within the swizzle column
+                    const uint32_t cb = (kk * 32) / C::SW, off = (kk * 32) % C::SW;
+                    const uint32_t qa = sQa + t * C::QB + cb * kBM * C::SW + off;
+                    const uint32_t ka = kb + cb * kBN * C::SW + off;
+                    const uint64_t da = smem_desc(qa, 16, 8 * C::SW, C::SWZ);
+                    const uint64_t db = smem_desc(ka, 16, 8 * C::SW, C::SWZ);
                     if constexpr (FP8) mma_f8_ss(tS[t], da, db, C::IDESC_QK, kk > 0);
                     else mma_f16_ss(tS[t], da, db, C::IDESC_QK, kk > 0);
                 }
@@ -433,9 +438,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                     const uint32_t sQva = smem_u32(sQv);
 #pragma unroll
                     for (int kk = 0; kk < C::QK_STEPS; ++kk) {
-                        const uint32_t cb = (kk * 32) / 128, off = (kk * 32) % 128;
-                        const uint64_t da = smem_desc(sQva + t * C::QB + cb * kBM * 128 + off, 16, 1024, 2);
-                        const uint64_t db = smem_desc(vb + cb * kBN * 128 + off, 16, 1024, 2);
+                        const uint32_t cb = (kk * 32) / C::SW, off = (kk * 32) % C::SW;
+                        const uint64_t da = smem_desc(sQva + t * C::QB + cb * kBM * C::SW + off, 16, 8 * C::SW, C::SWZ);
+                        const uint64_t db = smem_desc(vb + cb * kBN * C::SW + off, 16, 8 * C::SW, C::SWZ);
                         mma_f16_ss(tS[t], da, db, C::IDESC_QK, 1u);
                     }
                 } else {
@@ -445,8 +450,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             auto issue_pv = [&](int t, uint32_t vb, bool acc) {
 #pragma unroll
                 for (int kk = 0; kk < C::PV_STEPS; ++kk) {
-                    const uint32_t va = vb + kk * (C::KSTEP / 8) * 1024;
-                    const uint64_t db = smem_desc(va, kBN * 128, 1024, 2);
+                    // MN-major: swizzle columns of d kBN * SW bytes apart (LBO), 8-key
+                    // groups 8 * SW bytes apart (SBO); a K step of KSTEP keys
+                    const uint32_t va = vb + kk * (C::KSTEP / 8) * (8 * C::SW);
+                    const uint64_t db = smem_desc(va, kBN * C::SW, 8 * C::SW, C::SWZ);
                     const uint32_t pa = tS[t] + kk * 8;
                     if constexpr (FP8) mma_f8_ts(tO[t], pa, db, C::IDESC_PV, (acc || kk > 0) ? 1u : 0u);
                     else mma_f16_ts(tO[t], pa, db, C::IDESC_PV, (acc || kk > 0) ? 1u : 0u);
@@ -685,13 +692,14 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                         const int first = Lk - j * kBN;
                         uint8_t* base = vslot_buf(st);
                         const int nrow = kBN - first;
-                        const int n16 = nrow * C::NCHUNK * 8;     // 16-byte pieces
+                        constexpr int PPR = C::SW / 16;           // 16-byte pieces per column row
+                        const int n16 = nrow * C::NCHUNK * PPR;
                         for (int i = r; i < n16; i += kBM) {
-                            const int c = i / (nrow * 8);
-                            const int rem = i % (nrow * 8);
-                            const int row = first + rem / 8;
-                            const int piece = rem % 8;
-                            *reinterpret_cast<uint4*>(base + c * kBN * 128 + row * 128 + piece * 16) =
+                            const int c = i / (nrow * PPR);
+                            const int rem = i % (nrow * PPR);
+                            const int row = first + rem / PPR;
+                            const int piece = rem % PPR;
+                            *reinterpret_cast<uint4*>(base + c * kBN * C::SW + row * C::SW + piece * 16) =
                                 make_uint4(0, 0, 0, 0);
                         }
                         fence_proxy_async_smem();

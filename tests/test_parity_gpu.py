@@ -393,13 +393,14 @@ def test_config_fp8_dense_causal_full():
                     assert np.max(np.abs(ll[b, :, i] - ref_l[:, 0])) <= tol_l, (name, b, i)
 
 
+@pytest.mark.parametrize("D", [64, 128])
 @pytest.mark.parametrize("L", [1, 100, 129, 300, 777])
 @pytest.mark.parametrize("causal", [True, False])
 @pytest.mark.parametrize("Hq,Hkv", [(2, 2), (4, 2), (3, 1)])
-def test_dense_fp8_small(L, causal, Hq, Hkv):
+def test_dense_fp8_small(L, causal, Hq, Hkv, D):
     """fp8 e4m3 dense attention over several 128-key tiles with a ragged tail, every
     output element against the oracle fed the dequantised values."""
-    w = W.dense(B=2, L=L, Hq=Hq, Hkv=Hkv, D=128, causal=causal, seed=11 * L + Hq)
+    w = W.dense(B=2, L=L, Hq=Hq, Hkv=Hkv, D=D, causal=causal, seed=11 * L + Hq + D)
     t = w.tensors
     qf, dq = W.quantize_e4m3(t["q"])
     kf, dk = W.quantize_e4m3(t["k"])
@@ -412,7 +413,7 @@ def test_dense_fp8_small(L, causal, Hq, Hkv):
     o_ref, lse_ref = oracle.attn_dense(oracle.dequant_e4m3(qf, dq), oracle.dequant_e4m3(kf, dk),
                                        oracle.dequant_e4m3(vf, dv), scale=w.params["scale"],
                                        causal=causal)
-    _cmp(o, lse, o_ref, lse_ref, TOL_O_FP8, None, "fp8 dense L%d" % L)
+    _cmp(o, lse, o_ref, lse_ref, TOL_O_FP8, None, "fp8 dense D%d L%d" % (D, L))
 
 
 @pytest.mark.parametrize("Hq,Hkv", [(32, 8), (8, 4), (4, 1), (16, 8)])

@@ -128,11 +128,12 @@ def test_prefill_only_qv_patch_mask():
     _cmp(o, lse, o_ref, lse_ref, TOL_O_BF16, TOL_LSE_BF16, "only_qv patch")
 
 
+@pytest.mark.parametrize("D", [64, 128])
 @pytest.mark.parametrize("causal", [True, False])
-def test_prefill_only_qv_fp8(causal):
+def test_prefill_only_qv_fp8(causal, D):
     """e4m3 qv and v with per-tensor descales; the score uses descale_qv * descale_v."""
     lens = [128, 400]
-    Hq, Hkv, D = 4, 2, 128
+    Hq, Hkv = 4, 2
     cu = W.cu_from_lens(lens)
     qv = W.randn_bf16((int(cu[-1]), Hq, D), 11, 1)
     v = W.randn_bf16((int(cu[-1]), Hkv, D), 11, 2)
