@@ -56,8 +56,10 @@ KERNEL_SOURCES = ["attention_paged_kv_gqa_b200/csrc/decode.cuh",
                   "attention_paged_kv_gqa_b200/csrc/ptx.cuh",
                   "attention_paged_kv_gqa_b200/csrc/prefill.cuh"]
 MEASURED_TRAFFIC = {
-    "decode": {"bytes": 578_804_992, "sources": "174caf089ea52021"},
-    "prefill": {"bytes": 2_071_334_656, "sources": "174caf089ea52021"},
+    "decode": {"bytes": 579_341_824, "sources": "0088487c8974d827"},
+    "decode_fp8": {"bytes": 291_313_664, "sources": "0088487c8974d827"},
+    "prefill": {"bytes": 2_005_632_512, "sources": "0088487c8974d827"},
+    "prefill_fp8": {"bytes": 172_875_520, "sources": "0088487c8974d827"},
 }
 
 
@@ -661,6 +663,7 @@ def run_fp8(c):
                      "kv len ~ U[1,8192]")
     e["bytes_per_step"] = nb
     e["keys_per_us"] = round(int(t["seqused_k"].sum()) / (dms * 1e3), 1)
+    e["traffic"] = measured_traffic("decode_fp8")
     c["line"]["decode_fp8"] = e
     c["launches"] += 2 * args.steps
     c["line"]["gpu_launches"] = c["launches"]
