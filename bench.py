@@ -208,11 +208,16 @@ class Clocks:
         fd, self.path = tempfile.mkstemp(suffix=".csv")
         os.close(fd)
         try:
+            # One query first, then the sampling loop with time to settle: the sampler's
+            # start-up (NVML initialisation) once stalled a timed step to twice its time.
+            subprocess.run(["nvidia-smi", "-i", str(self.dev), "--query-gpu=clocks.sm",
+                            "--format=csv,noheader"], stdout=subprocess.DEVNULL,
+                           stderr=subprocess.DEVNULL, timeout=30)
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.dev), "--query-gpu=" + self.FIELDS,
                  "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
-            time.sleep(0.3)
+            time.sleep(1.0)
         except Exception:
             self.proc = None
         return self
@@ -558,7 +563,11 @@ def run_decode(c):
                    "parallelism": "replicas" if world > 1 else "single",
                    "l2": "flushed between timed steps (read sweep of 512 MiB); 574 MB of K/V "
                          "per step, larger than L2",
-                   "bytes_per_step": nbytes},
+                   "bytes_per_step": nbytes,
+                   "step_us": {"mean": round(ms * 1e3, 2),
+                               "median": round(statistics.median(times) * 1e3, 2),
+                               "min": round(min(times) * 1e3, 2),
+                               "max": round(max(times) * 1e3, 2)}},
         "roofline": roofline(kernel_gbs, "GB/s", "hbm", peaks, c["peak_kind"],
                              measured_traffic("decode"),
                              "decode_pages_kernel<128> + decode_pages_combine_kernel<128>"),
