@@ -417,7 +417,10 @@ attn_status_t attn_bwd_varlen(
  *   call before any stream capture.  The address is kept for the life of the
  *   process, so this entry point must not be used on a device after
  *   cudaDeviceReset (or any other teardown of its primary context).
- *   Errors: bad arguments get the same status as from attn_decode_paged.
+ *   dtype: ATTN_BF16; ATTN_FP8_E4M3 returns ATTN_ERR_UNSUPPORTED (this call
+ *   takes no descales).
+ *   Errors: bad arguments get the same status as from attn_decode_paged
+ *   (for bf16).
  *   Sharing: every call on a device uses the same scratch and leaves its
  *   contents behind (nothing in it needs to start zeroed).  Calls whose
  *   kernels could overlap on the GPU (different streams without ordering)
