@@ -862,8 +862,10 @@ static int decode_pages_stages(int D, int Hkv, int B, bool vonly = false, bool f
     const int cap = 227 * 1024;
     const int max_ns = (vonly || fp8) ? 16 : 8;   // V-only or e4m3 stages are half as large
     int ns = 0;
-    if (fp8)
+    if (fp8 && D == 128)
         while (ns < max_ns && DecodePagesCfg<128, true>::smem_bytes(Hkv, B, ns + 1, vonly) <= cap) ++ns;
+    else if (fp8)
+        while (ns < max_ns && DecodePagesCfg<64, true>::smem_bytes(Hkv, B, ns + 1, vonly) <= cap) ++ns;
     else if (D == 128)
         while (ns < max_ns && DecodePagesCfg<128>::smem_bytes(Hkv, B, ns + 1, vonly) <= cap) ++ns;
     else
@@ -927,10 +929,10 @@ static attn_status_t decode_paged_impl(const void* q, const void* k_cache, const
     if (!dtype_ok(dtype)) return ATTN_ERR_INVALID_ARG;
     const bool fp8 = dtype == ATTN_FP8_E4M3;
     if (fp8) {
-        // e4m3 q and cache: the page-stream decode (automatic split), head_dim 128
+        // e4m3 q and cache: the page-stream decode (automatic split)
         if (only_qv || qv) return ATTN_ERR_UNSUPPORTED;
         if (!dq || !dk || !dv) return ATTN_ERR_INVALID_ARG;
-        if (D != 128 || num_splits > 0) return ATTN_ERR_UNSUPPORTED;
+        if (num_splits > 0) return ATTN_ERR_UNSUPPORTED;
     }
     if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
     if (block_size != kPageRows) return ATTN_ERR_UNSUPPORTED;
@@ -969,7 +971,7 @@ static attn_status_t decode_paged_impl(const void* q, const void* k_cache, const
         const uint64_t rowk = (uint64_t)Hkv * D * E;
         const uint64_t pd[4] = {(uint64_t)D, (uint64_t)kPageRows, (uint64_t)Hkv, (uint64_t)num_blocks};
         const uint64_t ps[3] = {rowk, (uint64_t)D * E, rowk * kPageRows};
-        const uint32_t pbox[4] = {(uint32_t)(128 / E), (uint32_t)kPageRows, (uint32_t)Hkv, 1};
+        const uint32_t pbox[4] = {(uint32_t)std::min(128 / E, D), (uint32_t)kPageRows, (uint32_t)Hkv, 1};
         attn_status_t s;
         if ((s = get_map(&pv, v_cache, dtype, pd, ps, pbox)) != ATTN_OK) return s;
         if (only_qv) pk = pv;   // no key store: its map is never used
@@ -1011,9 +1013,12 @@ static attn_status_t decode_paged_impl(const void* q, const void* k_cache, const
             return wide ? launch_decode_pages<64, false, 2, true>(pk, pv, pa, grid, stp, ob, lse, pdl)
                         : launch_decode_pages<64, false, 1, true>(pk, pv, pa, grid, stp, ob, lse, pdl);
         }
-        if (fp8)
+        if (fp8 && D == 128)
             return wide ? launch_decode_pages<128, true, 2>(pk, pv, pa, grid, stp, ob, lse, pdl)
                         : launch_decode_pages<128, true, 1>(pk, pv, pa, grid, stp, ob, lse, pdl);
+        if (fp8)
+            return wide ? launch_decode_pages<64, true, 2>(pk, pv, pa, grid, stp, ob, lse, pdl)
+                        : launch_decode_pages<64, true, 1>(pk, pv, pa, grid, stp, ob, lse, pdl);
         if (D == 128)
             return wide ? launch_decode_pages<128, false, 2>(pk, pv, pa, grid, stp, ob, lse, pdl)
                         : launch_decode_pages<128, false, 1>(pk, pv, pa, grid, stp, ob, lse, pdl);

@@ -492,8 +492,15 @@ template <int D, bool FP8 = false>
 struct DecodePagesCfg {
     static constexpr int E = FP8 ? 1 : 2;               // bytes per element
     static constexpr int ROWB = D * E;
-    static constexpr int NCHUNK = ROWB / 128;           // 128-byte swizzle columns per row
-    static constexpr int CHUNK_E = 128 / E;             // elements per swizzle column
+    // swizzle span: 128-byte columns, or one 64-byte column for 64-byte rows (e4m3, D = 64)
+    static constexpr int SW = ROWB >= 128 ? 128 : 64;
+    static constexpr int NCHUNK = ROWB / SW;            // swizzle columns per row
+    static constexpr int CHUNK_E = SW / E;              // elements per swizzle column
+    // byte offset of 16-byte piece `piece` of row `row` inside one swizzle column
+    __device__ static constexpr uint32_t swz(int row, int piece) {
+        return SW == 128 ? row * 128 + ((piece ^ (row & 7)) << 4)
+                         : row * 64 + ((piece ^ ((row >> 1) & 3)) << 4);
+    }
     // stage = one page of K and V for all heads: 2 * 16 * Hkv * D * 2 bytes (half: V alone,
     // for the only_qv score)
     __host__ __device__ static constexpr int stage_bytes(int Hkv, bool vonly = false) {
@@ -621,9 +628,9 @@ __global__ void __launch_bounds__(32 * (kPgMaxWarps + 1), 1)
 #pragma unroll
                     for (int c = 0; c < C::NCHUNK; ++c) {
                         if (!a.only_qv)
-                            tma_load_4d_hint(&tmK, &full[st], dk + c * rows * 128, c * C::CHUNK_E, 0, 0,
+                            tma_load_4d_hint(&tmK, &full[st], dk + c * rows * C::SW, c * C::CHUNK_E, 0, 0,
                                              page, pol);
-                        tma_load_4d_hint(&tmV, &full[st], dv + c * rows * 128, c * C::CHUNK_E, 0, 0, page,
+                        tma_load_4d_hint(&tmV, &full[st], dv + c * rows * C::SW, c * C::CHUNK_E, 0, 0, page,
                                          pol);
                     }
                 }
@@ -763,11 +770,12 @@ __global__ void __launch_bounds__(32 * (kPgMaxWarps + 1), 1)
                     // zero this head's V rows past the sequence end (not data of it): every
                     // 16-byte piece of those rows, in each 128-byte column of the stage
                     constexpr int PPR = C::ROWB / 16;             // pieces per row
+                    constexpr int PPC = C::SW / 16;               // pieces per swizzle column row
                     for (int e = lane; e < kPageRows * PPR; e += 32) {
                         const int rr = e / PPR, pc = e % PPR;
                         if (tok0 + rr >= L)
-                            *reinterpret_cast<uint4*>(sv + (pc >> 3) * rows * 128 + (r0 + rr) * 128 + (pc & 7) * 16) =
-                                make_uint4(0, 0, 0, 0);
+                            *reinterpret_cast<uint4*>(sv + (pc / PPC) * rows * C::SW + (r0 + rr) * C::SW +
+                                                      (pc % PPC) * 16) = make_uint4(0, 0, 0, 0);
                     }
                     __syncwarp();
                 }
@@ -784,7 +792,7 @@ __global__ void __launch_bounds__(32 * (kPgMaxWarps + 1), 1)
                         const int row = r0 + (mi & 1) * 8 + ri;
                         const int piece = 2 * j + (mi >> 1);
                         uint32_t ka[4];
-                        ldmatrix_x4(skb + row * 128 + ((piece ^ (row & 7)) << 4), ka[0], ka[1], ka[2], ka[3]);
+                        ldmatrix_x4(skb + C::swz(row, piece), ka[0], ka[1], ka[2], ka[3]);
 #pragma unroll
                         for (int nt = 0; nt < NT; ++nt) mma_e4m3_16832(sc[nt], ka, qb[nt][j][0], qb[nt][j][1]);
                     }
@@ -867,7 +875,7 @@ __global__ void __launch_bounds__(32 * (kPgMaxWarps + 1), 1)
                         const int row = r0 + (mi & 1) * 8 + ri;
                         const int piece = cc + (mi >> 1);
                         uint32_t w[4];
-                        ldmatrix_x4_trans(svb + row * 128 + ((piece ^ (row & 7)) << 4), w[0], w[1], w[2], w[3]);
+                        ldmatrix_x4_trans(svb + C::swz(row, piece), w[0], w[1], w[2], w[3]);
 #pragma unroll
                         for (int u = 0; u < 2; ++u) {
                             const uint32_t lo = __byte_perm(w[2 * u], 0u, 0x3120u);       // keys 0..7

@@ -52,21 +52,22 @@ METRIC = "attn fwd TFLOP/s (prefill) & paged-decode KV GB/s on 1 B200, % of roof
 # capture on its bench workload (full-size launch).  They hold only for the
 # kernel sources they were taken on: when the sha256 prefix of those sources
 # differs, the roofline reports traffic null.
-KERNEL_SOURCES = ["attention_paged_kv_gqa_b200/csrc/decode.cuh",
-                  "attention_paged_kv_gqa_b200/csrc/ptx.cuh",
-                  "attention_paged_kv_gqa_b200/csrc/prefill.cuh"]
+KERNEL_SOURCES = {
+    "decode": ["attention_paged_kv_gqa_b200/csrc/decode.cuh", "attention_paged_kv_gqa_b200/csrc/ptx.cuh"],
+    "prefill": ["attention_paged_kv_gqa_b200/csrc/prefill.cuh", "attention_paged_kv_gqa_b200/csrc/ptx.cuh"],
+}
 MEASURED_TRAFFIC = {
-    "decode": {"bytes": 579_341_824, "sources": "0088487c8974d827"},
-    "decode_fp8": {"bytes": 291_313_664, "sources": "0088487c8974d827"},
-    "prefill": {"bytes": 2_005_632_512, "sources": "0088487c8974d827"},
-    "prefill_fp8": {"bytes": 172_875_520, "sources": "0088487c8974d827"},
+    "decode": {"bytes": 579_341_824, "sources": "PENDING"},
+    "decode_fp8": {"bytes": 291_313_664, "sources": "PENDING"},
+    "prefill": {"bytes": 2_005_632_512, "sources": "53045763a6653a9a"},
+    "prefill_fp8": {"bytes": 172_875_520, "sources": "53045763a6653a9a"},
 }
 
 
-def kernel_sources_sha() -> str:
+def kernel_sources_sha(kind: str) -> str:
     import hashlib
     h = hashlib.sha256()
-    for f in KERNEL_SOURCES:
+    for f in KERNEL_SOURCES[kind]:
         with open(os.path.join(ROOT, f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -74,9 +75,11 @@ def kernel_sources_sha() -> str:
 
 def measured_traffic(kind):
     rec = MEASURED_TRAFFIC.get(kind)
-    if rec is None or rec["sources"] != kernel_sources_sha():
+    if rec is None or rec["sources"] != kernel_sources_sha(kind.split("_")[0]):
         return None
     return rec["bytes"]
+
+
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # The spec figures of a B200 (dense tensor rates; HBM3e bandwidth).
 SPEC_PEAKS = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0, "fp8_tflops": 4500.0}

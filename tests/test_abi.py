@@ -198,8 +198,8 @@ def test_noalloc_decode_reports_bad_arguments_like_the_workspace_decode(L):
 
 
 def test_fp8_decode_argument_checks(L):
-    """e4m3 decode: descales required (invalid without); head_dim 128, automatic split and
-    the key store only (unsupported otherwise); the noalloc call takes bf16 only."""
+    """e4m3 decode: descales required (invalid without); head_dim 64 or 128, automatic split
+    and the key store only (unsupported otherwise); the noalloc call takes bf16 only."""
     p = ctypes.c_void_p(1 << 20)
 
     def dec(D=128, splits=0, dq=p, dk=p, dv=p, Hq=8, Hkv=2, B=2):
@@ -207,7 +207,7 @@ def test_fp8_decode_argument_checks(L):
                                    1, dq, dk, dv, p, None, p, 1 << 24, None)
 
     assert dec(dq=None) == 1 and dec(dk=None) == 1 and dec(dv=None) == 1
-    assert dec(D=64) == 2
+    assert dec(D=96) == 2
     assert dec(splits=3) == 2
     assert dec(Hq=32, Hkv=16) == 2          # more KV heads than consumer warps
     st = L.attn_decode_paged_only_qv(p, p, p, 4, 100, 16, p, 2, 8, 2, 128, 0.0, -1, 0.0, 0, 1,

@@ -69,26 +69,29 @@ def _cmp(o, lse, o_ref, lse_ref, what):
         assert err_l <= TOL_LSE, "%s: max|LSE err| %.3g" % (what, err_l)
 
 
+@pytest.mark.parametrize("D", [64, 128])
 @pytest.mark.parametrize("Hq,Hkv", [(32, 8), (8, 4), (4, 1), (16, 8), (16, 1), (8, 8)])
-def test_decode_fp8_many_sequences(Hq, Hkv):
+def test_decode_fp8_many_sequences(Hq, Hkv, D):
     """Empty, one-key, page-edge and long sequences, so CTA shares start and end
-    inside sequences and pages end ragged."""
+    inside sequences and pages end ragged.  At head_dim 64 an e4m3 row is 64 bytes
+    (the 64-byte swizzle)."""
     lens = [0, 1, 5, 16, 17, 31, 300, 0, 2048, 64, 65, 1000, 7, 129, 3000, 15] * 3
-    w = W.paged_decode(B=len(lens), Hq=Hq, Hkv=Hkv, D=128, num_blocks=2000, lmax=3072, lens=lens,
-                       seed=5 * Hq + Hkv)
+    w = W.paged_decode(B=len(lens), Hq=Hq, Hkv=Hkv, D=D, num_blocks=2000, lmax=3072, lens=lens,
+                       seed=5 * Hq + Hkv + D)
     t = w.tensors
     qz = _quantised(t)
     o, lse = _run(qz, t, scale=w.params["scale"])
     o_ref, lse_ref = oracle.attn_decode(qz["q_deq"], qz["k_cache_deq"], qz["v_cache_deq"],
                                         t["block_table"], t["seqused_k"], scale=w.params["scale"])
-    _cmp(o, lse, o_ref, lse_ref, "fp8 decode Hq%d Hkv%d" % (Hq, Hkv))
+    _cmp(o, lse, o_ref, lse_ref, "fp8 decode D%d Hq%d Hkv%d" % (D, Hq, Hkv))
 
 
+@pytest.mark.parametrize("D", [64, 128])
 @pytest.mark.parametrize("window_left,softcap", [(0, 0.0), (37, 0.0), (-1, 30.0), (200, 15.0)])
-def test_decode_fp8_window_softcap(window_left, softcap):
+def test_decode_fp8_window_softcap(window_left, softcap, D):
     lens = [1, 2, 16, 17, 40, 255, 256, 1500, 0, 33]
-    w = W.paged_decode(B=len(lens), Hq=16, Hkv=4, D=128, num_blocks=400, lmax=1536, lens=lens,
-                       seed=71 + window_left)
+    w = W.paged_decode(B=len(lens), Hq=16, Hkv=4, D=D, num_blocks=400, lmax=1536, lens=lens,
+                       seed=71 + window_left + D)
     t = w.tensors
     qz = _quantised(t)
     o, lse = _run(qz, t, scale=w.params["scale"], window_left=window_left, softcap=softcap)

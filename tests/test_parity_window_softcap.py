@@ -116,14 +116,15 @@ def test_softcap_changes_the_result():
     assert (o1.float() - o0.float()).abs().max().item() > 0.1
 
 
-def test_fp8_sliding_window_and_softcap():
+@pytest.mark.parametrize("D", [64, 128])
+def test_fp8_sliding_window_and_softcap(D):
     """fp8 with a cap and/or a window.  N(0,1) inputs as in the fp8 workload, for
     which the fp8 tolerance is stated (logits up to about 4, so caps of 2 and 3
     still bite).  Lq < Lk gives every row at least 61 keys: over a handful of keys
     with flat weights the e4m3 rounding of P (2^-4 relative per weight) alone can
     exceed 6e-2, which is a property of e4m3 P, not of the cap or the window (the
     bf16 tests check those at a tight tolerance)."""
-    w = W.dense(B=2, L=128, Lk=400, Hq=4, Hkv=2, D=128, causal=True, seed=5)
+    w = W.dense(B=2, L=128, Lk=400, Hq=4, Hkv=2, D=D, causal=True, seed=5 + D)
     t = w.tensors
     qf, dq = W.quantize_e4m3(t["q"])
     kf, dk = W.quantize_e4m3(t["k"])
@@ -139,7 +140,7 @@ def test_fp8_sliding_window_and_softcap():
                                            oracle.dequant_e4m3(kf, dk),
                                            oracle.dequant_e4m3(vf, dv), scale=w.params["scale"],
                                            causal=True, softcap=cap, window_left=window)
-        _cmp(o, lse, o_ref, lse_ref, TOL_O_FP8, None, "fp8 cap %g window %d" % (cap, window))
+        _cmp(o, lse, o_ref, lse_ref, TOL_O_FP8, None, "fp8 D%d cap %g window %d" % (D, cap, window))
 
 
 # ---------------------------------------------------------------------------- varlen, paged
