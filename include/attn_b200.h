@@ -264,7 +264,7 @@ size_t attn_decode_workspace_size(int B, int num_heads_q, int num_heads_kv, int 
  *   num_splits   key-range splits per sequence; <= 0 chooses automatically.
  *   dtype        ATTN_BF16, or ATTN_FP8_E4M3 for an e4m3 q and cache with
  *                descale_q/k/v (device fp32 scalars, all three required):
- *                head_dim 128, num_splits <= 0, at most 8 KV heads.
+ *                num_splits <= 0, at most 8 KV heads.
  *   o            [B, Hq, D] bf16.   lse [B, Hq] fp32 or NULL.
  *   workspace    >= attn_decode_workspace_size(...) bytes of device memory,
  *                16-byte aligned; its contents on entry do not matter.
