@@ -272,7 +272,8 @@ def flush_l2(flush):
 def time_steps(step_fn, steps, warmup, world, flush):
     """Per-step device times (ms) with CUDA events on the current stream, L2 flushed between steps."""
     stream = torch.cuda.current_stream()
-    for _ in range(warmup):
+    for _ in range(warmup):            # the warm-up steps are the timed steps' sequence, untimed
+        flush_l2(flush)
         step_fn()
     barrier(world)
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
