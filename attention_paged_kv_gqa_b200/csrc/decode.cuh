@@ -1,8 +1,11 @@
 // decode.cuh -- paged GQA decode on sm_100a: one query token per sequence,
 // key range split across CTAs (split-KV), then an LSE-weighted combine.
 //
-// The work is HBM-bound (about 4 flop per byte of K/V at group size 4), so the
-// kernel is built around the memory path: a producer warp fetches each 16-token
+// Two kernels, both HBM-bound (about 4 flop per byte of K/V at group size 4)
+// and built around the memory path.  The page-stream kernel further below is
+// the default (automatic split); the per-head split kernel here serves an
+// explicit split count and the shapes the page stream does not take.  In the
+// split kernel a producer warp fetches each 16-token
 // page of K and V straight from the paged cache through block_table with TMA
 // (128-byte swizzle, no gather pass), several stages deep; four consumer warps
 // each own 16 keys of a 64-key stage and keep their own online-softmax state,
