@@ -57,8 +57,8 @@ KERNEL_SOURCES = {
     "prefill": ["attention_paged_kv_gqa_b200/csrc/prefill.cuh", "attention_paged_kv_gqa_b200/csrc/ptx.cuh"],
 }
 MEASURED_TRAFFIC = {
-    "decode": {"bytes": 579_056_128, "sources": "fe600f513bd77e6c"},
-    "decode_fp8": {"bytes": 294_267_904, "sources": "fe600f513bd77e6c"},
+    "decode": {"bytes": 579_056_128, "sources": "e1e056b670478940"},
+    "decode_fp8": {"bytes": 294_267_904, "sources": "e1e056b670478940"},
     "prefill": {"bytes": 2_005_632_512, "sources": "53045763a6653a9a"},
     "prefill_fp8": {"bytes": 172_875_520, "sources": "53045763a6653a9a"},
 }
