@@ -151,8 +151,11 @@ attn_status_t get_map(CUtensorMap* out, const void* ptr, int dtype, const uint64
     CUtensorMap m;
     const cuuint32_t estride[4] = {1, 1, 1, 1};
     // the swizzle span is the box's row: 128 bytes, or 64 (e4m3 rows of head_dim 64)
+    // (rows wider than 128 bytes: no swizzle, for row-by-row reads of whole rows)
     const uint32_t row_bytes = box[0] * (dtype == ATTN_FP8_E4M3 ? 1u : 2u);
-    const CUtensorMapSwizzle swz = row_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
+    const CUtensorMapSwizzle swz = row_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                   : row_bytes <= 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                                      : CU_TENSOR_MAP_SWIZZLE_NONE;
     const CUresult r = enc(&m,
                            dtype == ATTN_FP8_E4M3 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
                                                   : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
@@ -481,6 +484,22 @@ attn_status_t launch_backward(const CUtensorMap& mq, const CUtensorMap& mdo, con
 }  // namespace
 
 // ==================================================================== C ABI
+template <int D>
+static attn_status_t launch_patch_stream(const PatchMaps& maps, const PatchArgs& pa, int n_hg, int n_rg,
+                                         cudaStream_t st) {
+    static std::atomic<uint64_t> attr_mask{0};   // one bit per device
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const uint64_t bit = 1ull << (dev & 63);
+    if (!(attr_mask.load() & bit)) {
+        const attn_status_t s = set_smem(patch_stream_kernel<D>, patch_stream_smem_bytes());
+        if (s != ATTN_OK) return s;
+        attr_mask.fetch_or(bit);
+    }
+    patch_stream_kernel<D><<<(unsigned)(n_hg * n_rg), kPsThreads, patch_stream_smem_bytes(), st>>>(maps, pa, n_hg);
+    return launch_status();
+}
+
 extern "C" {
 
 const char* attn_status_string(attn_status_t s) {
@@ -809,10 +828,34 @@ attn_status_t attn_fwd_patch(const void* q, const void* k, const void* v,
     pa.Hkv = Hkv;
     pa.group = Hq / Hkv;
     pa.total_q = total_q;
+    pa.total_k = total_k;
     pa.scale = resolve_scale(softmax_scale, D);
     pa.o = static_cast<__nv_bfloat16*>(o);
     pa.lse = lse;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // no grouped heads: heads in 512-byte slices, each query's rows streamed through
+    // shared memory by bulk copies
+    if (Hq == Hkv && Hq % (256 / D) == 0) {
+        const int n_hg = Hq / (256 / D);
+        const int n_rg = std::max(1, sm_count(dev) / n_hg);
+        PatchMaps maps;
+        const uint64_t C = (uint64_t)Hq * D;          // elements of a row (Hq == Hkv)
+        const uint64_t dq4[4] = {C, (uint64_t)total_q, 1, 1};
+        const uint64_t sq3[3] = {C * 2, C * 2 * (uint64_t)total_q, C * 2 * (uint64_t)total_q};
+        const uint32_t bq4[4] = {256, (uint32_t)kPsQ, 1, 1};
+        attn_status_t s;
+        if ((s = get_map(&maps.q, q, ATTN_BF16, dq4, sq3, bq4)) != ATTN_OK) return s;
+        const uint64_t nk = (uint64_t)std::max(total_k, 1);
+        const uint64_t dk4[4] = {C, nk, 1, 1};
+        const uint64_t sk3[3] = {C * 2, C * 2 * nk, C * 2 * nk};
+        for (int pc = 0; pc < 4; ++pc) {
+            const uint32_t bk4[4] = {256, (uint32_t)(8 << pc), 1, 1};
+            if ((s = get_map(&maps.k[pc], k, ATTN_BF16, dk4, sk3, bk4)) != ATTN_OK) return s;
+            if ((s = get_map(&maps.v[pc], v, ATTN_BF16, dk4, sk3, bk4)) != ATTN_OK) return s;
+        }
+        return D == 128 ? launch_patch_stream<128>(maps, pa, n_hg, n_rg, st)
+                        : launch_patch_stream<64>(maps, pa, n_hg, n_rg, st);
+    }
     // a warp per query (all heads) where a lane's share of the heads' columns is small;
     // otherwise a warp per (query, head)
     const long long qblocks = std::min<long long>((total_q + kPatchWarps - 1) / kPatchWarps,

@@ -191,10 +191,12 @@ attn_status_t attn_fwd_varlen_paged(
  *   q [total_q, Hq, D], k/v packed [total_k, Hkv, D], cu_seqlens_q/k int32 [B+1],
  *   patch_kv_range int32 [total_q, 2], o [total_q, Hq, D] bf16, lse [Hq, total_q] or NULL.
  *   max_interval  the caller's bound on end - start over all queries.  It only
- *                 chooses the kernel, never the result: up to 64 (bf16) a CUDA-core
- *                 kernel reads each key and value row once per query head (one
- *                 warp per query and head); above that, or for fp8, the tiled
- *                 tensor-core kernel of attn_fwd_varlen_paged runs.
+ *                 chooses the kernel, never the result: up to 64 (bf16) CUDA-core
+ *                 kernels read each key and value row once per query (with
+ *                 Hq == Hkv the rows of consecutive queries stream through
+ *                 shared memory; with grouped heads one warp takes a query);
+ *                 above that, or for fp8, the tiled tensor-core kernel of
+ *                 attn_fwd_varlen_paged runs.
  * Supported: head_dim in {64, 128}.
  */
 attn_status_t attn_fwd_patch(

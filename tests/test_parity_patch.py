@@ -118,3 +118,28 @@ def test_patch_short_intervals_ragged(D, Hq, Hkv):
     o, lse, o_ref, lse_ref = _run(q, k, v, cq, ck, ranges, Hkv, 16, 0.15, max(lens_q))
     _cmp(o, lse, o_ref, lse_ref, "patch short D%d Hq%d Hkv%d" % (D, Hq, Hkv))
 
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_patch_equal_heads_long_intervals_and_many_sequences(D):
+    """Hq == Hkv (the streaming kernel): intervals longer than the caller's max_interval
+    (it chooses the kernel, never the result), overlapping and out-of-order intervals, and
+    more sequences than fit the kernel's shared-memory sequence table."""
+    rng = np.random.default_rng(300 + D)
+    B = 300
+    lens_q = rng.integers(0, 6, B)
+    lens_k = rng.integers(0, 200, B)
+    cq, ck = W.cu_from_lens(lens_q), W.cu_from_lens(lens_k)
+    rows = []
+    for b in range(B):
+        for i in range(int(lens_q[b])):
+            s0 = int(rng.integers(-3, int(lens_k[b]) + 3))
+            n = int(rng.choice([0, 1, 5, 16, 40, 64, 65, 150]))
+            rows.append((s0, s0 + n))
+    ranges = torch.tensor(rows, dtype=torch.int32).reshape(-1, 2)
+    Hq = 8
+    q = W.randn_bf16((int(cq[-1]), Hq, D), 6, 1)
+    k = W.randn_bf16((int(ck[-1]), Hq, D), 6, 2)
+    v = W.randn_bf16((int(ck[-1]), Hq, D), 6, 3)
+    o, lse, o_ref, lse_ref = _run(q, k, v, cq, ck, ranges, Hq, 16, 0.15, int(lens_q.max()))
+    _cmp(o, lse, o_ref, lse_ref, "patch long/many D%d" % D)
