@@ -962,7 +962,7 @@ def run_patch_and_small(c):
     nb = patch_bytes(P)
     e = entry(nb / (pms * 1e-3) / 1e9, "GB/s", pms, "hbm", peaks)
     e["workload"] = "B=4 x 8192 bytes, %d patch queries, H=16, D=64" % P["total_q"]
-    e["kernel"] = "patch_query_kernel<64,16> (attn_fwd_patch)"
+    e["kernel"] = "patch_stream_kernel<64> (attn_fwd_patch)"
     e["tiled_kernel"] = entry(nb / (tms * 1e-3) / 1e9, "GB/s", tms, "hbm", peaks)
     out = {"patch": e}
     del d
