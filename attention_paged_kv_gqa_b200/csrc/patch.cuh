@@ -231,7 +231,7 @@ __global__ void __launch_bounds__(32 * kPatchWarps, 2) patch_query_kernel(const 
 // kPsStages stages deep, so the whole CTA
 // keeps tens of KB of reads in flight instead of one dependent row at a time.
 // The consumer warps take a chunk's queries one per warp (LPH = 32 / HG lanes
-// per head, 8 columns a lane, two keys a step) and read only shared memory.
+// per head, 8 columns a lane, up to four keys a step) and read only shared memory.
 // They form kPsTeams teams that take alternate chunks; chunk c uses stage
 // c % kPsStages, so each stage serves one team, which waits for every phase of
 // its barriers in turn (a parity wait cannot tell phases two apart).  One team
@@ -562,9 +562,45 @@ __global__ void __launch_bounds__(kPsThreads, 1)
                     for (int c = 0; c < 8; ++c) acc[c] = fmaf(p1, vf1[c], fmaf(p0, vf0[c], acc[c] * alpha));
                     mrow = mn;
                 };
+                // four keys a step where four remain
+                auto step4 = [&](int r) {
+                    float d[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        float kf[8];
+                        bf16x8_to_f32(*reinterpret_cast<const uint4*>(sK(st) + (r + u) * kPsSlice + lane * 16), kf);
+                        d[u] = 0.0f;
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) d[u] = fmaf(qf[c], kf[c], d[u]);
+                    }
+#pragma unroll
+                    for (int off = 1; off < LPH; off <<= 1)
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) d[u] += __shfl_xor_sync(0xffffffffu, d[u], off);
+                    float sc[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) sc[u] = d[u] * sl2;
+                    const float mn = fmaxf(mrow, fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3])));
+                    const float alpha = (mrow == -INFINITY) ? 0.0f : ex2(mrow - mn);
+                    float pr[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) pr[u] = ex2(sc[u] - mn);
+                    l = l * alpha + ((pr[0] + pr[1]) + (pr[2] + pr[3]));
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) acc[c] *= alpha;
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        float vf[8];
+                        bf16x8_to_f32(*reinterpret_cast<const uint4*>(sV(st) + (r + u) * kPsSlice + lane * 16), vf);
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) acc[c] = fmaf(pr[u], vf[c], acc[c]);
+                    }
+                    mrow = mn;
+                };
                 const int rs = m.rs[t], re = m.re[t];
                 if (rs >= 0) {
                     int r = rs;
+                    for (; r + 3 < re; r += 4) step4(r);
                     for (; r + 1 < re; r += 2)
                         step2(*reinterpret_cast<const uint4*>(sK(st) + r * kPsSlice + lane * 16),
                               *reinterpret_cast<const uint4*>(sV(st) + r * kPsSlice + lane * 16),
