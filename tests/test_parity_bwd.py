@@ -2,7 +2,7 @@
 
 The GPU backward is fed the GPU forward's O (bf16) and LSE (fp32), as a
 training step would be; the oracle recomputes both exactly.  Tolerance,
-derived from the arithmetic (the benchmark spec states none for the backward):
+derived from the arithmetic (no bound is stated for the backward):
 P and dS are rounded to bf16 (relative 2^-9) as tensor-core operands with
 fp32 accumulation, the outputs are bf16, and Delta = dO . O inherits the
 bf16 rounding of O, so per gradient tensor
