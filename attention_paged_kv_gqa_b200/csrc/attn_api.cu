@@ -494,6 +494,10 @@ static attn_status_t launch_patch_stream(const PatchMaps& maps, const PatchArgs&
     if (!(attr_mask.load() & bit)) {
         const attn_status_t s = set_smem(patch_stream_kernel<D>, patch_stream_smem_bytes());
         if (s != ATTN_OK) return s;
+        // kPsCtas CTAs share an SM: ask for the largest shared-memory carveout (a hint)
+        if (cudaFuncSetAttribute(patch_stream_kernel<D>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 (int)cudaSharedmemCarveoutMaxShared) != cudaSuccess)
+            cudaGetLastError();
         attr_mask.fetch_or(bit);
     }
     patch_stream_kernel<D><<<(unsigned)(n_hg * n_rg), kPsThreads, patch_stream_smem_bytes(), st>>>(maps, pa, n_hg);
@@ -837,7 +841,7 @@ attn_status_t attn_fwd_patch(const void* q, const void* k, const void* v,
     // shared memory by bulk copies
     if (Hq == Hkv && Hq % (256 / D) == 0) {
         const int n_hg = Hq / (256 / D);
-        const int n_rg = std::max(1, sm_count(dev) / n_hg);
+        const int n_rg = std::max(1, kPsCtas * sm_count(dev) / n_hg);
         PatchMaps maps;
         const uint64_t C = (uint64_t)Hq * D;          // elements of a row (Hq == Hkv)
         const uint64_t dq4[4] = {C, (uint64_t)total_q, 1, 1};

@@ -234,18 +234,23 @@ __global__ void __launch_bounds__(32 * kPatchWarps, 2) patch_query_kernel(const 
 // per head, 8 columns a lane, up to four keys a step) and read only shared memory.
 // They form kPsTeams teams that take alternate chunks; chunk c uses stage
 // c % kPsStages, so each stage serves one team, which waits for every phase of
-// its barriers in turn (a parity wait cannot tell phases two apart).  One team
-// of 8 warps with 3 stages of 64 rows is kept: two teams with 4 stages of 48
-// rows measured slower (3660 vs 3834 GB/s on the patch workload).  A query whose own
-// interval is longer than kPsRows is marked, and its consumer reads it from
-// global memory, so any interval length is correct.
+// its barriers in turn (a parity wait cannot tell phases two apart).  Two CTAs
+// share an SM, each with one team of 8 warps and 3 stages of 8 queries and 32
+// rows (110 KB): on the patch workload that measured 4352 GB/s against 3930 for
+// one CTA of 3 stages of 16 queries and 64 rows, in one A/B call; three CTAs of 2
+// stages gave 4129, and two teams in one CTA were slower still.  A CTA's time
+// follows its queries more than its bytes (a split of the query list for equal
+// bytes measured 3355 against 4026), so the list is split by count.  A query
+// whose own interval is longer than kPsRows is marked, and its consumer reads it
+// from global memory, so any interval length is correct.
 constexpr int kPsTeamWarps = 8;             // consumer warps of a team
 constexpr int kPsTeams = 1;                 // teams take alternate chunks (two measured slower)
 constexpr int kPsWarps = kPsTeams * kPsTeamWarps;
 constexpr int kPsThreads = 32 * (kPsWarps + 1);
 constexpr int kPsStages = 3;                // a multiple of kPsTeams: a stage serves one team only
-constexpr int kPsQ = 16;                    // queries per chunk
-constexpr int kPsRows = 64;                 // key rows per chunk
+constexpr int kPsQ = 8;                     // queries per chunk
+constexpr int kPsRows = 32;                 // key rows per chunk
+constexpr int kPsCtas = 2;                  // CTAs per SM (the grid is kPsCtas x the SM count)
 constexpr int kPsSlice = 512;               // bytes of one head group's slice of a row
 constexpr int kPsStageBytes = (kPsQ + 2 * kPsRows) * kPsSlice;
 constexpr int kPsCuMax = 255;               // sequences whose cu_seqlens go to shared memory
@@ -278,12 +283,13 @@ __host__ __device__ constexpr int patch_stream_smem_bytes() {
 }
 
 template <int D>
-__global__ void __launch_bounds__(kPsThreads, 1)
+__global__ void __launch_bounds__(kPsThreads, kPsCtas)
     patch_stream_kernel(const __grid_constant__ PatchMaps maps, const PatchArgs a, int n_hg) {
     constexpr int HG = 256 / D;             // heads per 512-byte slice
     constexpr int LPH = 32 / HG;            // lanes per head
     static_assert(HG * D * 2 == kPsSlice && LPH * 8 == D, "slice layout");
     static_assert(kPsStages % kPsTeams == 0, "a stage serves one team");
+    static_assert(kPsQ >= 8 && kPsRows % 8 == 0 && kPsRows <= 120, "groups of 8 queries; boxes of 8 to 64 rows");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
     PatchStreamMeta* meta = reinterpret_cast<PatchStreamMeta*>(smem + kPsStages * kPsStageBytes);
