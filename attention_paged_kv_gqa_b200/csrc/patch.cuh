@@ -281,6 +281,8 @@ __host__ __device__ constexpr int patch_stream_smem_bytes() {
     return 128 + kPsStages * kPsStageBytes + kPsStages * (int)sizeof(PatchStreamMeta) + 2 * kPsStages * 8 +
            2 * (kPsCuMax + 1) * 4;
 }
+// kPsCtas CTAs fit the SM's 228 KB of shared memory, 1 KB of it reserved per CTA
+static_assert(kPsCtas * (patch_stream_smem_bytes() + 1024) <= 228 * 1024, "CTAs per SM");
 
 template <int D>
 __global__ void __launch_bounds__(kPsThreads, kPsCtas)
