@@ -209,8 +209,7 @@ attn_status_t launch_maybe_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, 
         kernel<<<grid, block, smem, st>>>(args...);
         return launch_status();
     }
-    cudaLaunchConfig_t cfg;
-    std::memset(&cfg, 0, sizeof(cfg));
+    cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = block;
     cfg.dynamicSmemBytes = smem;
@@ -347,8 +346,7 @@ attn_status_t launch_decode(const CUtensorMap& mk, const CUtensorMap& mv, Decode
     // The combine kernel is launched as a programmatic dependent of the split
     // kernel: it is scheduled while the split grid runs and waits on the grid
     // dependency before reading the partials.
-    cudaLaunchConfig_t cfg;
-    std::memset(&cfg, 0, sizeof(cfg));
+    cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(a.B * a.Hq);
     cfg.blockDim = dim3(D);
     cfg.dynamicSmemBytes = 0;
@@ -426,8 +424,7 @@ attn_status_t launch_decode_pages(const CUtensorMap& mk, const CUtensorMap& mv, 
     attn_status_t s = launch_maybe_pdl(decode_pages_kernel<D, FP8, NT, HQ>, dim3(grid), dim3(32 * (a.Hkv + 1)),
                                        smem, st, pdl, mk, mv, a);
     if (s != ATTN_OK) return s;
-    cudaLaunchConfig_t cfg;
-    std::memset(&cfg, 0, sizeof(cfg));
+    cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(a.B * a.Hq);
     cfg.blockDim = dim3(D);
     cfg.stream = st;

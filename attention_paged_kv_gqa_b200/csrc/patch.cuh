@@ -344,7 +344,7 @@ __global__ void __launch_bounds__(kPsThreads, kPsCtas)
         // ---------------------------------------------------------------- producer
         int st = 0, issued = 0;
         uint32_t ph = 0;
-        bool ok = true, done_pushed = false;
+        bool ok = true;
         // The next batch's intervals are loaded while this batch's chunks are issued.
         int2 rng_next = make_int2(0, 0);
         if (q_begin + lane < q_end)
