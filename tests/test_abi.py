@@ -247,3 +247,80 @@ def test_fwd_qv_argument_checks(L):
     assert fwd(qv=None) == 1
     assert fwd(D=96) == 2
     assert fwd(dtype=1) == 2
+
+
+def test_kv_append_argument_checks(L):
+    """attn_kv_append_paged rejects bad calls on the host, before the device is touched."""
+    p = ctypes.c_void_p(1 << 20)
+    su_in, su_out = ctypes.c_void_p(1 << 21), ctypes.c_void_p(1 << 22)
+    odd = ctypes.c_void_p((1 << 20) + 8)
+    # (k_new, v_new, k_cache, v_cache, block_table, max_blocks, num_blocks, block_size,
+    #  cu_seqlens_new, seqused_k, seqused_k_out, B, total_new, Hkv, D, dtype)
+    good = [p, p, p, p, p, 4, 100, 16, None, su_in, su_out, 2, 2, 2, 128, 0]
+    cases = {
+        "null k_new": ({0: None}, 1), "null v_cache": ({3: None}, 1),
+        "null block_table": ({4: None}, 1), "null seqused_k": ({9: None}, 1),
+        "negative B": ({11: -1}, 1), "Hkv 0": ({13: 0}, 1), "max_blocks 0": ({5: 0}, 1),
+        "num_blocks 0": ({6: 0}, 1), "dtype 7": ({15: 7}, 1),
+        "one per sequence needs total_new == B": ({12: 3}, 1),
+        "seqused_k_out aliases seqused_k": ({10: su_in}, 1),
+        "block_size 32": ({7: 32}, 2),
+        "row not a multiple of 16 bytes": ({14: 4}, 1),
+        "misaligned k_new": ({0: odd}, 1), "misaligned k_cache": ({2: odd}, 1),
+    }
+    for name, (change, want) in cases.items():
+        a = list(good)
+        for i, val in change.items():
+            a[i] = val
+        assert L.attn_kv_append_paged(*a, None) == want, name
+
+
+def test_decode_append_checks_the_decode_half_first(L):
+    """attn_decode_paged_append validates the decode's arguments before the append could
+    be launched, so a bad call leaves the cache untouched."""
+    p = ctypes.c_void_p(1 << 20)
+    su_in, su_out = ctypes.c_void_p(1 << 21), ctypes.c_void_p(1 << 22)
+    odd = ctypes.c_void_p((1 << 20) + 8)
+    # (q, k_new, v_new, k_cache, v_cache, block_table, max_blocks, num_blocks, block_size,
+    #  seqused_k, seqused_k_out, B, Hq, Hkv, D, scale, window_left, softcap, num_splits, dtype,
+    #  o, lse, workspace, workspace_bytes)
+    good = [p, p, p, p, p, p, 4, 100, 16, su_in, su_out, 2, 8, 2, 128, 0.0, -1, 0.0, 0, 0,
+            p, None, p, 1 << 24]
+    cases = {
+        "no seqused_k_out": ({10: None}, 1), "null q": ({0: None}, 1), "null o": ({20: None}, 1),
+        "Hq not a multiple": ({12: 6, 13: 4}, 1), "dtype 7": ({19: 7}, 1),
+        "fp8": ({19: 1}, 2), "head_dim 96": ({14: 96}, 2), "group 32": ({12: 32, 13: 1}, 2),
+        "misaligned q": ({0: odd}, 1), "misaligned o": ({20: odd}, 1),
+        "no workspace": ({22: None}, 1), "workspace too small": ({23: 16}, 5),
+        "null k_new (the append half)": ({1: None}, 1),
+    }
+    for name, (change, want) in cases.items():
+        a = list(good)
+        for i, val in change.items():
+            a[i] = val
+        assert L.attn_decode_paged_append(*a, None) == want, name
+
+
+def test_backward_argument_checks(L):
+    p = ctypes.c_void_p(1 << 20)
+    cu = ctypes.c_void_p(1 << 21)
+    odd = ctypes.c_void_p((1 << 20) + 8)
+    assert L.attn_bwd_workspace_size(4, 10) >= 4 * 10 * 4
+    assert L.attn_bwd_workspace_size(0, 10) == 0
+    assert L.attn_bwd_workspace_size(4, -1) == 0
+    # (q, k, v, o, dout, lse, dq, dk, dv, cu_q, cu_k, B, total_q, total_k, max_q, max_k,
+    #  Hq, Hkv, D, scale, mask, window_left, workspace, workspace_bytes)
+    good = [p, p, p, p, p, p, p, p, p, cu, cu, 1, 64, 64, 64, 64, 4, 2, 128, 0.0, 1, -1, p, 1 << 20]
+    cases = {
+        "null dout": ({4: None}, 1), "null lse": ({5: None}, 1), "null dv": ({8: None}, 1),
+        "null cu_seqlens_k": ({10: None}, 1), "negative total_k": ({13: -1}, 1),
+        "Hq not a multiple": ({16: 3}, 1), "mask 9": ({20: 9}, 1), "patch mask": ({20: 2}, 2),
+        "window without causal": ({20: 0, 21: 8}, 2), "head_dim 96": ({18: 96}, 2),
+        "misaligned dq": ({6: odd}, 1), "misaligned v": ({2: odd}, 1),
+        "no workspace": ({22: None}, 1), "workspace too small": ({23: 64}, 5),
+    }
+    for name, (change, want) in cases.items():
+        a = list(good)
+        for i, val in change.items():
+            a[i] = val
+        assert L.attn_bwd_varlen(*a, None) == want, name
