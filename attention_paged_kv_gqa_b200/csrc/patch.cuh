@@ -268,7 +268,7 @@ struct PatchStreamMeta {
 
 // Tensor maps of the streamed slices: q as [total_q rows][Hq * D], k and v as
 // [total_k rows][Hkv * D], boxes of 256 elements (one head group's 512-byte
-// slice) by 16 rows (q) or 8, 16, 32, 64 rows (k, v: a chunk's span, rounded up
+// slice) by kPsQ rows (q) or 8, 16, 32, 64 rows (k, v: a chunk's span, rounded up
 // to 8 rows, is the sum of at most four of them).  No swizzle: the consumers read
 // whole 512-byte rows, 16 bytes a lane.
 struct PatchMaps {
